@@ -1,0 +1,364 @@
+#!/usr/bin/env python
+"""CSA decode benchmark: steps/s of (index score -> top-k -> sparse MQA
+attention) over a stack of CSA layers, on synthetic inputs shaped like the
+64K-context decode workload (21 CSA layers, batch 1, N = 16384 compressed
+entries per layer, 64 heads, top-512, 128-row window, bf16).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl lidx|reference]
+                    [--workload decode-64k|decode-128k-b32|decode-500k-b4]
+
+Prints one JSON line (rank 0).  With --gpus N > 1 under torchrun every rank
+runs an independent replica of the workload on its own GPU (the path does not
+shard); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "CSA decode steps/s (score+top-k+sparse attn) at 64K; HBM GB/s vs peak"
+UNIT = "steps/s"
+
+WORKLOADS = {
+    "decode-64k": synth.C2,
+    "decode-128k-b32": synth.C3,
+    "decode-500k-b4": synth.C4,
+}
+
+KEY_ROW_BYTES = {"f32": 512, "bf16": 256, "e4m3": 64 + 1 + 128}
+KV_ROW_BYTES = {"f32": 2048, "bf16": 1024, "e4m3": 448 + 7 + 128}
+Q_BYTES = {"f32": 4, "bf16": 2}
+
+
+def algorithmic_bytes(spec) -> dict:
+    """Inputs read once and outputs written once (intermediates excluded)."""
+    B, N, H, k = spec.B, spec.N, spec.H, spec.k
+    keys = B * N * KEY_ROW_BYTES[spec.key_dtype]
+    q_idx = B * H * 128 * Q_BYTES[spec.q_dtype]
+    w = B * H * 4
+    rows = B * k * KV_ROW_BYTES[spec.kv_dtype]
+    swa = B * spec.swa * KV_ROW_BYTES[spec.kv_dtype]
+    q_attn = B * H * 512 * Q_BYTES[spec.q_dtype]
+    out = B * H * 512 * 4
+    layer = keys + q_idx + w + rows + swa + q_attn + out
+    # the scoring kernel itself also writes its fp32 scores
+    score_launch = keys + q_idx + w + B * N * 4
+    return dict(layer=layer, step=layer * spec.layers, score_launch=score_launch)
+
+
+def peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm_gbs=float(d["hbm_gbs"]), source="measured")
+    return dict(hbm_gbs=6650.0, source="fallback")
+
+
+def scorer_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "lightning_indexer_top_index_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.startswith("score") or f in ("common.cuh", "kernels.cuh", "tc.cuh"):
+            h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per scorer launch from the committed ncu summary, if it was
+    taken on the current scorer source; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p)).get(workload)
+    if not d or d.get("source_hash") != scorer_source_hash():
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+# --------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.gpu), "-lms", "200"], stdout=self.f,
+                                         stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ the arms
+def oracle_layer_time(spec, layers) -> tuple:
+    """Time the oracle (score, top-k, attention of every sequence) on the given
+    layers' inputs; returns (seconds, layers done)."""
+    import oracle
+    t0 = time.perf_counter()
+    for inp in layers:
+        for b in range(spec.B):
+            N = spec.N
+            s = oracle.index_score(inp["q_idx"][b].reshape(1, 1, spec.H, 128), inp["w"][b],
+                                   inp["keys"].slice(b * N, (b + 1) * N), 1, 1, spec.H, N)
+            ids, n, _ = oracle.topk(s[0, 0], spec.k)
+            oracle.attn(inp["q_attn"][b], inp["kv"].slice(b * N, (b + 1) * N), N, ids[:n],
+                        swa=inp["swa"].slice(b * spec.swa, (b + 1) * spec.swa), swa_len=spec.swa, scale=spec.scale)
+    return time.perf_counter() - t0, len(layers)
+
+
+def run_reference(args, spec, cfg):
+    """The oracle arm: each step is one layer of the workload on the host."""
+    layers = [synth.decode_layer(spec, l % spec.layers) for l in range(min(spec.layers, 2))]
+    for i in range(args.warmup):
+        oracle_layer_time(spec, [layers[i % len(layers)]])
+    t, n = 0.0, 0
+    for i in range(args.steps):
+        dt, dn = oracle_layer_time(spec, [layers[i % len(layers)]])
+        t += dt
+        n += dn
+    step_s = t / n * spec.layers
+    v = 1.0 / step_s
+    sample = f"{n} single-layer samples of the {spec.layers}-layer step; steps/s = 1/(mean layer time x {spec.layers})"
+    line = {"metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": cfg, "impl": "reference",
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def make_replica_steps(spec, layers_inp, R, device):
+    import torch
+    import lightning_indexer_top_index_b200 as L
+    from lightning_indexer_top_index_b200.decode import DecodeStep, LayerCache
+
+    base = []
+    for inp in layers_inp:
+        base.append(LayerCache(
+            L.DeviceKV.from_arrays(spec.key_dtype, 128, inp["keys"].data, inp["keys"].scale, inp["keys"].rope,
+                                   batch_rows=spec.N, device=device),
+            L.DeviceKV.from_arrays(spec.kv_dtype, 512, inp["kv"].data, inp["kv"].scale, inp["kv"].rope,
+                                   batch_rows=spec.N, device=device),
+            L.DeviceKV.from_arrays(spec.kv_dtype, 512, inp["swa"].data, inp["swa"].scale, inp["swa"].rope,
+                                   batch_rows=spec.swa, device=device)))
+
+    def clone(kv):
+        return L.DeviceKV(kv.dtype, kv.dim, kv.data.clone(), None if kv.scale is None else kv.scale.clone(),
+                          None if kv.rope is None else kv.rope.clone(), kv.batch_rows)
+
+    qdt = torch.bfloat16 if spec.q_dtype == "bf16" else torch.float32
+    steps = []
+    for r in range(R):
+        caches = base if r == 0 else [LayerCache(clone(c.keys), clone(c.kv), clone(c.swa)) for c in base]
+        steps.append(DecodeStep(caches, spec.B, spec.H, spec.N, spec.k, spec.swa, spec.scale, q_dtype=qdt,
+                                device=device))
+    return steps
+
+
+def host_queries(spec, layers_inp):
+    """Per-step inputs on the host: q_idx [L][B][1][H][128], w [L][B][1][H], q_attn [L][B][H][512]."""
+    import torch
+
+    def t(x, dt):
+        a = torch.from_numpy(np.ascontiguousarray(x))
+        return a.view(torch.int16).view(torch.bfloat16) if dt == "bf16" else a
+
+    q_idx = torch.stack([t(i["q_idx"], spec.q_dtype) for i in layers_inp]).reshape(spec.layers, spec.B, 1, spec.H, 128)
+    w = torch.stack([torch.from_numpy(i["w"]) for i in layers_inp]).reshape(spec.layers, spec.B, 1, spec.H)
+    q_attn = torch.stack([t(i["q_attn"], spec.q_dtype) for i in layers_inp])
+    return q_idx, w, q_attn
+
+
+def run_lidx(args, spec, cfg, rank, world, local_rank):
+    import torch
+    import lightning_indexer_top_index_b200 as L  # noqa: F401
+
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+
+    layers_inp = [synth.decode_layer(spec, l) for l in range(spec.layers)]
+    ab = algorithmic_bytes(spec)
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    R = max(2, math.ceil(4 * l2 / ab["step"]))
+    steps = make_replica_steps(spec, layers_inp, R, device)
+    q_idx_h, w_h, q_attn_h = host_queries(spec, layers_inp)
+    for s in steps:
+        s.set_inputs(q_idx_h.to(device), w_h.to(device), q_attn_h.to(device))
+        s.capture()
+    torch.cuda.synchronize()
+
+    # ---- device-timed steps (inputs resident)
+    for i in range(args.warmup):
+        steps[i % R].replay()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(args.steps):
+        steps[i % R].replay()
+    e1.record()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    if dist:
+        t = torch.tensor([ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+        dist.barrier()
+
+    # ---- live scorer timing: the same step with external events around each scoring launch
+    inst = steps[0]
+    events = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
+              for _ in range(spec.layers)]
+    g_inst = inst.capture(events)
+    durs = []
+    for i in range(max(3, min(args.steps, 20))):
+        for r in range(1, R):
+            steps[r].replay()  # evict the instrumented replica's keys from L2 between its replays
+        g_inst.replay()
+        torch.cuda.synchronize()
+        durs += [a.elapsed_time(b) for a, b in events]
+    score_ms = statistics.mean(durs)
+
+    # ---- end to end: pinned host queries in, attention outputs back, every step
+    q_idx_p, w_p, q_attn_p = q_idx_h.pin_memory(), w_h.pin_memory(), q_attn_h.pin_memory()
+    out_p = torch.empty(steps[0].out.shape, dtype=torch.float32).pin_memory()
+    for i in range(args.warmup):
+        s = steps[i % R]
+        s.set_inputs(q_idx_p, w_p, q_attn_p)
+        s.replay()
+        out_p.copy_(s.out, non_blocking=True)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record()
+    for i in range(args.steps):
+        s = steps[i % R]
+        s.set_inputs(q_idx_p, w_p, q_attn_p)
+        s.replay()
+        out_p.copy_(s.out, non_blocking=True)
+    f1.record()
+    torch.cuda.synchronize()
+    e2e_ms = f0.elapsed_time(f1) / args.steps
+    if dist:
+        t = torch.tensor([e2e_ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    h2d = sum(x.numel() * x.element_size() for x in (q_idx_p, w_p, q_attn_p))
+    d2h = out_p.numel() * out_p.element_size()
+
+    if rank == 0:
+        pk = peaks()
+        achieved = ab["score_launch"] / (score_ms * 1e-3) / 1e9
+        line = {
+            "metric": METRIC, "value": world * 1e3 / ms, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16" if spec.key_dtype == "bf16" else spec.key_dtype,
+            "data": "synthetic", "config": cfg,
+            "hbm_gbs_step": ab["step"] / (ms * 1e-3) / 1e9,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / pk["hbm_gbs"], "traffic": profiled_traffic(args.workload),
+                         "kernel": "lidx_index_score", "peak_source": pk["source"],
+                         "bytes_per_launch": ab["score_launch"], "avg_launch_us": score_ms * 1e3},
+            "e2e": {"value": world * 1e3 / e2e_ms, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": args.steps * steps[0].kernel_launches(),
+            "clocks": clk,
+        }
+        if world == 1:
+            sample_layers = layers_inp[:2]
+            t, n = oracle_layer_time(spec, sample_layers)
+            v = 1.0 / (t / n * spec.layers)
+            line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
+                                    "sample": f"{n} of the {spec.layers} layers of one step on the host, "
+                                              f"single thread; scaled by {spec.layers}/{n}"}
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="lidx", choices=["lidx", "reference"])
+    ap.add_argument("--workload", default="decode-64k", choices=sorted(WORKLOADS))
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    spec = WORKLOADS[args.workload]
+    ab = algorithmic_bytes(spec)
+    cfg = {"workload": spec.name, "layers": spec.layers, "batch": spec.B, "entries": spec.N, "heads": spec.H,
+           "top_k": spec.k, "swa": spec.swa, "key_format": spec.key_dtype, "kv_format": spec.kv_dtype,
+           "algorithmic_bytes_per_step": ab["step"],
+           "l2": "inputs larger than L2: rotating cache replicas, >= 4x L2 of step bytes",
+           "parallelism": f"replicas x{world}"}
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args, spec, cfg)
+        return
+    run_lidx(args, spec, cfg, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,287 @@
+/*
+ * lidx -- lightning indexer, top-k selection and sparse MQA decode for
+ * NVIDIA B200 (sm_100a).  C ABI of liblidx.so.
+ *
+ * The path (DeepSeek-V4-Flash architecture post, "Part 6", section (B)):
+ * in every CSA layer the lightning indexer scores each 4:1-compressed entry
+ * with its own 128-d index key (index_comp_kv), keeps the top 512 entries
+ * (n_indexer_top_k; 1024 for the Pro variant), and attention reads the
+ * selected 512-wide rows (attn_comp_kv, section (A)) plus a 128-row sliding
+ * window.  The evaluation side (FlashMemory-vs-native post, Act 3; FlashMemory
+ * deep-dive write-up, sections 2.2, 3.2 and 4.1) builds golden labels from
+ * dense attention (softmax, top-p 0.6, >= 3-of-21 layer vote), applies the
+ * memory-indexer gate (sigmoid >= 0.5, OR over layers 10/12/20) and measures
+ * set overlap.
+ *
+ * Conventions for every call:
+ *  - All pointers in the argument structs are DEVICE pointers unless noted.
+ *    The caller owns all memory; the library allocates and frees nothing.
+ *    Scratch memory is a caller-provided workspace whose size
+ *    lidx_workspace_size() reports; it must be 256-byte aligned.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Calls only enqueue work on it: no host synchronisation.
+ *  - Synchronous argument errors are returned as lidx_status before anything
+ *    is enqueued.  Data-dependent problems found on the device (an id outside
+ *    [0, N), a NaN score, a device wait that gave up) are OR-ed as bit flags
+ *    into a status word at the start of the workspace; read it with
+ *    lidx_read_device_status().  The kernels never trap.
+ *  - The library keeps no mutable global state besides cached device
+ *    properties, so concurrent calls on different streams with different
+ *    workspaces are safe.
+ */
+#ifndef LIDX_H
+#define LIDX_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define LIDX_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define LIDX_API __attribute__((visibility("default")))
+#else
+#define LIDX_API
+#endif
+
+typedef enum lidx_status {
+    LIDX_OK = 0,
+    LIDX_ERR_INVALID_ARG = 1, /* null pointer, bad size, misaligned buffer */
+    LIDX_ERR_UNSUPPORTED = 2, /* format/shape not implemented (e.g. f16 comp KV), or not sm_100 */
+    LIDX_ERR_CUDA = 3,        /* a CUDA runtime call failed */
+    LIDX_ERR_WORKSPACE = 4    /* workspace missing or smaller than lidx_workspace_size() */
+} lidx_status;
+
+/* Bit flags of the device status word (asynchronous). */
+#define LIDX_DEV_BOUNDS 0x1u  /* an id outside [0, N) was skipped */
+#define LIDX_DEV_NAN 0x2u     /* a NaN score / negative or NaN probability was excluded */
+#define LIDX_DEV_TIMEOUT 0x4u /* a bounded device wait gave up */
+
+/* Storage formats. */
+#define LIDX_F32 0
+#define LIDX_BF16 1
+#define LIDX_E4M3 2 /* OCP E4M3FN non-RoPE dims + E8M0 scale per 64 + bf16 RoPE dims */
+#define LIDX_F16 3  /* recognised and refused (LIDX_ERR_UNSUPPORTED), as the ds4 CUDA path refuses f16 comp KV */
+
+/*
+ * Rows of a cache (index keys, compressed KV or sliding-window rows).
+ *
+ * Logical row (width `dim`): for LIDX_F32 / LIDX_BF16 the `dim` stored
+ * values.  For LIDX_E4M3 (architecture post, "why quantising the KV does not
+ * save memory"): dims [0, dim-64) are E4M3 codes in `data`, scaled by
+ * 2^(e-127) where e is the E8M0 byte scale[(d)/64] of the row; dims
+ * [dim-64, dim) are the bf16 RoPE dims in `rope`.
+ *
+ * Row j of batch entry b is row b*batch_rows + j of every plane; row r of a
+ * plane starts at plane + r*ld (ld in elements of that plane).  Planes must
+ * be 16-byte aligned and ld*elem_size a multiple of 16 (scale plane: any ld).
+ */
+typedef struct lidx_kv {
+    int32_t dtype;        /* LIDX_F32 | LIDX_BF16 | LIDX_E4M3 */
+    int32_t dim;          /* 128 for index keys, 512 for attention rows */
+    const void *data;     /* F32: float, BF16: bf16, E4M3: uint8 codes */
+    const uint8_t *scale; /* E4M3 only: E8M0 codes, (dim-64)/64 per row */
+    const void *rope;     /* E4M3 only: bf16, 64 per row */
+    int64_t ld;           /* elements between rows of `data` */
+    int64_t ld_scale;     /* bytes between rows of `scale` */
+    int64_t ld_rope;      /* elements between rows of `rope` */
+    int64_t batch_rows;   /* rows between consecutive batch entries (>= N) */
+} lidx_kv;
+
+/* ------------------------------------------------------------------------
+ * lidx_index_score -- lightning indexer scores.
+ *
+ *   scores[b,t,j] = sum_h w[b,t,h] * max(q[b,t,h,:] . keys[b,j,:], 0)
+ *
+ * (head-weighted ReLU of MQA dot products; the ReLU-MQA indexer of the
+ * FlashMemory deep-dive write-up, reply #2, with the head weights applied
+ * outside the ReLU).  Accumulation is fp32.
+ *
+ *   q       [B][Q][H][128], q_dtype LIDX_F32 (with F32 keys) or LIDX_BF16
+ *           (with BF16 or E4M3 keys)
+ *   w       [B][Q][H] fp32 (any sign)
+ *   keys    dim 128
+ *   scores  [B][Q][ld_scores] fp32, ld_scores >= N; entries j >= N untouched
+ * Returns INVALID_ARG for null pointers / non-positive sizes / misaligned
+ * planes, UNSUPPORTED for other format combinations.
+ * ------------------------------------------------------------------------ */
+typedef struct lidx_score_args {
+    int32_t B, Q, H, N;
+    int32_t q_dtype;
+    const void *q;
+    const float *w;
+    lidx_kv keys;
+    float *scores;
+    int64_t ld_scores;
+} lidx_score_args;
+
+LIDX_API lidx_status lidx_index_score(const lidx_score_args *args, void *stream);
+
+/* ------------------------------------------------------------------------
+ * lidx_topk_select -- top-k row ids (architecture post, section (B):
+ * n_indexer_top_k, and the comp_allowed row set).
+ *
+ * For each (b,t): the k largest scores[b,t,0..N) among entries with
+ * allowed[b][j] != 0 (all entries when allowed is NULL).  Equal scores
+ * (+0 and -0 included) are ranked by index, lower first; NaN scores are
+ * never selected and set LIDX_DEV_NAN.
+ *
+ *   ids     [B][Q][k] int32: selected indices in ascending order, then -1
+ *   n_sel   [B][Q] int32 (optional): min(k, #eligible)
+ *   mask    [B][Q][N] uint8 (optional): 1 for selected entries (comp_allowed)
+ *   mask_bits [B][Q][ceil(N/32)] uint32 (optional): bit j%32 of word j/32
+ * Needs a workspace of lidx_workspace_size(LIDX_OP_TOPK).
+ * ------------------------------------------------------------------------ */
+typedef struct lidx_topk_args {
+    int32_t B, Q, N, k;
+    const float *scores;
+    int64_t ld_scores;
+    const uint8_t *allowed; /* optional [B][ld_allowed], shared by the Q queries */
+    int64_t ld_allowed;
+    int32_t *ids;
+    int32_t *n_sel;
+    uint8_t *mask;
+    uint32_t *mask_bits;
+} lidx_topk_args;
+
+LIDX_API lidx_status lidx_topk_select(const lidx_topk_args *args, void *ws, size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------------------
+ * lidx_sparse_attn_decode -- MQA attention of one decode token over the
+ * selected compressed rows plus the sliding window (architecture post,
+ * sections (A)-(B)).  K = V = the full 512-wide row.
+ *
+ *   R_b  = { kv row ids[b][i] : i < n_b, ids[b][i] >= 0 } U { swa rows 0..swa_len-1 }
+ *          with n_b = n_sel[b] if n_sel is given, else n_ids
+ *   out[b,h,:] = sum_{r in R_b} softmax_r(scale * q[b,h,:] . x_r) x_r
+ *   lse[b,h]   = log sum_{r in R_b} exp(scale * q[b,h,:] . x_r)   (optional)
+ *
+ *   q     [B][H][512], LIDX_F32 (with F32 rows) or LIDX_BF16
+ *   kv    comp_kv rows, dim 512, N entries per sequence
+ *   ids   [B][ld_ids] int32 (ascending not required; duplicates count twice)
+ *   swa   sliding-window rows, dim 512, same dtype as kv (swa_len may be 0)
+ *   out   [B][H][512] fp32
+ * Ids outside [-1, N) are skipped and set LIDX_DEV_BOUNDS.  Empty R gives
+ * out = 0 and lse = -inf.  Needs lidx_workspace_size(LIDX_OP_ATTN) bytes
+ * (split-K partial results).
+ * ------------------------------------------------------------------------ */
+typedef struct lidx_attn_args {
+    int32_t B, H;
+    int32_t q_dtype;
+    const void *q;
+    lidx_kv kv;
+    int32_t N;
+    const int32_t *ids;
+    int32_t n_ids;
+    int64_t ld_ids;
+    const int32_t *n_sel;
+    lidx_kv swa;
+    int32_t swa_len;
+    float scale;
+    float *out;
+    float *lse;
+} lidx_attn_args;
+
+LIDX_API lidx_status lidx_sparse_attn_decode(const lidx_attn_args *args, void *ws, size_t ws_bytes,
+                                    void *stream);
+
+/* ------------------------------------------------------------------------
+ * lidx_selection_eval -- selection evaluation over a tau-window.
+ * `ops` is a bit mask; the requested steps run in this order:
+ *
+ *  LIDX_EVAL_GOLDEN  (FlashMemory-vs-native post, Act 3; write-up 3.2 step 1)
+ *     probs[l][t][j] = (1/H) sum_h softmax_j(scale * qa[l][t][h] . kv_l[j])
+ *     over the N entries of layer l (kv rows l*kv.batch_rows + j).
+ *  LIDX_EVAL_TOPP    (write-up 3.2 step 2)
+ *     per row (l,t): with m_j = floor(probs_j * 2^40) and M = sum m_j, the
+ *     shortest prefix of the ranking (probs descending, ties to the lower
+ *     index) whose mass reaches ceil(M * top_p_num / top_p_den)
+ *     -> topp_bits[l][t][W].
+ *  LIDX_EVAL_VOTE    (write-up 3.2 step 3)
+ *     vote_bits[t] = { j : #{l : j in topp_bits[l][t]} >= min_votes },
+ *     window_bits = union over t of vote_bits[t].
+ *  LIDX_EVAL_LSA     (write-up sections 2.2 and 4.1)
+ *     fetched_bits = { j : exists g, gate_logits[g][j] + gate_bias >= 0 }
+ *     (sigmoid(z) >= 0.5 <=> z >= 0; the sum is rounded to fp32).
+ *  LIDX_EVAL_OVERLAP (FlashMemory-vs-native post, Acts 1 and 3)
+ *     counts[p] = { |A_p & B_p|, |A_p|, |B_p| } with A_p = set_a + p*ld_a,
+ *     B_p = set_b + p*ld_b (ld 0 reuses one set for all pairs).
+ *
+ * Bit sets are uint32 [.][W], W = ceil(N/32), bit j%32 of word j/32; bits at
+ * and beyond N are written as 0 and must be 0 on input.  Inputs of a step
+ * may be the outputs of an earlier step in the same call.
+ * Needs lidx_workspace_size(LIDX_OP_EVAL) bytes.
+ * ------------------------------------------------------------------------ */
+#define LIDX_EVAL_GOLDEN 0x1u
+#define LIDX_EVAL_TOPP 0x2u
+#define LIDX_EVAL_VOTE 0x4u
+#define LIDX_EVAL_LSA 0x8u
+#define LIDX_EVAL_OVERLAP 0x10u
+
+typedef struct lidx_eval_args {
+    uint32_t ops;
+    int32_t L, T, H, N;
+    /* GOLDEN */
+    int32_t qa_dtype;      /* LIDX_BF16 (LIDX_F32 with F32 rows) */
+    const void *qa;        /* [L][T][H][512] */
+    lidx_kv kv;            /* dim 512 */
+    float scale;
+    float *probs;          /* [L][T][N]: GOLDEN output, TOPP input */
+    /* TOPP */
+    uint32_t top_p_num, top_p_den;
+    uint32_t *topp_bits;   /* [L][T][W]: TOPP output, VOTE input */
+    /* VOTE */
+    int32_t min_votes;
+    uint32_t *vote_bits;   /* [T][W] (optional) */
+    uint32_t *window_bits; /* [W] */
+    /* LSA */
+    int32_t n_gate;
+    const float *gate_logits; /* [n_gate][N] */
+    float gate_bias;
+    uint32_t *fetched_bits;   /* [W] */
+    /* OVERLAP */
+    int32_t n_pairs;
+    const uint32_t *set_a;
+    int64_t ld_a;
+    const uint32_t *set_b;
+    int64_t ld_b;
+    int64_t *counts;          /* [n_pairs][3] */
+} lidx_eval_args;
+
+LIDX_API lidx_status lidx_selection_eval(const lidx_eval_args *args, void *ws, size_t ws_bytes,
+                                void *stream);
+
+/* ------------------------------------------------------------------------
+ * Workspace sizes, status, introspection.
+ * ------------------------------------------------------------------------ */
+#define LIDX_OP_SCORE 0
+#define LIDX_OP_TOPK 1
+#define LIDX_OP_ATTN 2
+#define LIDX_OP_EVAL 3
+
+/* Bytes of workspace call `op` needs for `args` (a pointer to the matching
+ * *_args struct, host memory).  Score needs none (0). */
+LIDX_API lidx_status lidx_workspace_size(int op, const void *args, size_t *bytes);
+
+/* Synchronises `stream`, copies the status word at the start of `ws` into
+ * *status (host) and clears it on the device. */
+LIDX_API lidx_status lidx_read_device_status(void *ws, uint32_t *status, void *stream);
+
+/* Static description of a status code. */
+LIDX_API const char *lidx_status_string(lidx_status s);
+
+/* LIDX_ABI_VERSION of the loaded library. */
+LIDX_API int lidx_abi_version(void);
+
+/* sizeof() of the argument structs as compiled into the library, for binding
+ * checks: which = 0 lidx_kv, 1 score, 2 topk, 3 attn, 4 eval. */
+LIDX_API size_t lidx_struct_size(int which);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LIDX_H */

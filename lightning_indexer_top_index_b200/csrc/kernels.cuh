@@ -1,0 +1,35 @@
+// Internal launchers of the lidx kernels.  Every launcher only enqueues work
+// on `st` and returns the launch error; arguments were validated by the C-ABI
+// layer (lidx_api.cu).
+#pragma once
+
+#include "common.cuh"
+
+namespace lidx {
+
+// Scratch layout inside a caller workspace: a 256-byte header whose first
+// word is the device status word, then the op's own region.
+struct WsHeader {
+  uint32_t status;
+  uint32_t pad[63];
+};
+
+// ---- index score
+cudaError_t launch_score_cc(const lidx_score_args &a, cudaStream_t st);
+// tcgen05 scorer; returns cudaErrorNotSupported when the shape is not covered.
+cudaError_t launch_score_tc(const lidx_score_args &a, cudaStream_t st);
+bool score_tc_supported(const lidx_score_args &a);
+
+// ---- top-k
+size_t topk_workspace(const lidx_topk_args &a);
+cudaError_t launch_topk(const lidx_topk_args &a, void *ws, cudaStream_t st);
+
+// ---- sparse attention decode
+size_t attn_workspace(const lidx_attn_args &a);
+cudaError_t launch_attn(const lidx_attn_args &a, void *ws, cudaStream_t st);
+
+// ---- selection evaluation
+size_t eval_workspace(const lidx_eval_args &a);
+cudaError_t launch_eval(const lidx_eval_args &a, void *ws, cudaStream_t st);
+
+}  // namespace lidx

@@ -1,0 +1,76 @@
+"""Shared helpers of the GPU parity tests: move synthetic inputs to the device
+and apply the parity rules.
+
+Tolerances (derived in the design doc from fp32 accumulation):
+  scores     |g - o| <= 1e-5 |o| + 1e-6 * sum_h |w_h| sum_d |q_hd k_jd|
+  attention  max_d |g - o| / max_d |o| <= 2e-3 per (b, h)
+  sets       bit-exact on identical inputs; end to end, differences only for
+             entries tied with the k-th score within 1e-6 relative
+"""
+import numpy as np
+import torch
+
+import lightning_indexer_top_index_b200 as L
+
+SCORE_RTOL = 1e-5
+SCORE_CTOL = 1e-6
+ATTN_TOL = 2e-3
+
+
+def dev_kv(kv, batch_rows=0):
+    """synth.KV -> DeviceKV on cuda:0."""
+    return L.DeviceKV.from_arrays(kv.dtype, kv.dim, kv.data, kv.scale, kv.rope, batch_rows=batch_rows)
+
+
+def dev_q(q, dtype):
+    """float32 array or bf16 bits -> torch tensor on cuda:0."""
+    t = torch.from_numpy(np.ascontiguousarray(q))
+    if dtype == "bf16":
+        t = t.view(torch.int16).view(torch.bfloat16)
+    return t.cuda().contiguous()
+
+
+def assert_scores_close(got, ref, cond):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    err = np.abs(got - ref)
+    bound = SCORE_RTOL * np.abs(ref) + SCORE_CTOL * cond
+    bad = err > bound
+    assert not bad.any(), (f"{bad.sum()} scores outside tolerance; worst err {err.max():.3e} "
+                           f"bound there {bound.ravel()[np.argmax(err)]:.3e}")
+
+
+def assert_attn_close(got, ref):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    num = np.abs(got - ref).max(axis=-1)
+    den = np.maximum(np.abs(ref).max(axis=-1), 1e-30)
+    rel = num / den
+    assert rel.max() <= ATTN_TOL, f"max relative error {rel.max():.3e}"
+    return rel.max()
+
+
+def topk_sets_equivalent(ids_gpu, ids_ref, scores_ref, bound=None, rtol=1e-6):
+    """End-to-end set check: every entry in the symmetric difference must tie
+    with the k-th selected oracle score, within rtol relative plus the score
+    tolerance `bound` (per entry) of both entries."""
+    a = set(int(i) for i in ids_gpu if i >= 0)
+    b = set(int(i) for i in ids_ref if i >= 0)
+    if a == b:
+        return True
+    if len(a) != len(b):
+        return False
+    sel = np.array(sorted(b))
+    jk = sel[np.argmin(scores_ref[sel])]
+    kth = float(scores_ref[jk])
+    for j in a ^ b:
+        slack = rtol * abs(kth)
+        if bound is not None:
+            slack += float(bound[j]) + float(bound[jk])
+        if abs(float(scores_ref[j]) - kth) > slack:
+            return False
+    return True
+
+
+def score_bound(ref, cond):
+    return SCORE_RTOL * np.abs(np.asarray(ref, dtype=np.float64)) + SCORE_CTOL * cond
