@@ -189,6 +189,35 @@ LIDX_API lidx_status lidx_sparse_attn_decode(const lidx_attn_args *args, void *w
                                     void *stream);
 
 /* ------------------------------------------------------------------------
+ * lidx_sparse_attn_decode_noalloc -- lidx_sparse_attn_decode without a
+ * caller workspace.  The pages have no counterpart: this exists for callers
+ * that cannot allocate device memory when they call, such as a plugin hosted
+ * by another runtime that provides no scratch allocator, or a serving loop
+ * that forbids cudaMalloc after start-up (it can synchronise the device and
+ * fragments a fixed memory budget).
+ *
+ * Same arguments and results as lidx_sparse_attn_decode.  The split-K
+ * scratch lives in a device array of LIDX_NOALLOC_SCRATCH_BYTES owned by the
+ * library; every GPU that loads the library holds it until the process exits.
+ * The call allocates nothing.
+ *  - Requests whose workspace (lidx_workspace_size(LIDX_OP_ATTN)) exceeds
+ *    LIDX_NOALLOC_SCRATCH_BYTES are rejected with LIDX_ERR_WORKSPACE before
+ *    anything is enqueued; use lidx_sparse_attn_decode for them.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - All calls share the array and it keeps the last call's contents; the
+ *    call clears the status word itself.  Calls whose work overlaps on the
+ *    GPU (e.g. on two streams) race on the array: serialise them.
+ *  - dev_status (optional, DEVICE pointer): receives this call's device
+ *    status word (LIDX_DEV_* flags) when the call's work completes.
+ * ------------------------------------------------------------------------ */
+#define LIDX_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+LIDX_API lidx_status lidx_sparse_attn_decode_noalloc(const lidx_attn_args *args, uint32_t *dev_status,
+                                                     void *stream);
+
+/* ------------------------------------------------------------------------
  * lidx_selection_eval -- selection evaluation over a tau-window.
  * `ops` is a bit mask; the requested steps run in this order:
  *

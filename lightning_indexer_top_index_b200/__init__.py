@@ -332,3 +332,32 @@ def read_device_status(ws: torch.Tensor, stream=None) -> int:
     _check(lib().lidx_read_device_status(C.c_void_p(ws.data_ptr()), C.byref(s), _stream(stream)),
            "lidx_read_device_status")
     return s.value
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def sparse_attn_decode_noalloc(q: torch.Tensor, kv: DeviceKV, N: int, ids: torch.Tensor, n_sel: torch.Tensor = None,
+                               swa: DeviceKV = None, swa_len: int = 0, scale: float = None, *, out=None, lse=None,
+                               want_lse=True, dev_status: torch.Tensor = None, stream=None):
+    """sparse_attn_decode for callers that cannot allocate device memory when
+    they call (a plugin hosted by a runtime that offers no scratch allocator,
+    a serving loop that forbids cudaMalloc after start-up): the split-K
+    scratch lives in a fixed 16 MiB device array owned by the library, shared
+    by all calls -- calls that overlap on the GPU race on it.  The first call
+    on a device should come before any stream capture.  Requests needing more
+    scratch than the array holds raise LidxError(ERR_WORKSPACE).  `out` and
+    `lse` are allocated here only when not given."""
+    l = lib()
+    f = l.lidx_sparse_attn_decode_noalloc
+    f.restype = C.c_int
+    f.argtypes = [C.POINTER(AttnArgs), C.c_void_p, C.c_void_p]
+    B, H, D = q.shape
+    if scale is None:
+        scale = D ** -0.5
+    out = torch.empty((B, H, D), dtype=torch.float32, device=q.device) if out is None else out
+    if want_lse and lse is None:
+        lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    a = attn_args(q, kv, N, ids, n_sel, swa, swa_len, scale, out, lse)
+    _check(f(C.byref(a), C.c_void_p(_ptr(dev_status)), _stream(stream)), "lidx_sparse_attn_decode_noalloc")
+    return out, lse
