@@ -1,10 +1,416 @@
-// tcgen05 / TMEM lightning-indexer scorer (filled in by the tensor-core path).
+// Lightning-indexer scores on the 5th-generation tensor cores (tcgen05).
+//
+//   s[b,t,j] = sum_h w[b,t,h] * max(q[b,t,h,:] . k[b,j,:], 0)
+//
+// (DeepSeek-V4-Flash architecture post, section (B); head-weighted ReLU-MQA
+// of the FlashMemory deep-dive write-up, reply #2.)
+//
+// Layout: keys on the MMA's M side (128 entries per tile), query heads on N
+// (QG queries x H heads, <= 256 columns).  One work unit is (sequence b,
+// query group g, key tile t); each CTA walks a contiguous range of units.
+//   warp 0      TMA producer: the query tile of (b,g) once, then key tiles
+//               through a kStages-deep ring of shared-memory stages
+//   warp 1      allocates TMEM; one lane issues the MMAs (K = 128 in steps of
+//               16) into one of two TMEM accumulators and commits
+//   warps 2-5   epilogue: each thread owns one key row (its TMEM lane), loads
+//               the H head dots of each query and reduces sum_h w_h max(x,0)
+//               in registers; 128 consecutive scores per query are stored
+//   warps 6-9   (E4M3 keys only) convert the FP8 non-RoPE half of each key
+//               tile to bf16 in the 128-byte-swizzled layout the MMA reads;
+//               the RoPE half arrives by TMA directly.  The power-of-two
+//               block scale is applied in the epilogue to a separate
+//               accumulator, so the FP8 path is exact.
+// One query group per (b,g): for decode (Q = 1) the query tile stays resident
+// and the kernel streams the keys once at HBM speed; for many queries
+// (prefill / evaluation) each key tile is reused by QG queries per MMA.
 #include "kernels.cuh"
+#include "tc.cuh"
 
 namespace lidx {
 
-bool score_tc_supported(const lidx_score_args &) { return false; }
+namespace {
 
-cudaError_t launch_score_tc(const lidx_score_args &, cudaStream_t) { return cudaErrorNotSupported; }
+constexpr int kStages = 4;
+constexpr int kTileM = 128;
+constexpr int kTileBytes = kTileM * 128 * 2;  // bf16 [128][128] as two 64-wide swizzled panels
+constexpr int kPanelBytes = kTileBytes / 2;
+constexpr int kF8Bytes = kTileM * 64;         // raw E4M3 half-tile
+
+struct TcParams {
+  int B, Q, H, N;
+  int QG, n_groups, n_tiles;
+  int NM;             // MMA N = QG*H
+  int cols_per_acc;   // TMEM columns per accumulator
+  uint32_t tmem_cols;
+  long long units;
+  int64_t key_batch_rows;
+  float *scores;
+  int64_t ld_scores;
+  const float *w;
+  const uint8_t *scale;
+  int64_t ld_scale;
+  uint32_t *status;
+};
+
+struct __align__(8) TcBarriers {
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+  uint64_t conv[kStages];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t bfull;
+  uint64_t bempty;
+  uint32_t tmem_base;
+  uint32_t abort;
+};
+
+__host__ __device__ constexpr size_t tc_smem_bytes(int NM, bool fp8) {
+  return 1024 + static_cast<size_t>(kStages) * kTileBytes + 2ull * NM * 128 + (fp8 ? kStages * kF8Bytes : 0) +
+         256 * sizeof(float) + sizeof(TcBarriers);
+}
+
+__device__ __forceinline__ void unit_coords(const TcParams &p, long long u, int &b, int &g, int &t, long long &bg) {
+  bg = u / p.n_tiles;
+  t = static_cast<int>(u % p.n_tiles);
+  b = static_cast<int>(bg / p.n_groups);
+  g = static_cast<int>(bg % p.n_groups);
+}
+
+__device__ __forceinline__ void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n)); }
+
+template <bool kFp8>
+__global__ void __launch_bounds__(kFp8 ? 320 : 192, 1)
+    score_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_rope,
+                    const __grid_constant__ CUtensorMap tm_q, const TcParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *sA = smem;
+  uint8_t *sB = sA + kStages * kTileBytes;
+  uint8_t *sF8 = sB + 2 * p.NM * 128;
+  float *sW = reinterpret_cast<float *>(sF8 + (kFp8 ? kStages * kF8Bytes : 0));
+  TcBarriers *bar = reinterpret_cast<TcBarriers *>(sW + 256);
+  volatile uint32_t *abort_flag = &bar->abort;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long u0 = blockIdx.x * p.units / gridDim.x, u1 = (blockIdx.x + 1) * p.units / gridDim.x;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; s++) {
+      tc::mbar_init(&bar->full[s], 1);
+      tc::mbar_init(&bar->empty[s], 1);
+      tc::mbar_init(&bar->conv[s], 128);
+    }
+    for (int a = 0; a < 2; a++) {
+      tc::mbar_init(&bar->tfull[a], 1);
+      tc::mbar_init(&bar->tempty[a], 4);
+    }
+    tc::mbar_init(&bar->bfull, 1);
+    tc::mbar_init(&bar->bempty, 1);
+    bar->abort = 0;
+    tc::fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tc::tma_prefetch_desc(&tm_a);
+    tc::tma_prefetch_desc(&tm_q);
+    if (kFp8) tc::tma_prefetch_desc(&tm_rope);
+  }
+  if (warp == 1) tc::tmem_alloc(&bar->tmem_base, p.tmem_cols);
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = bar->tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, bempty_par = 0;
+      uint32_t last_par[kStages];
+      bool used[kStages] = {};
+      bool b_loaded = false;
+      uint32_t bfull_last = 0;
+      long long prev_bg = -1;
+      for (long long u = u0; u < u1; u++) {
+        int b, g, t;
+        long long bg;
+        unit_coords(p, u, b, g, t, bg);
+        if (bg != prev_bg) {
+          if (prev_bg != -1) {
+            if (!tc::mbar_wait(&bar->bempty, bempty_par, abort_flag)) break;
+            bempty_par ^= 1;
+            bfull_last ^= 1;
+          }
+          const int qrow = (b * p.Q + g * p.QG) * p.H;
+          tc::mbar_arrive_expect_tx(&bar->bfull, 2 * p.NM * 128);
+          tc::tma_load_2d(sB, &tm_q, &bar->bfull, 0, qrow);
+          tc::tma_load_2d(sB + p.NM * 128, &tm_q, &bar->bfull, 64, qrow);
+          b_loaded = true;
+          prev_bg = bg;
+        }
+        if (!tc::mbar_wait(&bar->empty[stage], phase ^ 1, abort_flag)) break;
+        const int row = static_cast<int>(b * p.key_batch_rows + static_cast<int64_t>(t) * kTileM);
+        uint8_t *a = sA + stage * kTileBytes;
+        if (kFp8) {
+          tc::mbar_arrive_expect_tx(&bar->full[stage], kF8Bytes + kPanelBytes);
+          tc::tma_load_2d(sF8 + stage * kF8Bytes, &tm_a, &bar->full[stage], 0, row);
+          tc::tma_load_2d(a + kPanelBytes, &tm_rope, &bar->full[stage], 0, row);
+        } else {
+          tc::mbar_arrive_expect_tx(&bar->full[stage], kTileBytes);
+          tc::tma_load_2d(a, &tm_a, &bar->full[stage], 0, row);
+          tc::tma_load_2d(a + kPanelBytes, &tm_a, &bar->full[stage], 64, row);
+        }
+        last_par[stage] = phase;
+        used[stage] = true;
+        if (++stage == kStages) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      // never leave with copies in flight: wait (bounded) for every issued load
+      volatile uint32_t no_abort = 0;
+      for (int s = 0; s < kStages; s++)
+        if (used[s]) tc::mbar_wait(&bar->full[s], last_par[s], &no_abort);
+      if (b_loaded) tc::mbar_wait(&bar->bfull, bfull_last, &no_abort);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_par = 0, bfull_par = 0;
+      long long prev_bg = -1;
+      const uint32_t idesc = tc::idesc_bf16(kTileM, kFp8 ? p.H : p.NM);
+      const uint32_t a_base = tc::smem_u32(sA), b_base = tc::smem_u32(sB);
+      for (long long u = u0; u < u1; u++) {
+        int b, g, t;
+        long long bg;
+        unit_coords(p, u, b, g, t, bg);
+        if (bg != prev_bg) {
+          if (prev_bg != -1) tc::mma_commit(&bar->bempty);
+          if (!tc::mbar_wait(&bar->bfull, bfull_par, abort_flag)) break;
+          bfull_par ^= 1;
+          prev_bg = bg;
+        }
+        if (!tc::mbar_wait(kFp8 ? &bar->conv[stage] : &bar->full[stage], phase, abort_flag)) break;
+        if (!tc::mbar_wait(&bar->tempty[acc], acc_par ^ 1, abort_flag)) break;
+        tc::tc_fence_after();
+        const uint32_t d = tmem + acc * p.cols_per_acc;
+        const uint32_t a = a_base + stage * kTileBytes;
+        if (kFp8) {
+#pragma unroll
+          for (int kk = 0; kk < 4; kk++)
+            tc::mma_bf16(d, tc::desc_kmajor_sw128(a + kk * 32), tc::desc_kmajor_sw128(b_base + kk * 32), idesc, kk > 0);
+#pragma unroll
+          for (int kk = 0; kk < 4; kk++)
+            tc::mma_bf16(d + p.H, tc::desc_kmajor_sw128(a + kPanelBytes + kk * 32),
+                         tc::desc_kmajor_sw128(b_base + p.NM * 128 + kk * 32), idesc, kk > 0);
+        } else {
+#pragma unroll
+          for (int k = 0; k < 8; k++) {
+            const uint32_t ao = (k >> 2) * kPanelBytes + (k & 3) * 32;
+            const uint32_t bo = (k >> 2) * p.NM * 128 + (k & 3) * 32;
+            tc::mma_bf16(d, tc::desc_kmajor_sw128(a + ao), tc::desc_kmajor_sw128(b_base + bo), idesc, k > 0);
+          }
+        }
+        tc::mma_commit(&bar->empty[stage]);
+        tc::mma_commit(&bar->tfull[acc]);
+        if (++stage == kStages) {
+          stage = 0;
+          phase ^= 1;
+        }
+        if (++acc == 2) {
+          acc = 0;
+          acc_par ^= 1;
+        }
+      }
+    }
+  } else if (warp < 6) {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const int etid = threadIdx.x - 64;
+    int acc = 0;
+    uint32_t acc_par = 0;
+    long long prev_bg = -1;
+    for (long long u = u0; u < u1; u++) {
+      int b, g, t;
+      long long bg;
+      unit_coords(p, u, b, g, t, bg);
+      if (bg != prev_bg) {
+        named_sync(2, 128);
+        const int nq = min(p.QG, p.Q - g * p.QG);
+        for (int i = etid; i < p.QG * p.H; i += 128)
+          sW[i] = (i / p.H) < nq ? p.w[static_cast<int64_t>(b * p.Q + g * p.QG) * p.H + i] : 0.f;
+        named_sync(2, 128);
+        prev_bg = bg;
+      }
+      // lane 0 waits, the warp follows its verdict; after a give-up the
+      // warp keeps walking the units (skipping the work) so the named
+      // barriers above stay matched
+      bool ready = false;
+      if (lane == 0) ready = tc::mbar_wait(&bar->tfull[acc], acc_par, abort_flag);
+      ready = __shfl_sync(0xFFFFFFFFu, ready, 0);
+      if (ready) {
+        tc::tc_fence_after();
+        const uint32_t base = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + acc * p.cols_per_acc;
+        const int j = t * kTileM + row;
+        float v[32], r[32];
+        if (kFp8) {
+          float sc = 0.f;
+          if (j < p.N) sc = e8m0_to_f32(p.scale[(b * p.key_batch_rows + j) * p.ld_scale]);
+          float s = 0.f;
+          for (int c0 = 0; c0 < p.H; c0 += 32) {
+            tc::tmem_ld32(base + c0, v);
+            tc::tmem_ld32(base + p.H + c0, r);
+#pragma unroll
+            for (int i = 0; i < 32; i++) s = fmaf(sW[c0 + i], fmaxf(fmaf(sc, v[i], r[i]), 0.f), s);
+          }
+          if (j < p.N) p.scores[static_cast<int64_t>(b * p.Q + g) * p.ld_scores + j] = s;
+        } else {
+          for (int qi = 0; qi < p.QG; qi++) {
+            float s = 0.f;
+            for (int c0 = 0; c0 < p.H; c0 += 32) {
+              tc::tmem_ld32(base + qi * p.H + c0, v);
+#pragma unroll
+              for (int i = 0; i < 32; i++) s = fmaf(sW[qi * p.H + c0 + i], fmaxf(v[i], 0.f), s);
+            }
+            const int qq = g * p.QG + qi;
+            if (j < p.N && qq < p.Q) p.scores[static_cast<int64_t>(b * p.Q + qq) * p.ld_scores + j] = s;
+          }
+        }
+      }
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0 && ready) tc::mbar_arrive(&bar->tempty[acc]);
+      if (++acc == 2) {
+        acc = 0;
+        acc_par ^= 1;
+      }
+    }
+  } else if (kFp8) {
+    // ------------------------------------------------------------ FP8 -> bf16
+    const int r = threadIdx.x - 192;  // tile row
+    int stage = 0;
+    uint32_t phase = 0;
+    for (long long u = u0; u < u1; u++) {
+      if (!tc::mbar_wait(&bar->full[stage], phase, abort_flag)) break;
+      const uint4 *src = reinterpret_cast<const uint4 *>(sF8 + stage * kF8Bytes + r * 64);
+      uint8_t *dst = sA + stage * kTileBytes + r * 128;
+#pragma unroll
+      for (int c = 0; c < 4; c++) {
+        const uint4 x = src[c];
+        const uint32_t wv[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+        for (int h = 0; h < 2; h++) {  // 16 FP8 bytes -> two 16-byte chunks of 8 bf16
+          uint32_t o[4];
+#pragma unroll
+          for (int i = 0; i < 4; i++) {
+            const uint32_t word = wv[h * 2 + i / 2];
+            const uint32_t lo = e4m3_to_bf16_bits((word >> (16 * (i & 1))) & 0xFFu);
+            const uint32_t hi = e4m3_to_bf16_bits((word >> (16 * (i & 1) + 8)) & 0xFFu);
+            o[i] = lo | (hi << 16);
+          }
+          const int chunk = c * 2 + h;
+          *reinterpret_cast<uint4 *>(dst + ((chunk ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+      }
+      tc::fence_proxy_async_smem();
+      tc::mbar_arrive(&bar->conv[stage]);
+      if (++stage == kStages) {
+        stage = 0;
+        phase ^= 1;
+      }
+    }
+  }
+
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, p.tmem_cols);
+  }
+  if (threadIdx.x == 0 && bar->abort) raise_status(p.status, LIDX_DEV_TIMEOUT);
+}
+
+int sm_count() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+int choose_qg(const lidx_score_args &a) {
+  if (a.keys.dtype == LIDX_E4M3) return 1;
+  return std::max(1, std::min(a.Q, 256 / a.H));
+}
+
+}  // namespace
+
+bool score_tc_supported(const lidx_score_args &a) {
+  if (a.q_dtype != LIDX_BF16) return false;
+  if (a.keys.dtype != LIDX_BF16 && a.keys.dtype != LIDX_E4M3) return false;
+  if (a.H % 32 != 0) return false;
+  if (a.keys.dtype == LIDX_E4M3 ? a.H > 128 : a.H > 256) return false;
+  const int64_t rows = static_cast<int64_t>(a.B - 1) * a.keys.batch_rows + a.N;
+  if (rows >= (1ll << 31) || static_cast<int64_t>(a.B) * a.Q * a.H >= (1ll << 31)) return false;
+  return true;
+}
+
+cudaError_t launch_score_tc(const lidx_score_args &a, cudaStream_t st) {
+  const bool fp8 = a.keys.dtype == LIDX_E4M3;
+  TcParams p{};
+  p.B = a.B;
+  p.Q = a.Q;
+  p.H = a.H;
+  p.N = a.N;
+  p.QG = choose_qg(a);
+  p.n_groups = (a.Q + p.QG - 1) / p.QG;
+  p.n_tiles = (a.N + kTileM - 1) / kTileM;
+  p.NM = p.QG * a.H;
+  p.cols_per_acc = fp8 ? 2 * a.H : p.NM;
+  uint32_t cols = 32;
+  while (cols < static_cast<uint32_t>(2 * p.cols_per_acc)) cols <<= 1;
+  p.tmem_cols = cols;
+  p.units = static_cast<long long>(a.B) * p.n_groups * p.n_tiles;
+  p.key_batch_rows = a.B > 1 ? a.keys.batch_rows : a.N;
+  p.scores = a.scores;
+  p.ld_scores = a.ld_scores;
+  p.w = a.w;
+  p.scale = a.keys.scale;
+  p.ld_scale = a.keys.ld_scale;
+  p.status = nullptr;
+
+  const uint64_t rows = static_cast<uint64_t>(a.B - 1) * p.key_batch_rows + a.N;
+  CUtensorMap tm_a, tm_rope, tm_q;
+  bool ok;
+  if (fp8) {
+    ok = make_tmap_2d(&tm_a, a.keys.data, CU_TENSOR_MAP_DATA_TYPE_UINT8, 64, rows, a.keys.ld, 64, kTileM,
+                      CU_TENSOR_MAP_SWIZZLE_NONE) &&
+         make_tmap_2d(&tm_rope, a.keys.rope, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 64, rows, a.keys.ld_rope * 2, 64,
+                      kTileM, CU_TENSOR_MAP_SWIZZLE_128B);
+  } else {
+    ok = make_tmap_2d(&tm_a, a.keys.data, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 128, rows, a.keys.ld * 2, 64, kTileM,
+                      CU_TENSOR_MAP_SWIZZLE_128B);
+    tm_rope = tm_a;
+  }
+  const uint64_t qrows = static_cast<uint64_t>(a.B) * a.Q * a.H;
+  ok = ok && make_tmap_2d(&tm_q, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 128, qrows, 256, 64, p.NM,
+                          CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!ok) return cudaErrorInvalidValue;
+
+  const size_t smem = tc_smem_bytes(p.NM, fp8);
+  const int grid = static_cast<int>(std::min<long long>(p.units, sm_count()));
+  if (fp8) {
+    cudaFuncSetAttribute(score_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    score_tc_kernel<true><<<grid, 320, smem, st>>>(tm_a, tm_rope, tm_q, p);
+  } else {
+    cudaFuncSetAttribute(score_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    score_tc_kernel<false><<<grid, 192, smem, st>>>(tm_a, tm_rope, tm_q, p);
+  }
+  return cudaGetLastError();
+}
 
 }  // namespace lidx
