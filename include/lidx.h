@@ -39,7 +39,7 @@
 extern "C" {
 #endif
 
-#define LIDX_ABI_VERSION 1
+#define LIDX_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define LIDX_API __attribute__((visibility("default")))
@@ -59,6 +59,14 @@ typedef enum lidx_status {
 #define LIDX_DEV_BOUNDS 0x1u  /* an id outside [0, N) was skipped */
 #define LIDX_DEV_NAN 0x2u     /* a NaN score / negative or NaN probability was excluded */
 #define LIDX_DEV_TIMEOUT 0x4u /* a bounded device wait gave up */
+
+/* Launch flags (the `flags` field of the score, top-k and attention args). */
+#define LIDX_LAUNCH_PDL 0x1u /* programmatic dependent launch: the kernels may start while the previous
+                              * kernel on the stream still runs.  Before waiting for it they only set up
+                              * and read cache-side inputs (index keys, compressed KV and window rows,
+                              * E8M0 scales, attention queries); everything else is read, and every
+                              * global write is made, after the wait.  So with this flag the cache-side
+                              * inputs must not be written by kernels that may still be running. */
 
 /* Storage formats. */
 #define LIDX_F32 0
@@ -116,6 +124,7 @@ typedef struct lidx_score_args {
     lidx_kv keys;
     float *scores;
     int64_t ld_scores;
+    uint32_t flags; /* LIDX_LAUNCH_* */
 } lidx_score_args;
 
 LIDX_API lidx_status lidx_index_score(const lidx_score_args *args, void *stream);
@@ -145,6 +154,7 @@ typedef struct lidx_topk_args {
     int32_t *n_sel;
     uint8_t *mask;
     uint32_t *mask_bits;
+    uint32_t flags; /* LIDX_LAUNCH_* */
 } lidx_topk_args;
 
 LIDX_API lidx_status lidx_topk_select(const lidx_topk_args *args, void *ws, size_t ws_bytes, void *stream);
@@ -183,6 +193,7 @@ typedef struct lidx_attn_args {
     float scale;
     float *out;
     float *lse;
+    uint32_t flags; /* LIDX_LAUNCH_* */
 } lidx_attn_args;
 
 LIDX_API lidx_status lidx_sparse_attn_decode(const lidx_attn_args *args, void *ws, size_t ws_bytes,

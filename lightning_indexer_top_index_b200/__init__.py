@@ -29,6 +29,7 @@ DTYPES = {"f32": F32, "bf16": BF16, "e4m3": E4M3, "f16": F16}
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_WORKSPACE = 0, 1, 2, 3, 4
 DEV_BOUNDS, DEV_NAN, DEV_TIMEOUT = 0x1, 0x2, 0x4
+LAUNCH_PDL = 0x1
 
 EVAL_GOLDEN, EVAL_TOPP, EVAL_VOTE, EVAL_LSA, EVAL_OVERLAP = 0x1, 0x2, 0x4, 0x8, 0x10
 OP_SCORE, OP_TOPK, OP_ATTN, OP_EVAL = 0, 1, 2, 3
@@ -67,21 +68,21 @@ class KVArgs(C.Structure):
 class ScoreArgs(C.Structure):
     _fields_ = [("B", C.c_int32), ("Q", C.c_int32), ("H", C.c_int32), ("N", C.c_int32),
                 ("q_dtype", C.c_int32), ("q", C.c_void_p), ("w", C.c_void_p), ("keys", KVArgs),
-                ("scores", C.c_void_p), ("ld_scores", C.c_int64)]
+                ("scores", C.c_void_p), ("ld_scores", C.c_int64), ("flags", C.c_uint32)]
 
 
 class TopkArgs(C.Structure):
     _fields_ = [("B", C.c_int32), ("Q", C.c_int32), ("N", C.c_int32), ("k", C.c_int32),
                 ("scores", C.c_void_p), ("ld_scores", C.c_int64), ("allowed", C.c_void_p),
                 ("ld_allowed", C.c_int64), ("ids", C.c_void_p), ("n_sel", C.c_void_p), ("mask", C.c_void_p),
-                ("mask_bits", C.c_void_p)]
+                ("mask_bits", C.c_void_p), ("flags", C.c_uint32)]
 
 
 class AttnArgs(C.Structure):
     _fields_ = [("B", C.c_int32), ("H", C.c_int32), ("q_dtype", C.c_int32), ("q", C.c_void_p),
                 ("kv", KVArgs), ("N", C.c_int32), ("ids", C.c_void_p), ("n_ids", C.c_int32),
                 ("ld_ids", C.c_int64), ("n_sel", C.c_void_p), ("swa", KVArgs), ("swa_len", C.c_int32),
-                ("scale", C.c_float), ("out", C.c_void_p), ("lse", C.c_void_p)]
+                ("scale", C.c_float), ("out", C.c_void_p), ("lse", C.c_void_p), ("flags", C.c_uint32)]
 
 
 class EvalArgs(C.Structure):
@@ -238,11 +239,11 @@ def workspace(nbytes: int, device="cuda") -> torch.Tensor:
     return torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=device)
 
 
-def topk_args(scores, k, allowed=None, ids=None, n_sel=None, mask=None, mask_bits=None) -> TopkArgs:
+def topk_args(scores, k, allowed=None, ids=None, n_sel=None, mask=None, mask_bits=None, flags=0) -> TopkArgs:
     B, Q, N = scores.shape[0], scores.shape[1], scores.shape[2]
     return TopkArgs(B, Q, N, k, scores.data_ptr(), scores.stride(1), _ptr(allowed),
                     0 if allowed is None else allowed.stride(0), _ptr(ids), _ptr(n_sel), _ptr(mask),
-                    _ptr(mask_bits))
+                    _ptr(mask_bits), flags)
 
 
 def topk_select(scores: torch.Tensor, k: int, allowed: torch.Tensor = None, *, want_mask=False,
@@ -265,13 +266,14 @@ def topk_select(scores: torch.Tensor, k: int, allowed: torch.Tensor = None, *, w
     return ids, n_sel, mask, bits
 
 
-def attn_args(q, kv: DeviceKV, N, ids, n_sel, swa: Optional[DeviceKV], swa_len, scale, out, lse) -> AttnArgs:
+def attn_args(q, kv: DeviceKV, N, ids, n_sel, swa: Optional[DeviceKV], swa_len, scale, out, lse,
+              flags=0) -> AttnArgs:
     B, H, D = q.shape
     n_ids = 0 if ids is None else ids.shape[-1]
     ld_ids = 0 if ids is None else ids.stride(0)
     swa_a = swa.args() if swa is not None else KVArgs(kv.dtype, kv.dim, None, None, None, 0, 0, 0, 0)
     return AttnArgs(B, H, _qdtype(q), q.data_ptr(), kv.args(), N, _ptr(ids), n_ids, ld_ids, _ptr(n_sel),
-                    swa_a, swa_len if swa is not None else 0, float(scale), out.data_ptr(), _ptr(lse))
+                    swa_a, swa_len if swa is not None else 0, float(scale), out.data_ptr(), _ptr(lse), flags)
 
 
 def sparse_attn_decode(q: torch.Tensor, kv: DeviceKV, N: int, ids: torch.Tensor, n_sel: torch.Tensor = None,

@@ -180,8 +180,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // Combine the split partials of one (b, h): base-2 log-sum-exp rescaling.
+// Thread t owns dims [4t, 4t+4); the split loads are independent, so they
+// overlap instead of forming a dependent chain.
 __global__ void __launch_bounds__(128) attn_merge_kernel(lidx_attn_args a, const float *part_o,
                                                           const float2 *part_ml, int n_split) {
+  pdl_trigger();
+  pdl_wait();  // the partials come from the previous kernel
   const int h = blockIdx.x, b = blockIdx.y, H = a.H;
   extern __shared__ float wgt[];  // [n_split]
   __shared__ float inv_l, lse2;
@@ -204,16 +208,38 @@ __global__ void __launch_bounds__(128) attn_merge_kernel(lidx_attn_args a, const
     }
   }
   __syncthreads();
-  float *out = a.out + (static_cast<size_t>(b) * H + h) * kD;
-  const float *po = part_o + (static_cast<size_t>(b) * n_split * H + h) * kD;
-  for (int d = threadIdx.x; d < kD; d += 128) {
-    float acc = 0.f;
-    for (int s = 0; s < n_split; s++) {
-      const float e = wgt[s];
-      if (e != 0.f) acc = fmaf(e, po[static_cast<size_t>(s) * H * kD + d], acc);
+  const float4 *po = reinterpret_cast<const float4 *>(part_o + (static_cast<size_t>(b) * n_split * H + h) * kD) + threadIdx.x;
+  const size_t stride4 = static_cast<size_t>(H) * kD / 4;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  int s = 0;
+  for (; s + 4 <= n_split; s += 4) {
+    float4 v[4];
+#pragma unroll
+    for (int i = 0; i < 4; i++) v[i] = po[(s + i) * stride4];
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+      const float e = wgt[s + i];
+      if (e != 0.f) {
+        acc.x = fmaf(e, v[i].x, acc.x);
+        acc.y = fmaf(e, v[i].y, acc.y);
+        acc.z = fmaf(e, v[i].z, acc.z);
+        acc.w = fmaf(e, v[i].w, acc.w);
+      }
     }
-    out[d] = acc * inv_l;
   }
+  for (; s < n_split; s++) {
+    const float e = wgt[s];
+    if (e != 0.f) {
+      const float4 v = po[s * stride4];
+      acc.x = fmaf(e, v.x, acc.x);
+      acc.y = fmaf(e, v.y, acc.y);
+      acc.z = fmaf(e, v.z, acc.z);
+      acc.w = fmaf(e, v.w, acc.w);
+    }
+  }
+  const float il = inv_l;
+  reinterpret_cast<float4 *>(a.out + (static_cast<size_t>(b) * H + h) * kD)[threadIdx.x] =
+      make_float4(acc.x * il, acc.y * il, acc.z * il, acc.w * il);
   if (threadIdx.x == 0 && a.lse) a.lse[static_cast<size_t>(b) * H + h] = lse2 * 0.6931471805599453f;
 }
 
@@ -224,19 +250,38 @@ int n_splits(const lidx_attn_args &a) {
 
 }  // namespace
 
+bool attn_tc_supported(const lidx_attn_args &a);
+int attn_tc_splits(const lidx_attn_args &a);
+cudaError_t launch_attn_tc(const lidx_attn_args &a, float *part_o, float2 *part_ml, int n_split, uint32_t *status,
+                           cudaStream_t st);
+
+cudaError_t launch_attn_merge(const lidx_attn_args &a, const float *part_o, const float2 *part_ml, int n_split,
+                              cudaStream_t st) {
+  return launch_kernel(attn_merge_kernel, dim3(a.H, a.B), dim3(128), n_split * sizeof(float), st,
+                       (a.flags & LIDX_LAUNCH_PDL) != 0, a, part_o, part_ml, n_split);
+}
+
+namespace {
+
+int splits_for(const lidx_attn_args &a) { return attn_tc_supported(a) ? attn_tc_splits(a) : n_splits(a); }
+
+size_t part_o_bytes(const lidx_attn_args &a, int ns) {
+  return ((static_cast<size_t>(ns) * a.B * a.H * kD * sizeof(float) + 255) / 256) * 256;
+}
+
+}  // namespace
+
 size_t attn_workspace(const lidx_attn_args &a) {
-  const size_t ns = static_cast<size_t>(n_splits(a));
-  const size_t o = ns * a.B * a.H * kD * sizeof(float);
-  const size_t ml = ns * a.B * a.H * sizeof(float2);
-  return LIDX_WS_HEADER + ((o + 255) / 256) * 256 + ml;
+  const int ns = splits_for(a);
+  return LIDX_WS_HEADER + part_o_bytes(a, ns) + static_cast<size_t>(ns) * a.B * a.H * sizeof(float2);
 }
 
 cudaError_t launch_attn(const lidx_attn_args &a, void *ws, cudaStream_t st) {
   uint32_t *status = static_cast<uint32_t *>(ws);
-  const int ns = n_splits(a);
+  const int ns = splits_for(a);
   float *part_o = reinterpret_cast<float *>(static_cast<char *>(ws) + LIDX_WS_HEADER);
-  const size_t o = static_cast<size_t>(ns) * a.B * a.H * kD * sizeof(float);
-  float2 *part_ml = reinterpret_cast<float2 *>(static_cast<char *>(ws) + LIDX_WS_HEADER + ((o + 255) / 256) * 256);
+  float2 *part_ml = reinterpret_cast<float2 *>(static_cast<char *>(ws) + LIDX_WS_HEADER + part_o_bytes(a, ns));
+  if (attn_tc_supported(a)) return launch_attn_tc(a, part_o, part_ml, ns, status, st);
   const size_t smem = (static_cast<size_t>(a.H) * kD + kRC * kXs + a.H * kRC) * sizeof(float);
   dim3 grid(ns, a.B);
   switch (a.kv.dtype) {
@@ -255,8 +300,7 @@ cudaError_t launch_attn(const lidx_attn_args &a, void *ws, cudaStream_t st) {
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  attn_merge_kernel<<<dim3(a.H, a.B), 128, ns * sizeof(float), st>>>(a, part_o, part_ml, ns);
-  return cudaGetLastError();
+  return launch_attn_merge(a, part_o, part_ml, ns, st);
 }
 
 }  // namespace lidx

@@ -5,6 +5,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/lidx.h"
 
 #define LIDX_WS_HEADER 256  // bytes at the start of every workspace: status word + counters
@@ -92,6 +94,33 @@ __device__ __forceinline__ T warp_inclusive_scan(T v) {
     if (lane >= static_cast<uint32_t>(o)) v += n;
   }
   return v;
+}
+
+// ----------------------------------------------------------------------------
+// Programmatic dependent launch.  pdl_trigger lets the next kernel on the
+// stream start its prologue; pdl_wait blocks until the previous kernel has
+// completed and its writes are visible.  Both are no-ops for a kernel that
+// was not launched as a programmatic dependent.
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Launch `kern` on `st`, as a programmatic dependent of the previous kernel
+// when `pdl` is set.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl,
+                          Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
 // Device status word at the start of a workspace.

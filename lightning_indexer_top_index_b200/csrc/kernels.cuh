@@ -21,6 +21,7 @@ cudaError_t launch_score_tc(const lidx_score_args &a, cudaStream_t st);
 bool score_tc_supported(const lidx_score_args &a);
 
 // ---- top-k
+bool topk_supported(const lidx_topk_args &a);
 size_t topk_workspace(const lidx_topk_args &a);
 cudaError_t launch_topk(const lidx_topk_args &a, void *ws, cudaStream_t st);
 

@@ -67,6 +67,7 @@ lidx_status check_topk(const lidx_topk_args *a) {
   if (a->allowed && a->ld_allowed < a->N) return LIDX_ERR_INVALID_ARG;
   if (!aligned(a->scores, 4) || !aligned(a->ids, 4) || (a->mask_bits && !aligned(a->mask_bits, 4)))
     return LIDX_ERR_INVALID_ARG;
+  if (!topk_supported(*a)) return LIDX_ERR_UNSUPPORTED;
   return LIDX_OK;
 }
 

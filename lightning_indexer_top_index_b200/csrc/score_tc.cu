@@ -94,6 +94,25 @@ __global__ void __launch_bounds__(kFp8 ? 320 : 192, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long u0 = blockIdx.x * p.units / gridDim.x, u1 = (blockIdx.x + 1) * p.units / gridDim.x;
 
+  // Key tiles of the first kStages units: cache-side data, issued before the
+  // block sync and before waiting for the previous kernel on the stream.
+  const long long n_pre = min(static_cast<long long>(kStages), u1 - u0);
+  auto issue_a = [&](long long u, int stage) {
+    int b, g, t;
+    long long bg;
+    unit_coords(p, u, b, g, t, bg);
+    const int row = static_cast<int>(b * p.key_batch_rows + static_cast<int64_t>(t) * kTileM);
+    uint8_t *a = sA + stage * kTileBytes;
+    if (kFp8) {
+      tc::mbar_arrive_expect_tx(&bar->full[stage], kF8Bytes + kPanelBytes);
+      tc::tma_load_2d(sF8 + stage * kF8Bytes, &tm_a, &bar->full[stage], 0, row);
+      tc::tma_load_2d(a + kPanelBytes, &tm_rope, &bar->full[stage], 0, row);
+    } else {
+      tc::mbar_arrive_expect_tx(&bar->full[stage], kTileBytes);
+      tc::tma_load_2d(a, &tm_a, &bar->full[stage], 0, row);
+      tc::tma_load_2d(a + kPanelBytes, &tm_a, &bar->full[stage], 64, row);
+    }
+  };
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; s++) {
       tc::mbar_init(&bar->full[s], 1);
@@ -108,28 +127,34 @@ __global__ void __launch_bounds__(kFp8 ? 320 : 192, 1)
     tc::mbar_init(&bar->bempty, 1);
     bar->abort = 0;
     tc::fence_barrier_init();
-  }
-  if (warp == 0 && lane == 0) {
     tc::tma_prefetch_desc(&tm_a);
     tc::tma_prefetch_desc(&tm_q);
     if (kFp8) tc::tma_prefetch_desc(&tm_rope);
+    for (long long i = 0; i < n_pre; i++) issue_a(u0 + i, static_cast<int>(i));
   }
   if (warp == 1) tc::tmem_alloc(&bar->tmem_base, p.tmem_cols);
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
+  pdl_trigger();
   const uint32_t tmem = bar->tmem_base;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0, bempty_par = 0;
+      uint32_t bempty_par = 0;
       uint32_t last_par[kStages];
       bool used[kStages] = {};
+      for (long long i = 0; i < n_pre; i++) {
+        last_par[i] = 0;
+        used[i] = true;
+      }
+      int stage = static_cast<int>(n_pre % kStages);
+      uint32_t phase = n_pre == kStages ? 1u : 0u;
       bool b_loaded = false;
       uint32_t bfull_last = 0;
       long long prev_bg = -1;
+      pdl_wait();  // queries and weights may come from the previous kernel
       for (long long u = u0; u < u1; u++) {
         int b, g, t;
         long long bg;
@@ -147,18 +172,9 @@ __global__ void __launch_bounds__(kFp8 ? 320 : 192, 1)
           b_loaded = true;
           prev_bg = bg;
         }
+        if (u - u0 < n_pre) continue;  // key tile already in flight
         if (!tc::mbar_wait(&bar->empty[stage], phase ^ 1, abort_flag)) break;
-        const int row = static_cast<int>(b * p.key_batch_rows + static_cast<int64_t>(t) * kTileM);
-        uint8_t *a = sA + stage * kTileBytes;
-        if (kFp8) {
-          tc::mbar_arrive_expect_tx(&bar->full[stage], kF8Bytes + kPanelBytes);
-          tc::tma_load_2d(sF8 + stage * kF8Bytes, &tm_a, &bar->full[stage], 0, row);
-          tc::tma_load_2d(a + kPanelBytes, &tm_rope, &bar->full[stage], 0, row);
-        } else {
-          tc::mbar_arrive_expect_tx(&bar->full[stage], kTileBytes);
-          tc::tma_load_2d(a, &tm_a, &bar->full[stage], 0, row);
-          tc::tma_load_2d(a + kPanelBytes, &tm_a, &bar->full[stage], 64, row);
-        }
+        issue_a(u, stage);
         last_par[stage] = phase;
         used[stage] = true;
         if (++stage == kStages) {
@@ -228,6 +244,7 @@ __global__ void __launch_bounds__(kFp8 ? 320 : 192, 1)
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const int etid = threadIdx.x - 64;
+    pdl_wait();  // head weights may come from the previous kernel
     int acc = 0;
     uint32_t acc_par = 0;
     long long prev_bg = -1;
@@ -402,15 +419,15 @@ cudaError_t launch_score_tc(const lidx_score_args &a, cudaStream_t st) {
   if (!ok) return cudaErrorInvalidValue;
 
   const size_t smem = tc_smem_bytes(p.NM, fp8);
+  const bool pdl = (a.flags & LIDX_LAUNCH_PDL) != 0;
   const int grid = static_cast<int>(std::min<long long>(p.units, sm_count()));
   if (fp8) {
     cudaFuncSetAttribute(score_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    score_tc_kernel<true><<<grid, 320, smem, st>>>(tm_a, tm_rope, tm_q, p);
+    return launch_kernel(score_tc_kernel<true>, dim3(grid), dim3(320), smem, st, pdl, tm_a, tm_rope, tm_q, p);
   } else {
     cudaFuncSetAttribute(score_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    score_tc_kernel<false><<<grid, 192, smem, st>>>(tm_a, tm_rope, tm_q, p);
+    return launch_kernel(score_tc_kernel<false>, dim3(grid), dim3(192), smem, st, pdl, tm_a, tm_rope, tm_q, p);
   }
-  return cudaGetLastError();
 }
 
 }  // namespace lidx

@@ -30,7 +30,8 @@ def test_exports_every_declared_symbol(lib):
     for n in names:
         assert hasattr(lib, n), n
     assert set(L.EXPORTS) <= set(names)
-    assert lib.lidx_abi_version() == 1
+    hdr = open(os.path.join(ROOT, "include", "lidx.h")).read()
+    assert lib.lidx_abi_version() == int(re.search(r"#define LIDX_ABI_VERSION (\d+)", hdr).group(1))
 
 
 def test_struct_sizes_match(lib):
