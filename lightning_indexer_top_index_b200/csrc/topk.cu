@@ -4,20 +4,22 @@
 //
 // Scores become order-preserving 32-bit keys (order_key: larger score ->
 // larger key, -0 folded onto +0, NaN and disallowed entries -> 0).  One CTA of
-// 512 threads selects within up to 32768 keys held in registers: thread t owns
-// the contiguous positions [t*ITEMS, (t+1)*ITEMS).
+// 1024 threads selects within up to 32768 keys held in registers: thread t
+// owns the contiguous positions [t*C, (t+1)*C), all loaded up front.
 //   1. One histogram pass over 256 linear value bins between the row's
-//      minimum and maximum.  The bin is a monotone function of the score, so
-//      the bin holding the k-th largest key, and the count above it, are
-//      exact; for score-like distributions that bin holds a few dozen keys.
-//   2. Those keys are compacted into shared memory and an exact radix select
-//      over only their differing bits (8-bit digits, per-warp histograms)
-//      pins the k-th key T and how many keys equal to T are taken.
-//      Degenerate rows (a bin too full to compact) run the same radix over
-//      the register-resident keys of that bin.
+//      minimum and maximum (found during the load).  The bin is a monotone
+//      function of the score, so the bin holding the k-th largest key, and
+//      the count above it, are exact; for score-like distributions that bin
+//      holds a few dozen keys.
+//   2. A block scan compacts that bin into shared memory; each candidate
+//      counts the candidates above and equal to it, which pins the k-th key
+//      T and how many keys equal to T are taken.  A bin too full for this
+//      runs an exact radix over the candidates' differing bits instead.
 //   3. One packed 64-bit block scan of (#keys > T, #keys == T) per thread gives
 //      each thread its output offset: ids come out ascending, ties resolved
 //      toward the lower index.
+// Every phase costs a few instructions per key; the few block barriers are
+// the floor.
 //
 // Rows longer than 32768 entries take two levels: chunks of 8192 keep their
 // own top-k (the global top-k is a subset of the union, under the same total
@@ -26,14 +28,15 @@
 #include <algorithm>
 
 #include "kernels.cuh"
+#include "tc.cuh"
 
 namespace lidx {
 
 namespace {
 
-constexpr int kThreads = 512;
+constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / 32;
-constexpr int kMaxItems = 64;
+constexpr int kMaxItems = 32;
 constexpr int kSingleMax = kThreads * kMaxItems;  // 32768
 constexpr int kChunk = 8192;
 
@@ -50,13 +53,14 @@ struct SelParams {
 };
 
 constexpr int kCandMax = 4096;
+constexpr int kRankMax = 1024;  // candidates resolved by direct rank counting
 
 struct SelSmem {
-  uint32_t whist[kWarps][256];  // per-warp histograms
+  uint32_t whist[8][256];       // histograms shared by groups of four warps
   uint32_t hist[256];
   uint32_t cand[kCandMax];      // keys of the threshold bin
-  unsigned long long warp_tot[kWarps];
   uint32_t red_a[kWarps], red_b[kWarps];
+  uint32_t red_tot;
   uint32_t n_elig;
   uint32_t nan_seen;
   uint32_t n_cand;
@@ -64,6 +68,7 @@ struct SelSmem {
   uint32_t above;
   uint32_t kmin, kmax;
   int32_t chunk_off[130];
+  uint64_t bar;
 };
 
 __device__ __forceinline__ float key_value(uint32_t key) {
@@ -97,7 +102,7 @@ __device__ __forceinline__ void block_minmax(SelSmem &sm, uint32_t lo, uint32_t 
 
 __device__ __forceinline__ void whist_clear(SelSmem &sm) {
   uint32_t *h = &sm.whist[0][0];
-  for (int i = threadIdx.x; i < kWarps * 256; i += kThreads) h[i] = 0u;
+  for (int i = threadIdx.x; i < 8 * 256; i += kThreads) h[i] = 0u;
 }
 
 // Merge the per-warp histograms of `nbins` bins and find the bin holding the
@@ -108,7 +113,7 @@ __device__ __forceinline__ void whist_find(SelSmem &sm, int nbins, uint32_t rem)
     uint32_t v = 0;
     if (static_cast<int>(threadIdx.x) < nbins)
 #pragma unroll
-      for (int w = 0; w < kWarps; w++) v += sm.whist[w][threadIdx.x];
+      for (int w = 0; w < 8; w++) v += sm.whist[w][threadIdx.x];
     sm.hist[threadIdx.x] = v;
   }
   __syncthreads();
@@ -138,47 +143,50 @@ __device__ __forceinline__ void whist_find(SelSmem &sm, int nbins, uint32_t rem)
   __syncthreads();
 }
 
-__device__ __forceinline__ unsigned long long block_exclusive_scan_u64(SelSmem &sm, unsigned long long v,
-                                                                        unsigned long long &total) {
+// Exclusive block scan of 32-bit values; warp totals are scanned by one warp.
+// Returns the thread's exclusive prefix; *total gets the block sum.
+__device__ __forceinline__ uint32_t block_exclusive_scan(SelSmem &sm, uint32_t v, uint32_t &total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  unsigned long long inc = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const unsigned long long n = __shfl_up_sync(0xFFFFFFFFu, inc, o);
-    if (lane >= o) inc += n;
-  }
-  if (lane == 31) sm.warp_tot[warp] = inc;
+  const uint32_t inc = warp_inclusive_scan(v);
+  if (lane == 31) sm.red_a[warp] = inc;
   __syncthreads();
-  unsigned long long before = 0, tot = 0;
-#pragma unroll
-  for (int w = 0; w < kWarps; w++) {
-    const unsigned long long x = sm.warp_tot[w];
-    before += (w < warp) ? x : 0ull;
-    tot += x;
+  if (warp == 0) {
+    const uint32_t x = sm.red_a[lane];
+    const uint32_t xi = warp_inclusive_scan(x);
+    sm.red_b[lane] = xi - x;
+    if (lane == 31) sm.red_tot = xi;
   }
-  total = tot;
-  return before + inc - v;
+  __syncthreads();
+  total = sm.red_tot;
+  return sm.red_b[warp] + inc - v;
 }
 
-template <int ITEMS, int MODE>
+// Monotone 8-bit bin of a key inside [flo, flo + 256/scale]: round((x-flo)*scale)
+// read off the mantissa of x*scale + 2^23 (no float-to-int conversion).
+__device__ __forceinline__ uint32_t lin_bin(uint32_t kk, float flo, float scale) {
+  const float t = fmaf(key_value(kk) - flo, scale, 8388608.f);
+  return min(__float_as_uint(t) - 0x4B000000u, 255u);
+}
+
+template <int C, int MODE>
 __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelParams p) {
+  extern __shared__ __align__(16) float rowbuf[];  // the row's scores (row modes)
   __shared__ SelSmem sm;
   const lidx_topk_args &a = p.a;
   const int tid = threadIdx.x, lane = tid & 31;
+  const int hg = (tid >> 5) & 7;  // histogram group
   const int row = blockIdx.y;
   const int chunk = blockIdx.x;
   const int k = MODE == kRowCandidates ? p.kc : a.k;
+  const int p0 = tid * C;
 
-  uint32_t key[ITEMS];
-  int len;  // number of positions this CTA selects from
   pdl_trigger();
   pdl_wait();  // the scores / candidates come from the previous kernel
   if (tid == 0) {
     sm.n_elig = 0;
     sm.nan_seen = 0;
-  }
-  if (MODE == kMergeFinal) {
-    if (tid == 0) {
+    sm.n_cand = 0;
+    if (MODE == kMergeFinal) {
       int off = 0;
       for (int c = 0; c < p.n_chunks; c++) {
         sm.chunk_off[c] = off;
@@ -187,13 +195,18 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelParams p) 
       sm.chunk_off[p.n_chunks] = off;
     }
   }
+  whist_clear(sm);
   __syncthreads();
+
+  // ---- keys into registers
+  uint32_t key[C];
+  int len;
   if (MODE == kMergeFinal) {
     len = sm.chunk_off[p.n_chunks];
     int c = 0;
 #pragma unroll
-    for (int i = 0; i < ITEMS; i++) {
-      const int pos = tid * ITEMS + i;
+    for (int i = 0; i < C; i++) {
+      const int pos = p0 + i;
       key[i] = 0u;
       if (pos < len) {
         while (pos >= sm.chunk_off[c + 1]) c++;
@@ -205,55 +218,60 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelParams p) 
     len = MODE == kRowCandidates ? min(kChunk, a.N - j0) : a.N;
     const float *s = a.scores + static_cast<size_t>(row) * a.ld_scores + j0;
     const uint8_t *al = a.allowed ? a.allowed + static_cast<size_t>(row / a.Q) * a.ld_allowed + j0 : nullptr;
-    uint32_t nanf = 0;
-    if (ITEMS % 4 == 0 && ((reinterpret_cast<uintptr_t>(s) & 15u) == 0) && (tid + 1) * ITEMS <= len) {
-#pragma unroll
-      for (int i = 0; i < ITEMS; i += 4) {
-        const float4 v = *reinterpret_cast<const float4 *>(s + tid * ITEMS + i);
-        key[i] = order_key(v.x);
-        key[i + 1] = order_key(v.y);
-        key[i + 2] = order_key(v.z);
-        key[i + 3] = order_key(v.w);
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < ITEMS; i++) {
-        const int pos = tid * ITEMS + i;
-        key[i] = pos < len ? order_key(s[pos]) : 0u;
-      }
+    // one bulk copy of the 16-byte-aligned body of the row into shared memory
+    const int head = static_cast<int>(((16u - (reinterpret_cast<uintptr_t>(s) & 15u)) & 15u) / 4u);
+    const int body = max(0, (len - head)) & ~3;
+    // shift the buffer so the body lands 16-byte aligned in shared memory too
+    float *sv = rowbuf + ((4 - head) & 3);
+    if (tid == 0) {
+      tc::mbar_init(&sm.bar, 1);
+      tc::fence_barrier_init();
     }
+    __syncthreads();
+    if (tid == 0 && body > 0) {
+      tc::mbar_arrive_expect_tx(&sm.bar, body * 4);
+      asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                       tc::smem_u32(sv + head)),
+                   "l"(s + head), "r"(body * 4), "r"(tc::smem_u32(&sm.bar))
+                   : "memory");
+    }
+    for (int j = tid; j < len; j += kThreads)
+      if (j < head || j >= head + body) sv[j] = s[j];
+    if (body > 0) {
+      volatile uint32_t no_abort = 0;
+      if (!tc::mbar_wait(&sm.bar, 0, &no_abort)) raise_status(p.status, LIDX_DEV_TIMEOUT);
+    }
+    __syncthreads();
+    uint32_t nanf = 0;
 #pragma unroll
-    for (int i = 0; i < ITEMS; i++) {
-      const int pos = tid * ITEMS + i;
-      if (pos < len) {
-        if (key[i] == 0u && !(al && !al[pos])) nanf = 1u;
-        if (al && !al[pos]) key[i] = 0u;
-      }
+    for (int i = 0; i < C; i++) {
+      const int pos = p0 + i;
+      uint32_t kk = pos < len ? order_key(sv[pos]) : 0u;
+      if (pos < len && kk == 0u && !(al && !al[pos])) nanf = 1u;
+      if (al && pos < len && !al[pos]) kk = 0u;
+      key[i] = kk;
     }
     if (nanf) sm.nan_seen = 1u;
   }
-  uint32_t elig = 0;
+  uint32_t elig = 0, lo = 0xFFFFFFFFu, hi = 0u;
 #pragma unroll
-  for (int i = 0; i < ITEMS; i++) elig += key[i] != 0u;
+  for (int i = 0; i < C; i++) {
+    if (key[i]) {
+      elig++;
+      lo = min(lo, key[i]);
+      hi = max(hi, key[i]);
+    }
+  }
   elig = warp_sum(elig);
   if (lane == 0 && elig) atomicAdd(&sm.n_elig, elig);
-  __syncthreads();
+  block_minmax(sm, lo, hi);  // includes the barrier that publishes n_elig
   const uint32_t n_elig = sm.n_elig;
+  const uint32_t kmin = sm.kmin, kmax = sm.kmax;
   if (MODE != kMergeFinal && tid == 0 && sm.nan_seen) raise_status(p.status, LIDX_DEV_NAN);
 
   // ---- exact k-th key T and the number `need` of keys equal to T to take
   uint32_t T = 0u, need = 0u;  // T = 0: take every eligible key
   if (n_elig > static_cast<uint32_t>(k)) {
-    const int warp = tid >> 5;
-    uint32_t lo = 0xFFFFFFFFu, hi = 0u;
-#pragma unroll
-    for (int i = 0; i < ITEMS; i++)
-      if (key[i]) {
-        lo = min(lo, key[i]);
-        hi = max(hi, key[i]);
-      }
-    block_minmax(sm, lo, hi);
-    const uint32_t kmin = sm.kmin, kmax = sm.kmax;
     uint32_t rem = static_cast<uint32_t>(k);
     if (kmin == kmax) {
       T = kmax;
@@ -265,100 +283,124 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelParams p) 
       const float scale0 = 256.f / range;
       const bool linear = isfinite(range) && range > 0.f && isfinite(scale0);
       const float scale = linear ? scale0 : 0.f;
-      auto bin_of = [&](uint32_t kk) -> uint32_t {
-        if (!linear) return kk >> 24;
-        const float t = (key_value(kk) - flo) * scale;
-        return t >= 255.f ? 255u : static_cast<uint32_t>(t);
-      };
-      whist_clear(sm);
-      if (tid == 0) sm.n_cand = 0;
-      __syncthreads();
+      // bins computed once, four per register; 0xFF..: no key (bins are 0..255)
+      uint32_t pbin[(C + 3) / 4];
 #pragma unroll
-      for (int i = 0; i < ITEMS; i++)
-        if (key[i]) atomicAdd(&sm.whist[warp][bin_of(key[i])], 1u);
+      for (int i = 0; i < (C + 3) / 4; i++) pbin[i] = 0u;
+#pragma unroll
+      for (int i = 0; i < C; i++) {
+        uint32_t b = 0u;
+        if (key[i]) {
+          b = linear ? lin_bin(key[i], flo, scale) : (key[i] >> 24);
+          atomicAdd(&sm.whist[hg][b], 1u);
+        }
+        pbin[i / 4] |= b << (8 * (i % 4));
+      }
+      auto bin_at = [&](int i) -> uint32_t { return (pbin[i / 4] >> (8 * (i % 4))) & 0xFFu; };
       whist_find(sm, 256, rem);
       const uint32_t dbin = sm.digit;
       rem -= sm.above;
-      // 2. compact the threshold bin
+      // 2. compact the threshold bin (index order, by block scan)
+      uint32_t nc = 0;
 #pragma unroll
-      for (int i = 0; i < ITEMS; i++) {
-        const bool c = key[i] != 0u && bin_of(key[i]) == dbin;
-        const uint32_t bal = __ballot_sync(0xFFFFFFFFu, c);
-        uint32_t base = 0;
-        if (lane == 0 && bal) base = atomicAdd(&sm.n_cand, static_cast<uint32_t>(__popc(bal)));
-        base = __shfl_sync(0xFFFFFFFFu, base, 0);
-        const uint32_t pos = base + __popc(bal & ((1u << lane) - 1u));
-        if (c && pos < kCandMax) sm.cand[pos] = key[i];
-      }
+      for (int i = 0; i < C; i++) nc += key[i] != 0u && bin_at(i) == dbin;
+      uint32_t n_cand;
+      uint32_t cpos = block_exclusive_scan(sm, nc, n_cand);
+#pragma unroll
+      for (int i = 0; i < C; i++)
+        if (key[i] != 0u && bin_at(i) == dbin) {
+          if (cpos < kCandMax) sm.cand[cpos] = key[i];
+          cpos++;
+        }
       __syncthreads();
-      const uint32_t n_cand = sm.n_cand;
-      const bool in_smem = n_cand <= static_cast<uint32_t>(kCandMax);
-      // candidate source: the compacted list, or the register keys of the bin
-      auto for_each_cand = [&](auto &&fn) {
-        if (in_smem) {
-          for (uint32_t i = tid; i < n_cand; i += kThreads) fn(sm.cand[i]);
-        } else {
-#pragma unroll
-          for (int i = 0; i < ITEMS; i++)
-            if (key[i] && bin_of(key[i]) == dbin) fn(key[i]);
+      if (n_cand <= static_cast<uint32_t>(kRankMax)) {
+        // 3a. each candidate counts the candidates above / equal to it
+        if (tid < static_cast<int>(n_cand)) {
+          const uint32_t mine = sm.cand[tid];
+          uint32_t gt = 0, eq = 0;
+          for (uint32_t j = 0; j < n_cand; j++) {
+            const uint32_t o = sm.cand[j];
+            gt += o > mine;
+            eq += o == mine;
+          }
+          if (gt < rem && gt + eq >= rem) {
+            sm.kmin = mine;        // T
+            sm.kmax = rem - gt;    // need
+          }
         }
-      };
-      uint32_t clo = 0xFFFFFFFFu, chi = 0u;
-      for_each_cand([&](uint32_t kk) {
-        clo = min(clo, kk);
-        chi = max(chi, kk);
-      });
-      block_minmax(sm, clo, chi);
-      const uint32_t cmin = sm.kmin, cmax = sm.kmax;
-      if (cmin == cmax) {
-        T = cmin;
-        need = rem;
+        __syncthreads();
+        T = sm.kmin;
+        need = sm.kmax;
       } else {
-        // 3. radix over the differing bits of the candidates
-        int bits_left = 32 - __clz(cmin ^ cmax);
-        uint32_t prefix = cmin & (bits_left == 32 ? 0u : ~((1u << bits_left) - 1u));
-        uint32_t pmask = bits_left == 32 ? 0u : ~((1u << bits_left) - 1u);
-        while (bits_left > 0) {
-          const int w = min(8, bits_left);
-          const int shift = bits_left - w;
-          const uint32_t dmask = (1u << w) - 1u;
-          whist_clear(sm);
-          __syncthreads();
-          for_each_cand([&](uint32_t kk) {
-            if ((kk & pmask) == prefix) atomicAdd(&sm.whist[warp][(kk >> shift) & dmask], 1u);
-          });
-          whist_find(sm, 1 << w, rem);
-          prefix |= sm.digit << shift;
-          pmask |= dmask << shift;
-          rem -= sm.above;
-          bits_left -= w;
+        // 3b. radix over the differing bits of the candidates
+        const bool in_list = n_cand <= static_cast<uint32_t>(kCandMax);
+        auto for_each_cand = [&](auto &&fn) {
+          if (in_list) {
+            for (uint32_t i = tid; i < n_cand; i += kThreads) fn(sm.cand[i]);
+          } else {
+#pragma unroll
+            for (int i = 0; i < C; i++)
+              if (key[i] != 0u && bin_at(i) == dbin) fn(key[i]);
+          }
+        };
+        uint32_t clo = 0xFFFFFFFFu, chi = 0u;
+        for_each_cand([&](uint32_t kk) {
+          clo = min(clo, kk);
+          chi = max(chi, kk);
+        });
+        block_minmax(sm, clo, chi);
+        const uint32_t cmin = sm.kmin, cmax = sm.kmax;
+        if (cmin == cmax) {
+          T = cmin;
+          need = rem;
+        } else {
+          int bits_left = 32 - __clz(cmin ^ cmax);
+          uint32_t pmask = bits_left == 32 ? 0u : ~((1u << bits_left) - 1u);
+          uint32_t prefix = cmin & pmask;
+          while (bits_left > 0) {
+            const int w = min(8, bits_left);
+            const int shift = bits_left - w;
+            const uint32_t dmask = (1u << w) - 1u;
+            __syncthreads();
+            whist_clear(sm);
+            __syncthreads();
+            for_each_cand([&](uint32_t kk) {
+              if ((kk & pmask) == prefix) atomicAdd(&sm.whist[hg][(kk >> shift) & dmask], 1u);
+            });
+            whist_find(sm, 1 << w, rem);
+            prefix |= sm.digit << shift;
+            pmask |= dmask << shift;
+            rem -= sm.above;
+            bits_left -= w;
+          }
+          T = prefix;
+          need = rem;
         }
-        T = prefix;
-        need = rem;
       }
     }
   }
 
   // ---- ordered emission
   uint32_t n_gt = 0, n_eq = 0;
-  if (T != 0u) {
 #pragma unroll
-    for (int i = 0; i < ITEMS; i++) {
+  for (int i = 0; i < C; i++) {
+    if (T == 0u) {
+      n_gt += key[i] != 0u;
+    } else {
       n_gt += key[i] > T;
       n_eq += key[i] == T;
     }
-  } else {
-#pragma unroll
-    for (int i = 0; i < ITEMS; i++) n_gt += key[i] != 0u;
   }
-  unsigned long long total;
-  const unsigned long long ex = block_exclusive_scan_u64(sm, (static_cast<unsigned long long>(n_gt) << 32) | n_eq, total);
-  const uint32_t gt_before = static_cast<uint32_t>(ex >> 32), eq_before = static_cast<uint32_t>(ex);
+  uint32_t total;
+  __syncthreads();
+  // (#gt << 16) | #eq: both at most 32768 per CTA
+  const uint32_t ex = block_exclusive_scan(sm, (n_gt << 16) | n_eq, total);
+  const uint32_t gt_before = ex >> 16, eq_before = ex & 0xFFFFu;
   uint32_t out = gt_before + min(eq_before, need);
   uint32_t eq_rank = eq_before;
-  const uint32_t n_out = static_cast<uint32_t>(total >> 32) + min(static_cast<uint32_t>(total), need);
+  const uint32_t n_out = (total >> 16) + min(total & 0xFFFFu, need);
 
-  uint64_t selbits = 0;
+  uint32_t selbits = 0;
   int32_t *ids = nullptr;
   uint32_t *ckey = nullptr;
   int32_t *cidx = nullptr;
@@ -370,7 +412,8 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelParams p) 
   }
   int c = 0;
 #pragma unroll
-  for (int i = 0; i < ITEMS; i++) {
+  for (int i = 0; i < C; i++) {
+    const int pos = p0 + i;
     const uint32_t kk = key[i];
     bool sel;
     if (T == 0u) {
@@ -383,7 +426,6 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelParams p) 
       }
     }
     if (sel) {
-      const int pos = tid * ITEMS + i;
       if (MODE == kRowCandidates) {
         ckey[out] = kk;
         cidx[out] = chunk * kChunk + pos;
@@ -394,7 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelParams p) 
         ids[out] = p.cand_idx[(static_cast<size_t>(row) * p.n_chunks + c) * p.kc + (pos - sm.chunk_off[c])];
       }
       out++;
-      if (ITEMS <= 64) selbits |= 1ull << i;
+      selbits |= 1u << i;
     }
   }
   if (MODE == kRowCandidates) {
@@ -408,26 +450,20 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelParams p) 
     if (a.mask) {
       uint8_t *m = a.mask + static_cast<size_t>(row) * N;
 #pragma unroll
-      for (int i = 0; i < ITEMS; i++) {
-        const int pos = tid * ITEMS + i;
-        if (pos < N) m[pos] = static_cast<uint8_t>((selbits >> i) & 1u);
-      }
+      for (int i = 0; i < C; i++)
+        if (p0 + i < N) m[p0 + i] = static_cast<uint8_t>((selbits >> i) & 1u);
     }
     if (a.mask_bits) {
       const int Wn = (N + 31) / 32;
       uint32_t *bw = a.mask_bits + static_cast<size_t>(row) * Wn;
-      if (ITEMS >= 32) {
-#pragma unroll
-        for (int w = 0; w < ITEMS / 32; w++) {
-          const int wi = tid * (ITEMS / 32) + w;
-          if (wi < Wn) bw[wi] = static_cast<uint32_t>(selbits >> (32 * w));
-        }
+      if (C == 32) {
+        if (tid < Wn) bw[tid] = selbits;
       } else {
-        uint32_t word = static_cast<uint32_t>(selbits) << ((tid * ITEMS) & 31);
+        uint32_t word = selbits << (p0 & 31);
 #pragma unroll
-        for (int o = 1; o < 32 / ITEMS; o <<= 1) word |= __shfl_xor_sync(0xFFFFFFFFu, word, o);
-        const int wi = (tid * ITEMS) >> 5;
-        if (((tid * ITEMS) & 31) == 0 && wi < Wn) bw[wi] = word;
+        for (int o = 1; o < 32 / C; o <<= 1) word |= __shfl_xor_sync(0xFFFFFFFFu, word, o);
+        const int wi = p0 >> 5;
+        if ((p0 & 31) == 0 && wi < Wn) bw[wi] = word;
       }
     }
   }
@@ -461,18 +497,24 @@ __global__ void mask_scatter_kernel(lidx_topk_args a) {
   }
 }
 
+template <int C, int MODE>
+cudaError_t launch_c(dim3 grid, const SelParams &p, cudaStream_t st, bool pdl) {
+  const size_t smem = MODE == kMergeFinal ? 0 : (static_cast<size_t>(C) * kThreads + 4) * sizeof(float);
+  // static + dynamic shared memory exceeds the default 48 KB window
+  cudaFuncSetAttribute(select_kernel<C, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  return launch_kernel(select_kernel<C, MODE>, grid, dim3(kThreads), smem, st, pdl, p);
+}
+
 template <int MODE>
 cudaError_t launch_items(int items, dim3 grid, const SelParams &p, cudaStream_t st) {
   const bool pdl = (p.a.flags & LIDX_LAUNCH_PDL) != 0;
-  const dim3 blk(kThreads);
   switch (items) {
-    case 1: return launch_kernel(select_kernel<1, MODE>, grid, blk, 0, st, pdl, p);
-    case 2: return launch_kernel(select_kernel<2, MODE>, grid, blk, 0, st, pdl, p);
-    case 4: return launch_kernel(select_kernel<4, MODE>, grid, blk, 0, st, pdl, p);
-    case 8: return launch_kernel(select_kernel<8, MODE>, grid, blk, 0, st, pdl, p);
-    case 16: return launch_kernel(select_kernel<16, MODE>, grid, blk, 0, st, pdl, p);
-    case 32: return launch_kernel(select_kernel<32, MODE>, grid, blk, 0, st, pdl, p);
-    default: return launch_kernel(select_kernel<64, MODE>, grid, blk, 0, st, pdl, p);
+    case 1: return launch_c<1, MODE>(grid, p, st, pdl);
+    case 2: return launch_c<2, MODE>(grid, p, st, pdl);
+    case 4: return launch_c<4, MODE>(grid, p, st, pdl);
+    case 8: return launch_c<8, MODE>(grid, p, st, pdl);
+    case 16: return launch_c<16, MODE>(grid, p, st, pdl);
+    default: return launch_c<32, MODE>(grid, p, st, pdl);
   }
 }
 
