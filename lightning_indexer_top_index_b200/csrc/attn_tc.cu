@@ -3,19 +3,24 @@
 // rows plus the 128-row sliding window; K = V = the full row).
 //
 // One CTA takes 128 rows of one sequence's row list (the window rows, then
-// the selected ids) and produces the split partial (m_h, l_h, O_h) in base-2 units:
-//   1. Q [64 heads][512] arrives by TMA; the 128 gathered rows are copied
-//      with cp.async straight into the 128-byte-swizzled K-major layout
-//      (E4M3 rows are converted in registers, the power-of-two block scale
-//      added to the bf16 exponent; RoPE dims copied as they are).
+// the selected ids) and produces the split partial (m_h, l_h, O_h) in base-2
+// units for the 64 heads:
+//   1. Q [64 heads][512] arrives by TMA.  A chunk made only of window rows
+//      (contiguous in memory) arrives as eight 128-row TMA boxes before the
+//      top-k kernel has finished; gathered bf16 rows are copied with
+//      cp.async, one warp per row, straight into the 128-byte-swizzled
+//      K-major layout; E4M3 rows are converted in registers (the
+//      power-of-two block scale added to the bf16 exponent; RoPE dims copied).
 //   2. MMA 1: S^T[row][head] = X . Q^T (M = 128 rows, N = 64 heads,
 //      K = 512) into TMEM.
-//   3. Softmax: 8 warps, each thread one row and 32 heads; per-head max and
-//      sum over rows by butterfly shuffles and a 4-warp exchange; P^T is
-//      written to shared memory as bf16 in the swizzled MN-major layout.
+//   3. Softmax: 16 warps; thread = one row and 16 heads (warp w: TMEM lane
+//      quarter w&3, heads 16*(w>>2)..); per-head max and sum over rows by
+//      butterfly shuffles and a 4-warp exchange; P^T is written to shared
+//      memory as bf16 hi and lo parts (p = hi + lo to ~16 bits) in the
+//      swizzled MN-major layout.
 //   4. MMA 2: O^T[d][head] = X^T . P^T, reading the same X tile as an
 //      MN-major operand (K = V), four 128-wide d tiles into TMEM.
-//   5. Each thread reads 64 heads of one d and stores the partial O.
+//   5. Warp w stores d tile w>>2, lanes = consecutive d: coalesced stores.
 // The partials are combined by the split-K merge kernel.
 #include "kernels.cuh"
 #include "tc.cuh"
@@ -30,7 +35,7 @@ namespace {
 constexpr int kD = 512;
 constexpr int kH = 64;
 constexpr int kRows = 128;
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;
 constexpr int kQBytes = kH * kD * 2;         // 64 KB: 8 panels of [64][128 B]
 constexpr int kQPanel = kH * 128;            // 8 KB
 constexpr int kXBytes = kRows * kD * 2;      // 128 KB: 8 panels of [128][128 B]
@@ -46,7 +51,7 @@ struct __align__(8) AttnTcSmem {
   uint32_t abort;
   int64_t row_src[kRows];  // byte offset of the row in its plane set; -1 when empty
   int32_t row_kind[kRows]; // 0 none, 1 selected, 2 window
-  float red[2][4][32];     // per head-half, per warp: max then sum
+  float red[4][4][16];     // per head group, per lane quarter: max, then sum
 };
 
 // Q is dead once MMA 1 has completed; P^T (hi and lo bf16 parts) reuses it.
@@ -68,8 +73,8 @@ __device__ __forceinline__ uint32_t x_off(int r, int c) {
 
 template <bool kFp8>
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const lidx_attn_args a, float *part_o, float2 *part_ml,
-                   int n_split, uint32_t *status) {
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_win,
+                   const lidx_attn_args a, float *part_o, float2 *part_ml, int n_split, uint32_t *status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sQ = smem;
@@ -86,6 +91,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int i0 = split * kRows;
   const bool pure_window = i0 + kRows <= swa_len;
 
+  const bool tma_window = !kFp8 && pure_window;  // 128 contiguous window rows
   if (tid == 0) {
     tc::mbar_init(&sm->q_full, 1);
     tc::mbar_init(&sm->s_full, 1);
@@ -93,9 +99,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     sm->abort = 0;
     tc::fence_barrier_init();
     tc::tma_prefetch_desc(&tm_q);
-    tc::mbar_arrive_expect_tx(&sm->q_full, kQBytes);
+    tc::mbar_arrive_expect_tx(&sm->q_full, kQBytes + (tma_window ? kXBytes : 0));
 #pragma unroll
     for (int p = 0; p < 8; p++) tc::tma_load_2d(sQ + p * kQPanel, &tm_q, &sm->q_full, 64 * p, b * kH);
+    if (tma_window) {
+      const int y = static_cast<int>(static_cast<int64_t>(b) * a.swa.batch_rows + i0);
+#pragma unroll
+      for (int p = 0; p < 8; p++) tc::tma_load_2d(sX + p * kXPanel, &tm_win, &sm->q_full, 64 * p, y);
+    }
   }
   if (tid < kRows) {
     const int i = i0 + tid;
@@ -115,15 +126,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   // and zero-fills the empty ones
   auto load_rows = [&](int pass) {
     if (!kFp8) {
-      for (int idx = tid; idx < kRows * 64; idx += kThreads) {
-        const int r = idx >> 6, c = idx & 63;
+      if (pass == 0 && tma_window) return;
+      const int warp_ = tid >> 5, lane_ = tid & 31;
+      for (int r = warp_; r < kRows; r += kThreads / 32) {
         const int kind = sm->row_kind[r];
         if (pass == 0 ? kind != 2 : kind == 2) continue;
         if (kind != 0) {
           const lidx_kv &kv = kind == 1 ? a.kv : a.swa;
-          cp_async16(xs + x_off(r, c), static_cast<const uint16_t *>(kv.data) + sm->row_src[r] * kv.ld + c * 8);
+          const uint16_t *src = static_cast<const uint16_t *>(kv.data) + sm->row_src[r] * kv.ld;
+          cp_async16(xs + x_off(r, lane_), src + lane_ * 8);
+          cp_async16(xs + x_off(r, lane_ + 32), src + (lane_ + 32) * 8);
         } else {
-          *reinterpret_cast<uint4 *>(sX + x_off(r, c)) = make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4 *>(sX + x_off(r, lane_)) = make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4 *>(sX + x_off(r, lane_ + 32)) = make_uint4(0, 0, 0, 0);
         }
       }
       return;
@@ -213,8 +228,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
-  // ---- 3. softmax over the 128 rows, per head
-  const int quarter = warp & 3, half = warp >> 2;
+  // ---- 3. softmax over the 128 rows, per head: warp w covers TMEM lane
+  // quarter w&3 (rows) and heads [16g, 16g+16), g = w>>2
+  const int quarter = warp & 3, g = warp >> 2;
   const int r = quarter * 32 + lane;
   const bool valid = sm->row_kind[r] != 0;
   bool ready = false;
@@ -223,36 +239,38 @@ __global__ void __launch_bounds__(kThreads, 1)
   float s[32];
   if (ready) {
     tc::tc_fence_after();
-    tc::tmem_ld32(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + half * 32, s);
+    tc::tmem_ld32(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + (g >> 1) * 32, s);
   }
+  const bool upper = (g & 1) != 0;  // this group's heads: columns 16..31 of the load
   const float c2 = a.scale * kLog2e;
-  float mx[32];
+  float mx[16];
 #pragma unroll
-  for (int h = 0; h < 32; h++) {
-    s[h] = valid && ready ? s[h] * c2 : -INFINITY;
+  for (int h = 0; h < 16; h++) {
+    const float x = upper ? s[16 + h] : s[h];
+    s[h] = valid && ready ? x * c2 : -INFINITY;
     mx[h] = s[h];
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1)
 #pragma unroll
-    for (int h = 0; h < 32; h++) mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xFFFFFFFFu, mx[h], o));
+    for (int h = 0; h < 16; h++) mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xFFFFFFFFu, mx[h], o));
   if (lane == 0)
 #pragma unroll
-    for (int h = 0; h < 32; h++) sm->red[half][quarter][h] = mx[h];
-  named_sync(1 + half, 128);
-  float pv[32];
+    for (int h = 0; h < 16; h++) sm->red[g][quarter][h] = mx[h];
+  named_sync(1 + g, 128);
+  float pv[16];
 #pragma unroll
-  for (int h = 0; h < 32; h++) {
-    const float m = fmaxf(fmaxf(sm->red[half][0][h], sm->red[half][1][h]), fmaxf(sm->red[half][2][h], sm->red[half][3][h]));
+  for (int h = 0; h < 16; h++) {
+    const float m = fmaxf(fmaxf(sm->red[g][0][h], sm->red[g][1][h]), fmaxf(sm->red[g][2][h], sm->red[g][3][h]));
     mx[h] = m;
     pv[h] = (m == -INFINITY || s[h] == -INFINITY) ? 0.f : exp2f(s[h] - m);
   }
-  // P^T row r, heads [32*half, 32*half+32): four 16-byte chunks of 8 bf16,
-  // as hi = bf16(p) and lo = bf16(p - hi) so the PV product keeps ~16 bits
+  // P^T row r, heads [16g, 16g+16): two 16-byte chunks of 8 bf16, as
+  // hi = bf16(p) and lo = bf16(p - hi) so the PV product keeps ~16 bits
   {
     uint8_t *prow = sP + r * 128;
 #pragma unroll
-    for (int cc = 0; cc < 4; cc++) {
+    for (int cc = 0; cc < 2; cc++) {
       uint32_t oh[4], ol[4];
 #pragma unroll
       for (int i = 0; i < 4; i++) {
@@ -263,33 +281,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         oh[i] = *reinterpret_cast<const uint32_t *>(&h2);
         ol[i] = *reinterpret_cast<const uint32_t *>(&l2);
       }
-      const int chunk = half * 4 + cc;
+      const int chunk = g * 2 + cc;
       const int off = (chunk ^ (r & 7)) << 4;
       *reinterpret_cast<uint4 *>(prow + off) = make_uint4(oh[0], oh[1], oh[2], oh[3]);
       *reinterpret_cast<uint4 *>(prow + kPBytes + off) = make_uint4(ol[0], ol[1], ol[2], ol[3]);
     }
   }
-  float sum[32];
+  float sum[16];
 #pragma unroll
-  for (int h = 0; h < 32; h++) sum[h] = pv[h];
+  for (int h = 0; h < 16; h++) sum[h] = pv[h];
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1)
 #pragma unroll
-    for (int h = 0; h < 32; h++) sum[h] += __shfl_xor_sync(0xFFFFFFFFu, sum[h], o);
-  named_sync(1 + half, 128);  // everyone has read the maxima
+    for (int h = 0; h < 16; h++) sum[h] += __shfl_xor_sync(0xFFFFFFFFu, sum[h], o);
+  named_sync(1 + g, 128);  // everyone has read the maxima
   if (lane == 0)
 #pragma unroll
-    for (int h = 0; h < 32; h++) sm->red[half][quarter][h] = sum[h];
-  named_sync(1 + half, 128);
+    for (int h = 0; h < 16; h++) sm->red[g][quarter][h] = sum[h];
+  named_sync(1 + g, 128);
   if (pure_window) pdl_wait();  // no global write before the previous kernel is done
-  if (quarter == 0) {
+  if (quarter == 0 && lane < 16) {
     const int h = lane;
-    const float l = sm->red[half][0][h] + sm->red[half][1][h] + sm->red[half][2][h] + sm->red[half][3][h];
+    const float l = sm->red[g][0][h] + sm->red[g][1][h] + sm->red[g][2][h] + sm->red[g][3][h];
     float m = mx[0];
 #pragma unroll
-    for (int i = 1; i < 32; i++)
+    for (int i = 1; i < 16; i++)
       if (i == h) m = mx[i];
-    part_ml[(static_cast<size_t>(b) * n_split + split) * kH + half * 32 + h] = make_float2(m, l);
+    part_ml[(static_cast<size_t>(b) * n_split + split) * kH + g * 16 + h] = make_float2(m, l);
   }
   tc::fence_proxy_async_smem();
   tc::tc_fence_before();
@@ -315,24 +333,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::mma_commit(&sm->o_full);
   }
 
-  // ---- 5. partial O out: warps 0-3 d tiles 0,1; warps 4-7 d tiles 2,3
+  // ---- 5. partial O out: warp w stores d tile w>>2, lanes = consecutive d
   bool oready = false;
   if (lane == 0) oready = ready && tc::mbar_wait(&sm->o_full, 0, abort_flag);
   oready = __shfl_sync(0xFFFFFFFFu, oready, 0);
   if (oready) {
     tc::tc_fence_after();
     float *po = part_o + (static_cast<size_t>(b) * n_split + split) * kH * kD;
+    const int d = g * 128 + quarter * 32 + lane;
 #pragma unroll
-    for (int t2 = 0; t2 < 2; t2++) {
-      const int dt = half * 2 + t2;
-      const int d = dt * 128 + quarter * 32 + lane;
+    for (int h0 = 0; h0 < kH; h0 += 32) {
+      float v[32];
+      tc::tmem_ld32(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + 64 + 64 * g + h0, v);
 #pragma unroll
-      for (int h0 = 0; h0 < kH; h0 += 32) {
-        float v[32];
-        tc::tmem_ld32(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + 64 + 64 * dt + h0, v);
-#pragma unroll
-        for (int h = 0; h < 32; h++) po[(h0 + h) * kD + d] = v[h];
-      }
+      for (int h = 0; h < 32; h++) po[(h0 + h) * kD + d] = v[h];
     }
   }
   tc::tc_fence_before();
@@ -364,17 +378,25 @@ cudaError_t launch_attn_tc(const lidx_attn_args &a, float *part_o, float2 *part_
                     CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   const int dt = a.n_ids > 0 ? a.kv.dtype : a.swa.dtype;
+  // window rows of one chunk as one 128-row box per 64-dim panel
+  CUtensorMap tm_win = tm_q;
+  if (dt == LIDX_BF16 && a.swa_len >= kRows) {
+    const uint64_t rows = static_cast<uint64_t>(a.B - 1) * (a.B > 1 ? a.swa.batch_rows : 0) + a.swa_len;
+    if (!make_tmap_2d(&tm_win, a.swa.data, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kD, rows, a.swa.ld * 2, 64, kRows,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+  }
   const size_t smem = smem_bytes();
   dim3 grid(n_split, a.B);
   const bool pdl = (a.flags & LIDX_LAUNCH_PDL) != 0;
   cudaError_t e;
   if (dt == LIDX_E4M3) {
     cudaFuncSetAttribute(attn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    e = launch_kernel(attn_tc_kernel<true>, grid, dim3(kThreads), smem, st, pdl, tm_q, a, part_o, part_ml, n_split,
+    e = launch_kernel(attn_tc_kernel<true>, grid, dim3(kThreads), smem, st, pdl, tm_q, tm_win, a, part_o, part_ml, n_split,
                       status);
   } else {
     cudaFuncSetAttribute(attn_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    e = launch_kernel(attn_tc_kernel<false>, grid, dim3(kThreads), smem, st, pdl, tm_q, a, part_o, part_ml, n_split,
+    e = launch_kernel(attn_tc_kernel<false>, grid, dim3(kThreads), smem, st, pdl, tm_q, tm_win, a, part_o, part_ml, n_split,
                       status);
   }
   if (e != cudaSuccess) return e;
