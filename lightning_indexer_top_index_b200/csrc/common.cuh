@@ -41,6 +41,26 @@ __device__ __forceinline__ uint16_t e4m3_to_bf16_bits(uint32_t c) {
 
 __device__ __forceinline__ float e4m3_to_f32(uint32_t c) { return bf16_to_f32(e4m3_to_bf16_bits(c)); }
 
+// Two E4M3 codes (bits 0-7 and 8-15 of `codes`) -> two bf16 (low and high
+// half of the result), each multiplied by `scale`, a power of two.  Every
+// step is exact: the hardware E4M3 -> f16 conversion (all E4M3 values are f16
+// normals or zero), f16 -> f32, the power-of-two product while it stays in
+// the f32 normal range, and the final rounding to bf16 of a value with at
+// most four significant bits.  NaN codes stay NaN.
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t codes, float scale = 1.f) {
+  uint32_t h2;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(static_cast<unsigned short>(codes & 0xFFFFu)));
+  float lo, hi;
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, h;\n\t}"
+      : "=f"(lo), "=f"(hi)
+      : "r"(h2));
+  lo *= scale;
+  hi *= scale;
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
 // E8M0 scale byte -> 2^(c-127) as float (c = 0 gives 2^-127, a subnormal;
 // 255 is NaN).
 __device__ __forceinline__ float e8m0_to_f32(uint32_t c) {

@@ -248,10 +248,24 @@ __global__ void __launch_bounds__(kFp8 ? 320 : 192, 1)
     int acc = 0;
     uint32_t acc_par = 0;
     long long prev_bg = -1;
+    // E4M3 block scales of this thread's key row, loaded two units ahead so
+    // that their latency hides behind the tiles in between
+    auto load_scale = [&](long long u) -> float {
+      if (!kFp8 || u >= u1) return 0.f;
+      int b, g, t;
+      long long bg;
+      unit_coords(p, u, b, g, t, bg);
+      const int j = t * kTileM + row;
+      return j < p.N ? e8m0_to_f32(p.scale[(b * p.key_batch_rows + j) * p.ld_scale]) : 0.f;
+    };
+    float sc_next0 = load_scale(u0), sc_next1 = load_scale(u0 + 1);
     for (long long u = u0; u < u1; u++) {
       int b, g, t;
       long long bg;
       unit_coords(p, u, b, g, t, bg);
+      const float sc = sc_next0;
+      sc_next0 = sc_next1;
+      sc_next1 = load_scale(u + 2);
       if (bg != prev_bg) {
         named_sync(2, 128);
         const int nq = min(p.QG, p.Q - g * p.QG);
@@ -272,8 +286,6 @@ __global__ void __launch_bounds__(kFp8 ? 320 : 192, 1)
         const int j = t * kTileM + row;
         float v[32], r[32];
         if (kFp8) {
-          float sc = 0.f;
-          if (j < p.N) sc = e8m0_to_f32(p.scale[(b * p.key_batch_rows + j) * p.ld_scale]);
           float s = 0.f;
           for (int c0 = 0; c0 < p.H; c0 += 32) {
             tc::tmem_ld32(base + c0, v);
@@ -305,30 +317,28 @@ __global__ void __launch_bounds__(kFp8 ? 320 : 192, 1)
     }
   } else if (kFp8) {
     // ------------------------------------------------------------ FP8 -> bf16
-    const int r = threadIdx.x - 192;  // tile row
+    // Pass i: thread t converts codes [16(t%4), +16) of row 32i + t/4, so
+    // each 8-lane phase reads 128 contiguous bytes of the raw half-tile and
+    // writes 8 distinct 16-byte slots of the swizzled panel (no bank
+    // conflicts either way).
+    const int t = threadIdx.x - 192;
     int stage = 0;
     uint32_t phase = 0;
     for (long long u = u0; u < u1; u++) {
       if (!tc::mbar_wait(&bar->full[stage], phase, abort_flag)) break;
-      const uint4 *src = reinterpret_cast<const uint4 *>(sF8 + stage * kF8Bytes + r * 64);
-      uint8_t *dst = sA + stage * kTileBytes + r * 128;
+      const uint8_t *src = sF8 + stage * kF8Bytes;
+      uint8_t *dst = sA + stage * kTileBytes;
 #pragma unroll
-      for (int c = 0; c < 4; c++) {
-        const uint4 x = src[c];
+      for (int i = 0; i < 4; i++) {
+        const int r = 32 * i + (t >> 2), c = t & 3;
+        const uint4 x = *reinterpret_cast<const uint4 *>(src + r * 64 + c * 16);
         const uint32_t wv[4] = {x.x, x.y, x.z, x.w};
+        uint32_t o[8];
 #pragma unroll
-        for (int h = 0; h < 2; h++) {  // 16 FP8 bytes -> two 16-byte chunks of 8 bf16
-          uint32_t o[4];
-#pragma unroll
-          for (int i = 0; i < 4; i++) {
-            const uint32_t word = wv[h * 2 + i / 2];
-            const uint32_t lo = e4m3_to_bf16_bits((word >> (16 * (i & 1))) & 0xFFu);
-            const uint32_t hi = e4m3_to_bf16_bits((word >> (16 * (i & 1) + 8)) & 0xFFu);
-            o[i] = lo | (hi << 16);
-          }
-          const int chunk = c * 2 + h;
-          *reinterpret_cast<uint4 *>(dst + ((chunk ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-        }
+        for (int k = 0; k < 8; k++) o[k] = e4m3x2_to_bf16x2(wv[k >> 1] >> (16 * (k & 1)));
+        uint8_t *drow = dst + r * 128;
+        *reinterpret_cast<uint4 *>(drow + (((2 * c) ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+        *reinterpret_cast<uint4 *>(drow + (((2 * c + 1) ^ (r & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
       }
       tc::fence_proxy_async_smem();
       tc::mbar_arrive(&bar->conv[stage]);
