@@ -180,67 +180,49 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // Combine the split partials of one (b, h): base-2 log-sum-exp rescaling.
-// Thread t owns dims [4t, 4t+4); the split loads are independent, so they
-// overlap instead of forming a dependent chain.
+// Thread t owns dims [4t, 4t+4).  Each batch of up to 8 splits issues its
+// partial-O loads and its (m, l) loads together, then folds them in with a
+// running maximum, so a merge of <= 8 splits costs one memory round trip.
 __global__ void __launch_bounds__(128) attn_merge_kernel(lidx_attn_args a, const float *part_o,
                                                           const float2 *part_ml, int n_split) {
   pdl_trigger();
   pdl_wait();  // the partials come from the previous kernel
   const int h = blockIdx.x, b = blockIdx.y, H = a.H;
-  extern __shared__ float wgt[];  // [n_split]
-  __shared__ float inv_l, lse2;
   const float2 *ml = part_ml + static_cast<size_t>(b) * n_split * H + h;
-  if (threadIdx.x < 32) {
-    float M = -INFINITY;
-    for (int s = threadIdx.x; s < n_split; s += 32) M = fmaxf(M, ml[static_cast<size_t>(s) * H].x);
-    M = warp_max(M);
-    float L = 0.f;
-    for (int s = threadIdx.x; s < n_split; s += 32) {
-      const float2 v = ml[static_cast<size_t>(s) * H];
-      const float e = v.x == -INFINITY ? 0.f : exp2f(v.x - M);
-      wgt[s] = e;
-      L += e * v.y;
-    }
-    L = warp_sum(L);
-    if (threadIdx.x == 0) {
-      inv_l = L > 0.f ? 1.f / L : 0.f;
-      lse2 = L > 0.f ? M + log2f(L) : -INFINITY;
-    }
-  }
-  __syncthreads();
   const float4 *po = reinterpret_cast<const float4 *>(part_o + (static_cast<size_t>(b) * n_split * H + h) * kD) + threadIdx.x;
   const size_t stride4 = static_cast<size_t>(H) * kD / 4;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  int s = 0;
-  for (; s + 4 <= n_split; s += 4) {
-    float4 v[4];
+  float M = -INFINITY, L = 0.f;
+  for (int s0 = 0; s0 < n_split; s0 += 8) {
+    float4 v[8];
+    float2 w[8];
 #pragma unroll
-    for (int i = 0; i < 4; i++) v[i] = po[(s + i) * stride4];
+    for (int i = 0; i < 8; i++) {
+      if (s0 + i < n_split) {
+        w[i] = ml[static_cast<size_t>(s0 + i) * H];
+        v[i] = po[(s0 + i) * stride4];
+      }
+    }
 #pragma unroll
-    for (int i = 0; i < 4; i++) {
-      const float e = wgt[s + i];
-      if (e != 0.f) {
-        acc.x = fmaf(e, v[i].x, acc.x);
-        acc.y = fmaf(e, v[i].y, acc.y);
-        acc.z = fmaf(e, v[i].z, acc.z);
-        acc.w = fmaf(e, v[i].w, acc.w);
+    for (int i = 0; i < 8; i++) {
+      if (s0 + i < n_split && w[i].x != -INFINITY) {
+        const float mn = fmaxf(M, w[i].x);
+        const float c = exp2f(M - mn);  // 0 while M is -inf
+        const float e = exp2f(w[i].x - mn);
+        L = fmaf(L, c, e * w[i].y);
+        acc.x = fmaf(acc.x, c, e * v[i].x);
+        acc.y = fmaf(acc.y, c, e * v[i].y);
+        acc.z = fmaf(acc.z, c, e * v[i].z);
+        acc.w = fmaf(acc.w, c, e * v[i].w);
+        M = mn;
       }
     }
   }
-  for (; s < n_split; s++) {
-    const float e = wgt[s];
-    if (e != 0.f) {
-      const float4 v = po[s * stride4];
-      acc.x = fmaf(e, v.x, acc.x);
-      acc.y = fmaf(e, v.y, acc.y);
-      acc.z = fmaf(e, v.z, acc.z);
-      acc.w = fmaf(e, v.w, acc.w);
-    }
-  }
-  const float il = inv_l;
+  const float il = L > 0.f ? 1.f / L : 0.f;
   reinterpret_cast<float4 *>(a.out + (static_cast<size_t>(b) * H + h) * kD)[threadIdx.x] =
       make_float4(acc.x * il, acc.y * il, acc.z * il, acc.w * il);
-  if (threadIdx.x == 0 && a.lse) a.lse[static_cast<size_t>(b) * H + h] = lse2 * 0.6931471805599453f;
+  if (threadIdx.x == 0 && a.lse)
+    a.lse[static_cast<size_t>(b) * H + h] = L > 0.f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
 }
 
 int n_splits(const lidx_attn_args &a) {
@@ -257,7 +239,7 @@ cudaError_t launch_attn_tc(const lidx_attn_args &a, float *part_o, float2 *part_
 
 cudaError_t launch_attn_merge(const lidx_attn_args &a, const float *part_o, const float2 *part_ml, int n_split,
                               cudaStream_t st) {
-  return launch_kernel(attn_merge_kernel, dim3(a.H, a.B), dim3(128), n_split * sizeof(float), st,
+  return launch_kernel(attn_merge_kernel, dim3(a.H, a.B), dim3(128), 0, st,
                        (a.flags & LIDX_LAUNCH_PDL) != 0, a, part_o, part_ml, n_split);
 }
 
