@@ -45,7 +45,9 @@ Q_BYTES = {"f32": 4, "bf16": 2}
 
 
 def algorithmic_bytes(spec) -> dict:
-    """Inputs read once and outputs written once (intermediates excluded)."""
+    """Inputs read once and outputs written once (intermediates excluded), per
+    step, per layer, and per launch of each library call (which counts the
+    intermediates it reads or writes: scores, ids)."""
     B, N, H, k = spec.B, spec.N, spec.H, spec.k
     keys = B * N * KEY_ROW_BYTES[spec.key_dtype]
     q_idx = B * H * 128 * Q_BYTES[spec.q_dtype]
@@ -54,10 +56,15 @@ def algorithmic_bytes(spec) -> dict:
     swa = B * spec.swa * KV_ROW_BYTES[spec.kv_dtype]
     q_attn = B * H * 512 * Q_BYTES[spec.q_dtype]
     out = B * H * 512 * 4
+    scores = B * N * 4
+    ids = B * (k + 1) * 4
     layer = keys + q_idx + w + rows + swa + q_attn + out
-    # the scoring kernel itself also writes its fp32 scores
-    score_launch = keys + q_idx + w + B * N * 4
-    return dict(layer=layer, step=layer * spec.layers, score_launch=score_launch)
+    per_call = {
+        "score": keys + q_idx + w + scores,
+        "topk": scores + ids,
+        "attn": ids + rows + swa + q_attn + out + B * H * 4,
+    }
+    return dict(layer=layer, step=layer * spec.layers, per_call=per_call)
 
 
 def peaks() -> dict:
@@ -68,23 +75,31 @@ def peaks() -> dict:
     return dict(hbm_gbs=6650.0, source="fallback")
 
 
-def scorer_source_hash() -> str:
+# source files of each library call's kernels
+CALL_SOURCES = {
+    "score": ("score_tc.cu", "score_cc.cu"),
+    "topk": ("topk.cu",),
+    "attn": ("attn.cu", "attn_tc.cu"),
+}
+CALL_NAMES = {"score": "lidx_index_score", "topk": "lidx_topk_select", "attn": "lidx_sparse_attn_decode"}
+
+
+def source_hash(call: str) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "lightning_indexer_top_index_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.startswith("score") or f in ("common.cuh", "kernels.cuh", "tc.cuh"):
-            h.update(open(os.path.join(csrc, f), "rb").read())
+    for f in CALL_SOURCES[call] + ("common.cuh", "kernels.cuh", "tc.cuh"):
+        h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload: str):
-    """DRAM bytes per scorer launch from the committed ncu summary, if it was
-    taken on the current scorer source; else None."""
+def profiled_traffic(workload: str, call: str):
+    """DRAM bytes per launch of `call` from the committed ncu summary, if it
+    was taken on the current source of that call's kernels; else None."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
-    d = json.load(open(p)).get(workload)
-    if not d or d.get("source_hash") != scorer_source_hash():
+    d = json.load(open(p)).get(workload, {}).get(call)
+    if not d or d.get("source_hash") != source_hash(call):
         return None
     return d.get("dram_bytes_per_launch")
 
@@ -263,19 +278,24 @@ def run_lidx(args, spec, cfg, rank, world, local_rank):
         ms = float(t.item())
         dist.barrier()
 
-    # ---- live scorer timing: the same step with external events around each scoring launch
+    # ---- live per-call timing: the same step with external events around
+    # every library call (which also shows each call's own launch latency)
     inst = steps[0]
-    events = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
-              for _ in range(spec.layers)]
+    calls = ("score", "topk", "attn")
+    events = [{c: (torch.cuda.Event(enable_timing=True, external=True),
+                   torch.cuda.Event(enable_timing=True, external=True)) for c in calls} for _ in range(spec.layers)]
     g_inst = inst.capture(events)
-    durs = []
+    durs = {c: [] for c in calls}
     for i in range(max(3, min(args.steps, 20))):
         for r in range(1, R):
-            steps[r].replay()  # evict the instrumented replica's keys from L2 between its replays
+            steps[r].replay()  # evict the instrumented replica's caches from L2 between its replays
         g_inst.replay()
         torch.cuda.synchronize()
-        durs += [a.elapsed_time(b) for a, b in events]
-    score_ms = statistics.mean(durs)
+        for ev in events:
+            for c in calls:
+                durs[c].append(ev[c][0].elapsed_time(ev[c][1]))
+    call_ms = {c: statistics.mean(durs[c]) for c in calls}
+    del g_inst
 
     # ---- end to end: pinned host queries in, attention outputs back, every step
     q_idx_p, w_p, q_attn_p = q_idx_h.pin_memory(), w_h.pin_memory(), q_attn_h.pin_memory()
@@ -307,7 +327,8 @@ def run_lidx(args, spec, cfg, rank, world, local_rank):
 
     if rank == 0:
         pk = peaks()
-        achieved = ab["score_launch"] / (score_ms * 1e-3) / 1e9
+        dom = max(calls, key=lambda c: call_ms[c])
+        achieved = ab["per_call"][dom] / (call_ms[dom] * 1e-3) / 1e9
         line = {
             "metric": METRIC, "value": world * 1e3 / ms, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -315,9 +336,11 @@ def run_lidx(args, spec, cfg, rank, world, local_rank):
             "data": "synthetic", "config": cfg,
             "hbm_gbs_step": ab["step"] / (ms * 1e-3) / 1e9,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                         "frac": achieved / pk["hbm_gbs"], "traffic": profiled_traffic(args.workload),
-                         "kernel": "lidx_index_score", "peak_source": pk["source"],
-                         "bytes_per_launch": ab["score_launch"], "avg_launch_us": score_ms * 1e3},
+                         "frac": achieved / pk["hbm_gbs"], "traffic": profiled_traffic(args.workload, dom),
+                         "kernel": CALL_NAMES[dom], "peak_source": pk["source"],
+                         "bytes_per_launch": ab["per_call"][dom], "avg_launch_us": call_ms[dom] * 1e3},
+            "calls": {CALL_NAMES[c]: {"avg_launch_us": call_ms[c] * 1e3, "bytes_per_launch": ab["per_call"][c],
+                                      "gbs": ab["per_call"][c] / (call_ms[c] * 1e-3) / 1e9} for c in calls},
             "e2e": {"value": world * 1e3 / e2e_ms, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": args.steps * steps[0].kernel_launches(),
             "clocks": clk,

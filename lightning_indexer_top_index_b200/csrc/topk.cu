@@ -37,7 +37,7 @@ constexpr int kMaxItems = 32;
 constexpr int kMaxCluster = 8;
 constexpr int kCandLocal = 1024;   // candidates a CTA publishes
 constexpr int kGatherMax = 4096;   // candidates every CTA can gather
-constexpr int kRankMax = 1024;     // candidates resolved by direct rank counting
+constexpr int kRankMax = 96;       // candidates resolved by direct rank counting (quadratic work)
 
 // Values other CTAs of the cluster read.
 struct Pub {
@@ -70,8 +70,17 @@ __device__ __forceinline__ uint32_t cluster_rank() {
   return r;
 }
 
-__device__ __forceinline__ void cluster_sync() {
+__device__ __forceinline__ void cluster_sync_hw() {
   asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Cluster barrier; a cluster of one CTA needs only the CTA barrier (no
+// cluster-scope fence).
+__device__ __forceinline__ void cluster_sync() {
+  if (gridDim.x == 1)
+    __syncthreads();
+  else
+    cluster_sync_hw();
 }
 
 // Load a 32-bit word of CTA `rank`'s shared memory at the local address `p`.
@@ -224,32 +233,60 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelParams p) 
   pdl_trigger();
   pdl_wait();  // the scores come from the previous kernel
 
-  // ---- 0. this CTA's slice: one bulk copy into shared memory, keys into registers
+  // ---- 0. this CTA's slice: one bulk copy into shared memory, then thread t
+  // takes positions [t*C, t*C + C) of the slice into registers
   const int len = max(0, min(p.slice, a.N - s0));
   const float *s = a.scores + static_cast<size_t>(row) * a.ld_scores + s0;
   const uint8_t *al = a.allowed ? a.allowed + static_cast<size_t>(row / a.Q) * a.ld_allowed + s0 : nullptr;
-  const int head = len > 0 ? static_cast<int>(((16u - (reinterpret_cast<uintptr_t>(s) & 15u)) & 15u) / 4u) : 0;
-  const int body = max(0, len - head) & ~3;
-  float *sv = rowbuf + ((4 - head) & 3);  // the body lands 16-byte aligned
-  if (tid == 0) {
-    tc::mbar_init(&sm.bar, 1);
-    tc::fence_barrier_init();
+  float val[C];
+  {
+    const int head = len > 0 ? static_cast<int>(((16u - (reinterpret_cast<uintptr_t>(s) & 15u)) & 15u) / 4u) : 0;
+    const int body = max(0, len - head) & ~3;
+    float *sv = rowbuf + ((4 - head) & 3);  // the body lands 16-byte aligned
+    if (tid == 0) {
+      tc::mbar_init(&sm.bar, 1);
+      tc::fence_barrier_init();
+    }
+    __syncthreads();
+    if (tid == 0 && body > 0) {
+      tc::mbar_arrive_expect_tx(&sm.bar, body * 4);
+      asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                       tc::smem_u32(sv + head)),
+                   "l"(s + head), "r"(body * 4), "r"(tc::smem_u32(&sm.bar))
+                   : "memory");
+    }
+    for (int j = tid; j < len; j += kThreads)
+      if (j < head || j >= head + body) sv[j] = s[j];
+    if (body > 0) {
+      volatile uint32_t no_abort = 0;
+      if (!tc::mbar_wait(&sm.bar, 0, &no_abort)) raise_status(p.status, LIDX_DEV_TIMEOUT);
+    }
+    __syncthreads();
+    if (C >= 4 && head == 0 && p0 + C <= len) {
+      // float4 reads; step j of thread t reads its float4 number
+      // (j + t*n/8) mod n (n = C/4), so that the 8 lanes of each phase hit 8
+      // different 16-byte bank groups
+      constexpr int n = C / 4 > 0 ? C / 4 : 1;
+      const int rot = (tid * n / 8) % n;
+      const float4 *src = reinterpret_cast<const float4 *>(sv + p0);
+#pragma unroll
+      for (int j = 0; j < n; j++) {
+        const int jj = (j + rot) % n;
+        const float4 v = src[jj];
+#pragma unroll
+        for (int q = 0; q < n; q++)
+          if (q == jj) {
+            val[4 * q] = v.x;
+            val[4 * q + 1] = v.y;
+            val[4 * q + 2] = v.z;
+            val[4 * q + 3] = v.w;
+          }
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < C; i++) val[i] = p0 + i < len ? sv[p0 + i] : 0.f;
+    }
   }
-  __syncthreads();
-  if (tid == 0 && body > 0) {
-    tc::mbar_arrive_expect_tx(&sm.bar, body * 4);
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                     tc::smem_u32(sv + head)),
-                 "l"(s + head), "r"(body * 4), "r"(tc::smem_u32(&sm.bar))
-                 : "memory");
-  }
-  for (int j = tid; j < len; j += kThreads)
-    if (j < head || j >= head + body) sv[j] = s[j];
-  if (body > 0) {
-    volatile uint32_t no_abort = 0;
-    if (!tc::mbar_wait(&sm.bar, 0, &no_abort)) raise_status(p.status, LIDX_DEV_TIMEOUT);
-  }
-  __syncthreads();
   uint32_t key[C];
   uint32_t nanf = 0, elig = 0, lo = 0xFFFFFFFFu, hi = 0u;
 #pragma unroll
@@ -257,7 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelParams p) 
     const int pos = p0 + i;
     const bool in = pos < len;
     const bool ok = in && !(al && !al[pos]);
-    uint32_t kk = in ? order_key(sv[pos]) : 0u;
+    uint32_t kk = in ? order_key(val[i]) : 0u;
     nanf |= (ok && kk == 0u) ? 1u : 0u;
     kk = ok ? kk : 0u;
     key[i] = kk;
@@ -265,6 +302,159 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelParams p) 
     lo = kk ? min(lo, kk) : lo;
     hi = max(hi, kk);
   }
+  // Exact k-th key T (and the number `need` of keys equal to T to take) among
+  // the keys in_bin(i) selects, given that `rem` of the k are still to be
+  // taken from that bin.
+  uint32_t T = 0u, need = 0u;  // T = 0: take every eligible key
+  auto resolve = [&](auto in_bin, uint32_t rem) {
+    // this CTA's keys of the threshold bin
+    uint32_t nc = 0;
+#pragma unroll
+    for (int i = 0; i < C; i++) nc += in_bin(i);
+    uint32_t n_local;
+    uint32_t cpos = cta_exclusive_scan(sm, nc, n_local);
+#pragma unroll
+    for (int i = 0; i < C; i++)
+      if (in_bin(i)) {
+        if (cpos < kCandLocal) sm.pub.cand[cpos] = key[i];
+        cpos++;
+      }
+    if (tid == 0) sm.pub.n_cand = n_local;
+    cluster_sync();
+    if (tid < 32) {  // lane r reads CTA r's count
+      const uint32_t n = static_cast<uint32_t>(tid) < G ? ld_remote(&sm.pub.n_cand, tid) : 0u;
+      const uint32_t inc = warp_inclusive_scan(n);
+      const uint32_t big = __ballot_sync(0xFFFFFFFFu, n > static_cast<uint32_t>(kCandLocal));
+      if (static_cast<uint32_t>(tid) < G) sm.cand_off[tid] = inc - n;
+      if (tid == 31) {
+        sm.cand_off[kMaxCluster] = inc;
+        sm.g[0] = big;
+      }
+    }
+    __syncthreads();
+    const uint32_t n_cand = sm.cand_off[kMaxCluster];
+    const bool too_many = sm.g[0] != 0u;
+    if (!too_many && n_cand <= static_cast<uint32_t>(kGatherMax)) {
+      // gather every candidate of the cluster (the same list in every CTA):
+      // warp r copies CTA r's list
+      {
+        const int warp = tid >> 5, lane = tid & 31;
+        if (static_cast<uint32_t>(warp) < G) {
+          const uint32_t off = sm.cand_off[warp];
+          const uint32_t n = (warp + 1 < static_cast<int>(G) ? sm.cand_off[warp + 1] : n_cand) - off;
+          for (uint32_t i = lane; i < n; i += 32) sm.gathered[off + i] = ld_remote(&sm.pub.cand[i], warp);
+        }
+      }
+      __syncthreads();
+      if (n_cand <= static_cast<uint32_t>(kRankMax)) {
+        if (tid < static_cast<int>(n_cand)) {
+          const uint32_t mine = sm.gathered[tid];
+          uint32_t gt = 0, eq = 0;
+          for (uint32_t j = 0; j < n_cand; j++) {
+            const uint32_t o = sm.gathered[j];
+            gt += o > mine;
+            eq += o == mine;
+          }
+          if (gt < rem && gt + eq >= rem) {
+            sm.T = mine;
+            sm.need = rem - gt;
+          }
+        }
+        __syncthreads();
+        T = sm.T;
+        need = sm.need;
+      } else {
+        // radix over the gathered candidates' differing bits (identical in every CTA)
+        uint32_t clo = 0xFFFFFFFFu, chi = 0u;
+        for (uint32_t i = tid; i < n_cand; i += kThreads) {
+          clo = min(clo, sm.gathered[i]);
+          chi = max(chi, sm.gathered[i]);
+        }
+        clo = cta_min(sm, clo);
+        chi = cta_max(sm, chi);
+        if (clo == chi) {
+          T = clo;
+          need = rem;
+        } else {
+          int bits_left = 32 - __clz(clo ^ chi);
+          uint32_t pmask = bits_left == 32 ? 0u : ~((1u << bits_left) - 1u);
+          uint32_t prefix = clo & pmask;
+          while (bits_left > 0) {
+            const int w = min(8, bits_left);
+            const int shift = bits_left - w;
+            const uint32_t dmask = (1u << w) - 1u;
+            __syncthreads();
+            if (tid < 256) sm.hist[tid] = 0u;
+            __syncthreads();
+            for (uint32_t i = tid; i < n_cand; i += kThreads) {
+              const uint32_t kk = sm.gathered[i];
+              if ((kk & pmask) == prefix) atomicAdd(&sm.hist[(kk >> shift) & dmask], 1u);
+            }
+            find_bin(sm, 1 << w, rem);
+            prefix |= sm.digit << shift;
+            pmask |= dmask << shift;
+            rem -= sm.above;
+            bits_left -= w;
+          }
+          T = prefix;
+          need = rem;
+        }
+      }
+    } else {
+      // a bin too full to gather: cluster-wide radix levels over the
+      // candidates' differing bits, each level one exchange of histograms
+      uint32_t clo = 0xFFFFFFFFu, chi = 0u;
+#pragma unroll
+      for (int i = 0; i < C; i++)
+        if (in_bin(i)) {
+          clo = min(clo, key[i]);
+          chi = max(chi, key[i]);
+        }
+      clo = cta_min(sm, clo);
+      chi = cta_max(sm, chi);
+      if (tid == 0) {
+        sm.pub.cmin = clo;
+        sm.pub.cmax = chi;
+      }
+      cluster_sync();
+      uint32_t cmin = 0xFFFFFFFFu, cmax = 0u;
+      for (uint32_t r = 0; r < G; r++) {
+        cmin = min(cmin, ld_remote(&sm.pub.cmin, r));
+        cmax = max(cmax, ld_remote(&sm.pub.cmax, r));
+      }
+      if (cmin == cmax) {
+        T = cmin;
+        need = rem;
+      } else {
+        int bits_left = 32 - __clz(cmin ^ cmax);
+        uint32_t pmask = bits_left == 32 ? 0u : ~((1u << bits_left) - 1u);
+        uint32_t prefix = cmin & pmask;
+        int buf = 1;
+        while (bits_left > 0) {
+          const int w = min(8, bits_left);
+          const int shift = bits_left - w;
+          const uint32_t dmask = (1u << w) - 1u;
+          __syncthreads();
+          clear_whist(sm);
+          __syncthreads();
+#pragma unroll
+          for (int i = 0; i < C; i++)
+            if (in_bin(i) && (key[i] & pmask) == prefix) atomicAdd(&sm.whist[hg][(key[i] >> shift) & dmask], 1u);
+          publish_hist(sm, buf);
+          cluster_sync();
+          cluster_find(sm, buf, 1 << w, rem, G);
+          prefix |= sm.digit << shift;
+          pmask |= dmask << shift;
+          rem -= sm.above;
+          bits_left -= w;
+          buf ^= 1;
+        }
+        T = prefix;
+        need = rem;
+      }
+    }
+  };
+
   // ---- 1. cluster-wide min / max / eligible count / NaN
   {
     const int lane = tid & 31, warp = tid >> 5;
@@ -330,7 +520,6 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelParams p) 
   if (rank == 0 && tid == 0 && sm.g[3]) raise_status(p.status, LIDX_DEV_NAN);
 
   // ---- 2./3. exact k-th key T and the number `need` of keys equal to T to take
-  uint32_t T = 0u, need = 0u;  // T = 0: take every eligible key
   if (n_elig > static_cast<uint32_t>(k)) {
     uint32_t rem = static_cast<uint32_t>(k);
     if (kmin == kmax) {
@@ -356,158 +545,13 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelParams p) 
         }
         pbin[i / 4] |= b << (8 * (i % 4));
       }
-      auto in_bin = [&](int i, uint32_t d) { return key[i] != 0u && ((pbin[i / 4] >> (8 * (i % 4))) & 0xFFu) == d; };
+      auto in_lin_bin = [&](int i, uint32_t d) { return key[i] != 0u && ((pbin[i / 4] >> (8 * (i % 4))) & 0xFFu) == d; };
       publish_hist(sm, 0);
       cluster_sync();
       cluster_find(sm, 0, 256, rem, G);
       const uint32_t dbin = sm.digit;
       rem -= sm.above;
-      // this CTA's keys of the threshold bin
-      uint32_t nc = 0;
-#pragma unroll
-      for (int i = 0; i < C; i++) nc += in_bin(i, dbin);
-      uint32_t n_local;
-      uint32_t cpos = cta_exclusive_scan(sm, nc, n_local);
-#pragma unroll
-      for (int i = 0; i < C; i++)
-        if (in_bin(i, dbin)) {
-          if (cpos < kCandLocal) sm.pub.cand[cpos] = key[i];
-          cpos++;
-        }
-      if (tid == 0) sm.pub.n_cand = n_local;
-      cluster_sync();
-      if (tid < 32) {  // lane r reads CTA r's count
-        const uint32_t n = static_cast<uint32_t>(tid) < G ? ld_remote(&sm.pub.n_cand, tid) : 0u;
-        const uint32_t inc = warp_inclusive_scan(n);
-        const uint32_t big = __ballot_sync(0xFFFFFFFFu, n > static_cast<uint32_t>(kCandLocal));
-        if (static_cast<uint32_t>(tid) < G) sm.cand_off[tid] = inc - n;
-        if (tid == 31) {
-          sm.cand_off[kMaxCluster] = inc;
-          sm.g[0] = big;
-        }
-      }
-      __syncthreads();
-      const uint32_t n_cand = sm.cand_off[kMaxCluster];
-      const bool too_many = sm.g[0] != 0u;
-      if (!too_many && n_cand <= static_cast<uint32_t>(kGatherMax)) {
-        // gather every candidate of the cluster (the same list in every CTA):
-        // warp r copies CTA r's list
-        {
-          const int warp = tid >> 5, lane = tid & 31;
-          if (static_cast<uint32_t>(warp) < G) {
-            const uint32_t off = sm.cand_off[warp];
-            const uint32_t n = (warp + 1 < static_cast<int>(G) ? sm.cand_off[warp + 1] : n_cand) - off;
-            for (uint32_t i = lane; i < n; i += 32) sm.gathered[off + i] = ld_remote(&sm.pub.cand[i], warp);
-          }
-        }
-        __syncthreads();
-        if (n_cand <= static_cast<uint32_t>(kRankMax)) {
-          if (tid < static_cast<int>(n_cand)) {
-            const uint32_t mine = sm.gathered[tid];
-            uint32_t gt = 0, eq = 0;
-            for (uint32_t j = 0; j < n_cand; j++) {
-              const uint32_t o = sm.gathered[j];
-              gt += o > mine;
-              eq += o == mine;
-            }
-            if (gt < rem && gt + eq >= rem) {
-              sm.T = mine;
-              sm.need = rem - gt;
-            }
-          }
-          __syncthreads();
-          T = sm.T;
-          need = sm.need;
-        } else {
-          // radix over the gathered candidates' differing bits (identical in every CTA)
-          uint32_t clo = 0xFFFFFFFFu, chi = 0u;
-          for (uint32_t i = tid; i < n_cand; i += kThreads) {
-            clo = min(clo, sm.gathered[i]);
-            chi = max(chi, sm.gathered[i]);
-          }
-          clo = cta_min(sm, clo);
-          chi = cta_max(sm, chi);
-          if (clo == chi) {
-            T = clo;
-            need = rem;
-          } else {
-            int bits_left = 32 - __clz(clo ^ chi);
-            uint32_t pmask = bits_left == 32 ? 0u : ~((1u << bits_left) - 1u);
-            uint32_t prefix = clo & pmask;
-            while (bits_left > 0) {
-              const int w = min(8, bits_left);
-              const int shift = bits_left - w;
-              const uint32_t dmask = (1u << w) - 1u;
-              __syncthreads();
-              if (tid < 256) sm.hist[tid] = 0u;
-              __syncthreads();
-              for (uint32_t i = tid; i < n_cand; i += kThreads) {
-                const uint32_t kk = sm.gathered[i];
-                if ((kk & pmask) == prefix) atomicAdd(&sm.hist[(kk >> shift) & dmask], 1u);
-              }
-              find_bin(sm, 1 << w, rem);
-              prefix |= sm.digit << shift;
-              pmask |= dmask << shift;
-              rem -= sm.above;
-              bits_left -= w;
-            }
-            T = prefix;
-            need = rem;
-          }
-        }
-      } else {
-        // a bin too full to gather: cluster-wide radix levels over the
-        // candidates' differing bits, each level one exchange of histograms
-        uint32_t clo = 0xFFFFFFFFu, chi = 0u;
-#pragma unroll
-        for (int i = 0; i < C; i++)
-          if (in_bin(i, dbin)) {
-            clo = min(clo, key[i]);
-            chi = max(chi, key[i]);
-          }
-        clo = cta_min(sm, clo);
-        chi = cta_max(sm, chi);
-        if (tid == 0) {
-          sm.pub.cmin = clo;
-          sm.pub.cmax = chi;
-        }
-        cluster_sync();
-        uint32_t cmin = 0xFFFFFFFFu, cmax = 0u;
-        for (uint32_t r = 0; r < G; r++) {
-          cmin = min(cmin, ld_remote(&sm.pub.cmin, r));
-          cmax = max(cmax, ld_remote(&sm.pub.cmax, r));
-        }
-        if (cmin == cmax) {
-          T = cmin;
-          need = rem;
-        } else {
-          int bits_left = 32 - __clz(cmin ^ cmax);
-          uint32_t pmask = bits_left == 32 ? 0u : ~((1u << bits_left) - 1u);
-          uint32_t prefix = cmin & pmask;
-          int buf = 1;
-          while (bits_left > 0) {
-            const int w = min(8, bits_left);
-            const int shift = bits_left - w;
-            const uint32_t dmask = (1u << w) - 1u;
-            __syncthreads();
-            clear_whist(sm);
-            __syncthreads();
-#pragma unroll
-            for (int i = 0; i < C; i++)
-              if (in_bin(i, dbin) && (key[i] & pmask) == prefix) atomicAdd(&sm.whist[hg][(key[i] >> shift) & dmask], 1u);
-            publish_hist(sm, buf);
-            cluster_sync();
-            cluster_find(sm, buf, 1 << w, rem, G);
-            prefix |= sm.digit << shift;
-            pmask |= dmask << shift;
-            rem -= sm.above;
-            bits_left -= w;
-            buf ^= 1;
-          }
-          T = prefix;
-          need = rem;
-        }
-      }
+      resolve([&](int i) { return in_lin_bin(i, dbin); }, rem);
     }
   }
 
@@ -545,7 +589,8 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelParams p) 
   eq_before += ex & 0xFFFFu;
   uint32_t out = gt_before + min(eq_before, need);
   uint32_t eq_rank = eq_before;
-  const uint32_t n_out = gt_total + min(eq_total, need);
+  // never more than k ids, whatever the counts above say
+  const uint32_t n_out = min(gt_total + min(eq_total, need), static_cast<uint32_t>(a.k));
   int32_t *ids = a.ids + static_cast<size_t>(row) * a.k;
   uint32_t selbits = 0;
 #pragma unroll
@@ -562,7 +607,8 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelParams p) 
       }
     }
     if (sel) {
-      ids[out++] = s0 + p0 + i;
+      if (out < static_cast<uint32_t>(a.k)) ids[out] = s0 + p0 + i;
+      out++;
       selbits |= 1u << i;
     }
   }

@@ -68,27 +68,29 @@ class DecodeStep:
 
     # ------------------------------------------------------------------ run
     def enqueue(self, stream=None, events: Optional[List] = None):
-        """Issue the step's library calls on `stream`.  With `events` (a list of
-        (start, end) external CUDA events per layer), bracket each layer's
-        scoring call for timing."""
+        """Issue the step's library calls on `stream`.  With `events` (per layer
+        a dict mapping "score", "topk" or "attn" to a (start, end) pair of
+        external CUDA events), bracket those calls for timing."""
         st = C.c_void_p((stream or torch.cuda.current_stream()).cuda_stream)
         lb = self._lib
+
+        def call(l, name, fn, *a):
+            ev = events[l].get(name) if events is not None else None
+            if ev is not None:
+                ev[0].record()
+            rc = fn(*a)
+            if ev is not None:
+                ev[1].record()
+            if rc:
+                raise LidxError(rc, fn.__name__)
+
         for l in range(self.L):
-            if events is not None:
-                events[l][0].record()
-            rc = lb.lidx_index_score(C.byref(self._score[l]), st)
-            if events is not None:
-                events[l][1].record()
-            if rc:
-                raise LidxError(rc, "lidx_index_score")
+            call(l, "score", lb.lidx_index_score, C.byref(self._score[l]), st)
             wt = self._ws_topk[l]
-            rc = lb.lidx_topk_select(C.byref(self._topk[l]), C.c_void_p(wt.data_ptr()), wt.numel(), st)
-            if rc:
-                raise LidxError(rc, "lidx_topk_select")
+            call(l, "topk", lb.lidx_topk_select, C.byref(self._topk[l]), C.c_void_p(wt.data_ptr()), wt.numel(), st)
             wa = self._ws_attn[l]
-            rc = lb.lidx_sparse_attn_decode(C.byref(self._attn[l]), C.c_void_p(wa.data_ptr()), wa.numel(), st)
-            if rc:
-                raise LidxError(rc, "lidx_sparse_attn_decode")
+            call(l, "attn", lb.lidx_sparse_attn_decode, C.byref(self._attn[l]), C.c_void_p(wa.data_ptr()), wa.numel(),
+                 st)
 
     def capture(self, events: Optional[List] = None) -> torch.cuda.CUDAGraph:
         """Record one step into a CUDA graph (the library calls only)."""
