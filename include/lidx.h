@@ -39,7 +39,7 @@
 extern "C" {
 #endif
 
-#define LIDX_ABI_VERSION 2
+#define LIDX_ABI_VERSION 3
 
 #if defined(__GNUC__)
 #define LIDX_API __attribute__((visibility("default")))
@@ -113,9 +113,22 @@ typedef struct lidx_kv {
  *   w       [B][Q][H] fp32 (any sign)
  *   keys    dim 128
  *   scores  [B][Q][ld_scores] fp32, ld_scores >= N; entries j >= N untouched
+ *   tile_stats  optional [B][Q][ceil(N/LIDX_STATS_SPAN)][2] uint32, 8-byte
+ *           aligned: the score bounds lidx_topk_select can start from (see
+ *           LIDX_STATS_SPAN)
  * Returns INVALID_ARG for null pointers / non-positive sizes / misaligned
  * planes, UNSUPPORTED for other format combinations.
  * ------------------------------------------------------------------------ */
+
+/* Score bounds per span of 32 entries (optional side output of
+ * lidx_index_score, input of lidx_topk_select).  For score row (b,t) and span
+ * i, entry [i][0] is the largest and [i][1] the smallest order-preserving key
+ * of the non-NaN scores j in [32i, min(32i+32, N)), or (0, 0xFFFFFFFF) when
+ * the span has none.  The key of a score s with IEEE bits u (-0 taken as +0)
+ * is u | 0x80000000 for s >= 0 and ~u for s < 0, so larger scores have larger
+ * keys.  With them the top-k reads the row's score range instead of
+ * exchanging it among its CTAs. */
+#define LIDX_STATS_SPAN 32
 typedef struct lidx_score_args {
     int32_t B, Q, H, N;
     int32_t q_dtype;
@@ -124,7 +137,8 @@ typedef struct lidx_score_args {
     lidx_kv keys;
     float *scores;
     int64_t ld_scores;
-    uint32_t flags; /* LIDX_LAUNCH_* */
+    uint32_t flags;       /* LIDX_LAUNCH_* */
+    uint32_t *tile_stats; /* optional score bounds, see LIDX_STATS_SPAN */
 } lidx_score_args;
 
 LIDX_API lidx_status lidx_index_score(const lidx_score_args *args, void *stream);
@@ -142,6 +156,9 @@ LIDX_API lidx_status lidx_index_score(const lidx_score_args *args, void *stream)
  *   n_sel   [B][Q] int32 (optional): min(k, #eligible)
  *   mask    [B][Q][N] uint8 (optional): 1 for selected entries (comp_allowed)
  *   mask_bits [B][Q][ceil(N/32)] uint32 (optional): bit j%32 of word j/32
+ *   tile_stats optional: the score bounds lidx_index_score wrote for exactly
+ *           these scores (LIDX_STATS_SPAN).  Bounds that do not hold give
+ *           wrong ids but never a write outside ids[b][t][0..k).
  * Needs a workspace of lidx_workspace_size(LIDX_OP_TOPK).
  * ------------------------------------------------------------------------ */
 typedef struct lidx_topk_args {
@@ -154,7 +171,8 @@ typedef struct lidx_topk_args {
     int32_t *n_sel;
     uint8_t *mask;
     uint32_t *mask_bits;
-    uint32_t flags; /* LIDX_LAUNCH_* */
+    uint32_t flags;             /* LIDX_LAUNCH_* */
+    const uint32_t *tile_stats; /* optional score bounds, see LIDX_STATS_SPAN */
 } lidx_topk_args;
 
 LIDX_API lidx_status lidx_topk_select(const lidx_topk_args *args, void *ws, size_t ws_bytes, void *stream);

@@ -30,6 +30,7 @@ DTYPES = {"f32": F32, "bf16": BF16, "e4m3": E4M3, "f16": F16}
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_WORKSPACE = 0, 1, 2, 3, 4
 DEV_BOUNDS, DEV_NAN, DEV_TIMEOUT = 0x1, 0x2, 0x4
 LAUNCH_PDL = 0x1
+STATS_SPAN = 32  # entries per score-bounds record (optional scorer output, top-k input)
 
 EVAL_GOLDEN, EVAL_TOPP, EVAL_VOTE, EVAL_LSA, EVAL_OVERLAP = 0x1, 0x2, 0x4, 0x8, 0x10
 OP_SCORE, OP_TOPK, OP_ATTN, OP_EVAL = 0, 1, 2, 3
@@ -68,14 +69,14 @@ class KVArgs(C.Structure):
 class ScoreArgs(C.Structure):
     _fields_ = [("B", C.c_int32), ("Q", C.c_int32), ("H", C.c_int32), ("N", C.c_int32),
                 ("q_dtype", C.c_int32), ("q", C.c_void_p), ("w", C.c_void_p), ("keys", KVArgs),
-                ("scores", C.c_void_p), ("ld_scores", C.c_int64), ("flags", C.c_uint32)]
+                ("scores", C.c_void_p), ("ld_scores", C.c_int64), ("flags", C.c_uint32), ("tile_stats", C.c_void_p)]
 
 
 class TopkArgs(C.Structure):
     _fields_ = [("B", C.c_int32), ("Q", C.c_int32), ("N", C.c_int32), ("k", C.c_int32),
                 ("scores", C.c_void_p), ("ld_scores", C.c_int64), ("allowed", C.c_void_p),
                 ("ld_allowed", C.c_int64), ("ids", C.c_void_p), ("n_sel", C.c_void_p), ("mask", C.c_void_p),
-                ("mask_bits", C.c_void_p), ("flags", C.c_uint32)]
+                ("mask_bits", C.c_void_p), ("flags", C.c_uint32), ("tile_stats", C.c_void_p)]
 
 
 class AttnArgs(C.Structure):
@@ -213,17 +214,19 @@ def _qdtype(t: torch.Tensor) -> int:
 
 # ---------------------------------------------------------------- the calls
 def index_score(q: torch.Tensor, w: torch.Tensor, keys: DeviceKV, N: int, scores: torch.Tensor = None,
-                stream=None) -> torch.Tensor:
+                stream=None, tile_stats: torch.Tensor = None) -> torch.Tensor:
     """scores[b,t,j] = sum_h w[b,t,h] * max(q[b,t,h] . keys[b,j], 0).
 
     q [B][Q][H][128] (float32 or bfloat16), w [B][Q][H] float32 -> scores
-    float32 [B][Q][N] (or the given tensor with a row stride >= N)."""
+    float32 [B][Q][N] (or the given tensor with a row stride >= N).  With
+    `tile_stats` (int32 [B][Q][ceil(N/STATS_SPAN)][2]) the call also writes
+    the score bounds topk_select can start from."""
     B, Q, H, D = q.shape
     assert q.is_contiguous() and w.is_contiguous() and w.dtype == torch.float32
     if scores is None:
         scores = torch.empty((B, Q, N), dtype=torch.float32, device=q.device)
     a = ScoreArgs(B, Q, H, N, _qdtype(q), q.data_ptr(), w.data_ptr(), keys.args(), scores.data_ptr(),
-                  scores.stride(1))
+                  scores.stride(1), 0, _ptr(tile_stats))
     _check(lib().lidx_index_score(C.byref(a), _stream(stream)), "lidx_index_score")
     return scores
 
@@ -239,26 +242,28 @@ def workspace(nbytes: int, device="cuda") -> torch.Tensor:
     return torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=device)
 
 
-def topk_args(scores, k, allowed=None, ids=None, n_sel=None, mask=None, mask_bits=None, flags=0) -> TopkArgs:
+def topk_args(scores, k, allowed=None, ids=None, n_sel=None, mask=None, mask_bits=None, flags=0,
+              tile_stats=None) -> TopkArgs:
     B, Q, N = scores.shape[0], scores.shape[1], scores.shape[2]
     return TopkArgs(B, Q, N, k, scores.data_ptr(), scores.stride(1), _ptr(allowed),
                     0 if allowed is None else allowed.stride(0), _ptr(ids), _ptr(n_sel), _ptr(mask),
-                    _ptr(mask_bits), flags)
+                    _ptr(mask_bits), flags, _ptr(tile_stats))
 
 
 def topk_select(scores: torch.Tensor, k: int, allowed: torch.Tensor = None, *, want_mask=False,
-                want_bits=False, ids=None, n_sel=None, ws=None, stream=None):
+                want_bits=False, ids=None, n_sel=None, ws=None, stream=None, tile_stats=None):
     """Top-k row ids of scores [B][Q][N] (N = scores.shape[2]).
 
     Returns (ids int32 [B][Q][k] ascending with -1 padding, n_sel int32 [B][Q],
-    mask uint8 [B][Q][N] or None, bits uint32 [B][Q][ceil(N/32)] or None)."""
+    mask uint8 [B][Q][N] or None, bits uint32 [B][Q][ceil(N/32)] or None).
+    `tile_stats` are the score bounds index_score wrote for these scores."""
     B, Q, N = scores.shape
     dev = scores.device
     ids = torch.empty((B, Q, k), dtype=torch.int32, device=dev) if ids is None else ids
     n_sel = torch.empty((B, Q), dtype=torch.int32, device=dev) if n_sel is None else n_sel
     mask = torch.empty((B, Q, N), dtype=torch.uint8, device=dev) if want_mask else None
     bits = torch.empty((B, Q, (N + 31) // 32), dtype=torch.int32, device=dev) if want_bits else None
-    a = topk_args(scores, k, allowed, ids, n_sel, mask, bits)
+    a = topk_args(scores, k, allowed, ids, n_sel, mask, bits, tile_stats=tile_stats)
     if ws is None:
         ws = workspace(workspace_size(OP_TOPK, a), dev)
     _check(lib().lidx_topk_select(C.byref(a), C.c_void_p(ws.data_ptr()), ws.numel(), _stream(stream)),

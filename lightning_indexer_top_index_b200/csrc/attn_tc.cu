@@ -24,15 +24,7 @@
 //   4. MMA 2: O^T[d][head] = X^T . P^T, reading the same X tile as an
 //      MN-major operand (K = V), four 128-wide d tiles (N = 16) into TMEM.
 //   5. Each warp stores two d tiles, lanes = consecutive d: coalesced stores.
-// When a sequence's row list spans at most 16 chunks, the chunks of one head
-// group run as one thread-block cluster and combine their partials through
-// distributed shared memory: each CTA parks its O^T and (m, l) in its own
-// shared memory, and after a cluster barrier CTA r rescales and sums slice r
-// of the 16 x 512 outputs over all CTAs of the cluster and writes the final
-// rows (no partials in global memory, no merge launch).  Longer lists store
-// the partials and the split-K merge kernel combines them.
-#include <atomic>
-
+// The partials are combined by the split-K merge kernel.
 #include "kernels.cuh"
 #include "tc.cuh"
 
@@ -55,7 +47,6 @@ constexpr int kQBytes = kHG * kD * 2;        // 16 KB: 8 panels of [16 heads][12
 constexpr int kQPanel = kHG * 128;           // 2 KB
 constexpr int kPBytes = kHG * kRows * 2;     // 2 KB: one bf16 P^T [16 heads][64 rows]
 constexpr uint32_t kTmemCols = 128;          // S^T at [0,16), O^T tile t at [32+16t, 48+16t)
-constexpr int kMaxCluster = 16;              // chunks combined in one cluster (non-portable size)
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct __align__(8) AttnTcSmem {
@@ -67,11 +58,6 @@ struct __align__(8) AttnTcSmem {
   int64_t row_src[kRows];  // row index in its cache; -1 when empty
   int32_t row_kind[kRows]; // 0 none, 1 selected, 2 window
   float red[2][2][8];      // per head half, per warp of the pair
-  // cluster combine
-  float2 ml[kHG];                  // this CTA's (m, l) per head, base 2
-  float2 all_ml[kMaxCluster][kHG]; // every CTA's (m, l), gathered
-  float wgt[kMaxCluster][kHG];     // 2^(m_c - M) per CTA and head
-  float inv_l[kHG], lse2[kHG];
 };
 
 // smem: X (64 KB) | Q (16 KB) | P^T hi, lo (2 x 2 KB) | bookkeeping.  Q
@@ -86,36 +72,12 @@ __device__ __forceinline__ void cp_async_wait_all() {
 }
 __device__ __forceinline__ void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n)); }
 
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ void cluster_barrier() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-__device__ __forceinline__ uint32_t remote_addr(const void *p, uint32_t rank) {
-  uint32_t a;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(tc::smem_u32(p)), "r"(rank));
-  return a;
-}
-__device__ __forceinline__ float4 ld_remote_f4(uint32_t addr) {
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0,%1,%2,%3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
-  return v;
-}
-__device__ __forceinline__ float2 ld_remote_f2(uint32_t addr) {
-  float2 v;
-  asm volatile("ld.shared::cluster.v2.f32 {%0,%1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
-  return v;
-}
-
 // byte offset of dims [8c, 8c+8) of row r inside the 64-row K-major swizzled tile
 __device__ __forceinline__ uint32_t x_off(int r, int c) {
   return (c >> 3) * kXPanel + r * 128 + (((c & 7) ^ (r & 7)) << 4);
 }
 
-template <bool kFp8, bool kFused>
+template <bool kFp8>
 __global__ void __launch_bounds__(kThreads, 2)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_win,
                    const lidx_attn_args a, float *part_o, float2 *part_ml, int n_split, uint32_t *status) {
@@ -330,10 +292,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
       for (int i = 1; i < 8; i++)
         if (i == lane) m = mx[i];
-      if (kFused)
-        sm->ml[half * 8 + lane] = ready ? make_float2(m, l) : make_float2(-INFINITY, 0.f);
-      else
-        part_ml[(static_cast<size_t>(b) * n_split + split) * kH + hg * kHG + half * 8 + lane] = make_float2(m, l);
+      part_ml[(static_cast<size_t>(b) * n_split + split) * kH + hg * kHG + half * 8 + lane] = make_float2(m, l);
     }
   }
   tc::fence_proxy_async_smem();
@@ -365,12 +324,9 @@ __global__ void __launch_bounds__(kThreads, 2)
   bool oready = false;
   if (lane == 0) oready = !*abort_flag && tc::mbar_wait(&sm->o_full, 0, abort_flag);
   oready = __shfl_sync(0xFFFFFFFFu, oready, 0);
-  // fused: O^T lands in this CTA's shared memory (the X tile is dead) as
-  // [16 heads][512 d]; otherwise in the global partials
-  float *po = kFused ? reinterpret_cast<float *>(sX)
-                     : part_o + ((static_cast<size_t>(b) * n_split + split) * kH + hg * kHG) * kD;
   if (oready) {
     tc::tc_fence_after();
+    float *po = part_o + ((static_cast<size_t>(b) * n_split + split) * kH + hg * kHG) * kD;
 #pragma unroll
     for (int j = 0; j < 2; j++) {
       const int dt = (warp >> 2) + 2 * j;
@@ -380,9 +336,6 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
       for (int h = 0; h < kHG; h++) po[h * kD + d] = v[h];
     }
-  } else if (kFused && tid == 0) {
-#pragma unroll
-    for (int h = 0; h < kHG; h++) sm->ml[h] = make_float2(-INFINITY, 0.f);  // contributes nothing
   }
   tc::tc_fence_before();
   __syncthreads();
@@ -391,125 +344,6 @@ __global__ void __launch_bounds__(kThreads, 2)
     tc::tmem_dealloc(tmem, kTmemCols);
   }
   if (tid == 0 && sm->abort) raise_status(status, LIDX_DEV_TIMEOUT);
-
-  if (kFused) {
-    // ---- 6. cluster combine: CTA r owns outputs [r*S, r*S + S) of the
-    // 16 x 512 (head, d) block; every CTA's O and (m, l) are read over DSMEM
-    const int n = static_cast<int>(gridDim.x);  // the cluster spans the row chunks
-    const uint32_t rank = cluster_ctarank();
-    cluster_barrier();
-    if (tid < kHG * n) {
-      const int c = tid / kHG, h = tid % kHG;
-      sm->all_ml[c][h] = ld_remote_f2(remote_addr(&sm->ml[h], c));
-    }
-    __syncthreads();
-    if (tid < kHG) {
-      float M = -INFINITY;
-      for (int c = 0; c < n; c++) M = fmaxf(M, sm->all_ml[c][tid].x);
-      float Lsum = 0.f;
-      for (int c = 0; c < n; c++) {
-        const float2 v = sm->all_ml[c][tid];
-        const float w = v.x == -INFINITY ? 0.f : exp2f(v.x - M);
-        sm->wgt[c][tid] = w;
-        Lsum += w * v.y;
-      }
-      sm->inv_l[tid] = Lsum > 0.f ? 1.f / Lsum : 0.f;
-      sm->lse2[tid] = Lsum > 0.f ? M + log2f(Lsum) : -INFINITY;
-    }
-    __syncthreads();
-    constexpr int kF4 = kHG * kD / 4;        // float4 outputs of the block
-    const int per = (kF4 + n - 1) / n;
-    const int f0 = static_cast<int>(rank) * per, f1 = min(kF4, f0 + per);
-    float *out = a.out + (static_cast<size_t>(b) * kH + hg * kHG) * kD;
-    for (int f = f0 + tid; f < f1; f += kThreads) {
-      const int h = (4 * f) / kD;
-      float4 v[kMaxCluster];
-#pragma unroll
-      for (int c = 0; c < kMaxCluster; c++)
-        if (c < n) v[c] = ld_remote_f4(remote_addr(po + 4 * f, c));
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int c = 0; c < kMaxCluster; c++) {
-        const float w = c < n ? sm->wgt[c][h] : 0.f;
-        if (w != 0.f) {
-          acc.x = fmaf(w, v[c].x, acc.x);
-          acc.y = fmaf(w, v[c].y, acc.y);
-          acc.z = fmaf(w, v[c].z, acc.z);
-          acc.w = fmaf(w, v[c].w, acc.w);
-        }
-      }
-      const float il = sm->inv_l[h];
-      reinterpret_cast<float4 *>(out)[f] = make_float4(acc.x * il, acc.y * il, acc.z * il, acc.w * il);
-    }
-    if (rank == 0 && tid < kHG && a.lse)
-      a.lse[static_cast<size_t>(b) * kH + hg * kHG + tid] = sm->lse2[tid] * 0.6931471805599453f;
-    cluster_barrier();  // keep this CTA's shared memory until every CTA has read it
-  }
-}
-
-}  // namespace
-
-namespace {
-
-// Whether clusters of n chunk-CTAs fit on the device (cached per variant).
-template <bool kFp8>
-bool cluster_fits(int n, size_t smem) {
-  static std::atomic<int> cache[kMaxCluster + 1];  // 0 unknown, 1 yes, 2 no
-  if (n < 1 || n > kMaxCluster) return false;
-  int c = cache[n].load(std::memory_order_relaxed);
-  if (c == 0) {
-    auto kern = attn_tc_kernel<kFp8, true>;
-    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (n > 8) cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(n, kGroups, 1);
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = smem;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = n;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int clusters = 0;
-    const cudaError_t e = cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg);
-    if (e != cudaSuccess) cudaGetLastError();  // clear; fall back to the merge kernel
-    c = (e == cudaSuccess && clusters > 0) ? 1 : 2;
-    cache[n].store(c, std::memory_order_relaxed);
-  }
-  return c == 1;
-}
-
-template <bool kFp8>
-cudaError_t launch_variant(const CUtensorMap &tm_q, const CUtensorMap &tm_win, const lidx_attn_args &a, float *part_o,
-                           float2 *part_ml, int n_split, uint32_t *status, cudaStream_t st, bool pdl, size_t smem,
-                           bool &fused) {
-  fused = cluster_fits<kFp8>(n_split, smem);
-  auto kern = fused ? attn_tc_kernel<kFp8, true> : attn_tc_kernel<kFp8, false>;
-  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(n_split, kGroups, a.B);
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[2];
-  int na = 0;
-  if (fused) {
-    attr[na].id = cudaLaunchAttributeClusterDimension;
-    attr[na].val.clusterDim.x = n_split;
-    attr[na].val.clusterDim.y = 1;
-    attr[na].val.clusterDim.z = 1;
-    na++;
-  }
-  if (pdl) {
-    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[na].val.programmaticStreamSerializationAllowed = 1;
-    na++;
-  }
-  cfg.attrs = attr;
-  cfg.numAttrs = na;
-  return cudaLaunchKernelEx(&cfg, kern, tm_q, tm_win, a, part_o, part_ml, n_split, status);
 }
 
 }  // namespace
@@ -541,14 +375,19 @@ cudaError_t launch_attn_tc(const lidx_attn_args &a, float *part_o, float2 *part_
       return cudaErrorInvalidValue;
   }
   const size_t smem = smem_bytes();
+  dim3 grid(n_split, kGroups, a.B);
   const bool pdl = (a.flags & LIDX_LAUNCH_PDL) != 0;
   cudaError_t e;
-  bool fused = false;
-  if (dt == LIDX_E4M3)
-    e = launch_variant<true>(tm_q, tm_win, a, part_o, part_ml, n_split, status, st, pdl, smem, fused);
-  else
-    e = launch_variant<false>(tm_q, tm_win, a, part_o, part_ml, n_split, status, st, pdl, smem, fused);
-  if (e != cudaSuccess || fused) return e;
+  if (dt == LIDX_E4M3) {
+    cudaFuncSetAttribute(attn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    e = launch_kernel(attn_tc_kernel<true>, grid, dim3(kThreads), smem, st, pdl, tm_q, tm_win, a, part_o, part_ml, n_split,
+                      status);
+  } else {
+    cudaFuncSetAttribute(attn_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    e = launch_kernel(attn_tc_kernel<false>, grid, dim3(kThreads), smem, st, pdl, tm_q, tm_win, a, part_o, part_ml, n_split,
+                      status);
+  }
+  if (e != cudaSuccess) return e;
   return launch_attn_merge(a, part_o, part_ml, n_split, st);
 }
 

@@ -58,6 +58,7 @@ lidx_status check_score(const lidx_score_args *a) {
   if (a->keys.dtype == LIDX_F32 && a->q_dtype != LIDX_F32) return LIDX_ERR_UNSUPPORTED;
   if (a->keys.dtype != LIDX_F32 && a->q_dtype != LIDX_BF16) return LIDX_ERR_UNSUPPORTED;
   if (!aligned(a->q, 4) || !aligned(a->w, 4) || !aligned(a->scores, 4)) return LIDX_ERR_INVALID_ARG;
+  if (a->tile_stats && !aligned(a->tile_stats, 8)) return LIDX_ERR_INVALID_ARG;
   return LIDX_OK;
 }
 
@@ -67,6 +68,7 @@ lidx_status check_topk(const lidx_topk_args *a) {
   if (a->allowed && a->ld_allowed < a->N) return LIDX_ERR_INVALID_ARG;
   if (!aligned(a->scores, 4) || !aligned(a->ids, 4) || (a->mask_bits && !aligned(a->mask_bits, 4)))
     return LIDX_ERR_INVALID_ARG;
+  if (a->tile_stats && !aligned(a->tile_stats, 8)) return LIDX_ERR_INVALID_ARG;
   if (!topk_supported(*a)) return LIDX_ERR_UNSUPPORTED;
   return LIDX_OK;
 }

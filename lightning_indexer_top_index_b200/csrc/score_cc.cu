@@ -73,31 +73,42 @@ __global__ void __launch_bounds__(kThreads) score_cc_kernel(lidx_score_args a, i
   for (int i = threadIdx.x; i < Hp; i += kThreads) w_s[i] = i < a.H ? a.w[static_cast<size_t>(bt) * a.H + i] : 0.f;
   __syncthreads();
   const int j = blockIdx.x * kThreads + threadIdx.x;
-  if (j >= a.N) return;
-  const int64_t row = static_cast<int64_t>(b) * a.keys.batch_rows + j;
+  const bool valid = j < a.N;
   float score = 0.f;
-  for (int h0 = 0; h0 < Hp; h0 += HG) {
-    float acc[HG];
+  if (valid) {
+    const int64_t row = static_cast<int64_t>(b) * a.keys.batch_rows + j;
+    for (int h0 = 0; h0 < Hp; h0 += HG) {
+      float acc[HG];
 #pragma unroll
-    for (int i = 0; i < HG; i++) acc[i] = 0.f;
+      for (int i = 0; i < HG; i++) acc[i] = 0.f;
 #pragma unroll 1
-    for (int d0 = 0; d0 < kD; d0 += 8) {
-      float kv[8];
-      load8<KT>(a.keys, row, d0, kv);
+      for (int d0 = 0; d0 < kD; d0 += 8) {
+        float kv[8];
+        load8<KT>(a.keys, row, d0, kv);
 #pragma unroll
-      for (int hh = 0; hh < HG; hh++) {
-        const float4 *qp = reinterpret_cast<const float4 *>(q_s + (h0 + hh) * kD + d0);
-        float4 x = qp[0], y = qp[1];
-        float s = acc[hh];
-        s = fmaf(x.x, kv[0], s); s = fmaf(x.y, kv[1], s); s = fmaf(x.z, kv[2], s); s = fmaf(x.w, kv[3], s);
-        s = fmaf(y.x, kv[4], s); s = fmaf(y.y, kv[5], s); s = fmaf(y.z, kv[6], s); s = fmaf(y.w, kv[7], s);
-        acc[hh] = s;
+        for (int hh = 0; hh < HG; hh++) {
+          const float4 *qp = reinterpret_cast<const float4 *>(q_s + (h0 + hh) * kD + d0);
+          float4 x = qp[0], y = qp[1];
+          float s = acc[hh];
+          s = fmaf(x.x, kv[0], s); s = fmaf(x.y, kv[1], s); s = fmaf(x.z, kv[2], s); s = fmaf(x.w, kv[3], s);
+          s = fmaf(y.x, kv[4], s); s = fmaf(y.y, kv[5], s); s = fmaf(y.z, kv[6], s); s = fmaf(y.w, kv[7], s);
+          acc[hh] = s;
+        }
       }
-    }
 #pragma unroll
-    for (int hh = 0; hh < HG; hh++) score = fmaf(w_s[h0 + hh], fmaxf(acc[hh], 0.f), score);
+      for (int hh = 0; hh < HG; hh++) score = fmaf(w_s[h0 + hh], fmaxf(acc[hh], 0.f), score);
+    }
+    a.scores[static_cast<size_t>(bt) * a.ld_scores + j] = score;
   }
-  a.scores[static_cast<size_t>(bt) * a.ld_scores + j] = score;
+  if (a.tile_stats) {  // score bounds of this warp's span of 32 entries (whole warps)
+    const uint32_t kk = valid ? order_key(score) : 0u;
+    const uint32_t mx = __reduce_max_sync(0xFFFFFFFFu, kk);
+    const uint32_t mn = __reduce_min_sync(0xFFFFFFFFu, kk ? kk : 0xFFFFFFFFu);
+    const int j0 = j & ~31;
+    const int n_spans = (a.N + LIDX_STATS_SPAN - 1) / LIDX_STATS_SPAN;
+    if ((threadIdx.x & 31) == 0 && j0 < a.N)
+      reinterpret_cast<uint2 *>(a.tile_stats)[static_cast<size_t>(bt) * n_spans + j0 / 32] = make_uint2(mx, mn);
+  }
 }
 
 template <int KT>

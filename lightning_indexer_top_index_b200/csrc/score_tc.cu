@@ -49,6 +49,8 @@ struct TcParams {
   const float *w;
   const uint8_t *scale;
   int64_t ld_scale;
+  uint32_t *stats;    // optional score bounds per span of 32 entries
+  int n_spans;
   uint32_t *status;
 };
 
@@ -259,6 +261,17 @@ __global__ void __launch_bounds__(kFp8 ? 320 : 192, 1)
       return j < p.N ? e8m0_to_f32(p.scale[(b * p.key_batch_rows + j) * p.ld_scale]) : 0.f;
     };
     float sc_next0 = load_scale(u0), sc_next1 = load_scale(u0 + 1);
+    // Score bounds of this warp's 32 keys of a tile (one span record), for the
+    // top-k: the largest and the smallest non-NaN order key.  Called by whole
+    // warps.
+    auto span_stats = [&](float sv, bool valid, int srow, int t) {
+      const uint32_t kk = valid ? order_key(sv) : 0u;
+      const uint32_t mx = __reduce_max_sync(0xFFFFFFFFu, kk);
+      const uint32_t mn = __reduce_min_sync(0xFFFFFFFFu, kk ? kk : 0xFFFFFFFFu);
+      const int j0 = t * kTileM + quarter * 32;
+      if (lane == 0 && j0 < p.N)
+        reinterpret_cast<uint2 *>(p.stats)[static_cast<size_t>(srow) * p.n_spans + j0 / 32] = make_uint2(mx, mn);
+    };
     for (long long u = u0; u < u1; u++) {
       int b, g, t;
       long long bg;
@@ -294,6 +307,7 @@ __global__ void __launch_bounds__(kFp8 ? 320 : 192, 1)
             for (int i = 0; i < 32; i++) s = fmaf(sW[c0 + i], fmaxf(fmaf(sc, v[i], r[i]), 0.f), s);
           }
           if (j < p.N) p.scores[static_cast<int64_t>(b * p.Q + g) * p.ld_scores + j] = s;
+          if (p.stats) span_stats(s, j < p.N, b * p.Q + g, t);
         } else {
           for (int qi = 0; qi < p.QG; qi++) {
             float s = 0.f;
@@ -304,6 +318,7 @@ __global__ void __launch_bounds__(kFp8 ? 320 : 192, 1)
             }
             const int qq = g * p.QG + qi;
             if (j < p.N && qq < p.Q) p.scores[static_cast<int64_t>(b * p.Q + qq) * p.ld_scores + j] = s;
+            if (p.stats && qq < p.Q) span_stats(s, j < p.N, b * p.Q + qq, t);
           }
         }
       }
@@ -408,6 +423,8 @@ cudaError_t launch_score_tc(const lidx_score_args &a, cudaStream_t st) {
   p.w = a.w;
   p.scale = a.keys.scale;
   p.ld_scale = a.keys.ld_scale;
+  p.stats = a.tile_stats;
+  p.n_spans = (a.N + LIDX_STATS_SPAN - 1) / LIDX_STATS_SPAN;
   p.status = nullptr;
 
   const uint64_t rows = static_cast<uint64_t>(a.B - 1) * p.key_batch_rows + a.N;

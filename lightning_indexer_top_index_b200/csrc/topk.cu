@@ -44,6 +44,7 @@ struct Pub {
   uint32_t kmin, kmax, elig, nan;
   uint32_t cmin, cmax;
   uint32_t n_cand, overflow;
+  uint32_t above;  // this CTA's keys above the threshold bin
   uint32_t gt, eq;
   uint32_t hist[2][256];
   uint32_t cand[kCandLocal];
@@ -56,10 +57,12 @@ struct SelSmem {
   uint32_t gathered[kGatherMax];
   uint32_t red_a[kWarps], red_b[kWarps];
   uint32_t red_tot;
-  uint32_t digit, above;
+  uint32_t digit, above, total;
   uint32_t T, need;
   uint32_t g[4];                       // cluster-wide values broadcast to the CTA
   uint32_t cand_off[kMaxCluster + 1];  // prefix of the CTAs' candidate counts
+  uint32_t above_r[kMaxCluster];       // every CTA's count above the threshold bin
+  uint32_t cnt_gt[kMaxCluster], cnt_eq[kMaxCluster];  // every CTA's keys > T and == T
   uint64_t bar;
 };
 
@@ -72,6 +75,15 @@ __device__ __forceinline__ uint32_t cluster_rank() {
 
 __device__ __forceinline__ void cluster_sync_hw() {
   asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Split cluster barrier: arrive once this CTA reads no more remote shared
+// memory, wait before exiting (so no CTA leaves while others read it).
+__device__ __forceinline__ void cluster_arrive() {
+  if (gridDim.x > 1) asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  if (gridDim.x > 1) asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
 // Cluster barrier; a cluster of one CTA needs only the CTA barrier (no
@@ -179,6 +191,7 @@ __device__ __forceinline__ void find_bin(SelSmem &sm, int nbins, uint32_t rem) {
     }
     const uint32_t inc = warp_inclusive_scan(sum);
     const uint32_t before = inc - sum;
+    if (lane == 31) sm.total = inc;
     if (before < rem && inc >= rem) {
       uint32_t acc = before;
 #pragma unroll
@@ -232,6 +245,14 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelParams p) 
 
   pdl_trigger();
   pdl_wait();  // the scores come from the previous kernel
+
+  // The scorer's score bounds of the row, if given (one span record per
+  // thread now; longer rows read the rest later).
+  const int n_spans = (a.N + LIDX_STATS_SPAN - 1) / LIDX_STATS_SPAN;
+  const uint2 *stp =
+      a.tile_stats ? reinterpret_cast<const uint2 *>(a.tile_stats) + static_cast<size_t>(row) * n_spans : nullptr;
+  uint2 st0 = make_uint2(0u, 0xFFFFFFFFu);
+  if (stp && tid < n_spans) st0 = stp[tid];
 
   // ---- 0. this CTA's slice: one bulk copy into shared memory, then thread t
   // takes positions [t*C, t*C + C) of the slice into registers
@@ -306,23 +327,32 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelParams p) 
   // the keys in_bin(i) selects, given that `rem` of the k are still to be
   // taken from that bin.
   uint32_t T = 0u, need = 0u;  // T = 0: take every eligible key
-  auto resolve = [&](auto in_bin, uint32_t rem) {
-    // this CTA's keys of the threshold bin
+  // fast: the candidates were gathered, so every CTA knows every CTA's counts
+  // of keys > T and == T (sm.cnt_gt / cnt_eq) and the emission needs no
+  // exchange; this CTA has arrived on the final cluster barrier
+  bool fast = false;
+  auto resolve = [&](auto in_bin, auto above_bin, uint32_t rem) {
+    // this CTA's keys of the threshold bin (low 16 bits) and above it (high)
     uint32_t nc = 0;
 #pragma unroll
-    for (int i = 0; i < C; i++) nc += in_bin(i);
-    uint32_t n_local;
-    uint32_t cpos = cta_exclusive_scan(sm, nc, n_local);
+    for (int i = 0; i < C; i++) nc += in_bin(i) ? 1u : above_bin(i) ? 0x10000u : 0u;
+    uint32_t packed_total;
+    uint32_t cpos = cta_exclusive_scan(sm, nc, packed_total) & 0xFFFFu;  // at most 32768 each
+    const uint32_t n_local = packed_total & 0xFFFFu;
 #pragma unroll
     for (int i = 0; i < C; i++)
       if (in_bin(i)) {
         if (cpos < kCandLocal) sm.pub.cand[cpos] = key[i];
         cpos++;
       }
-    if (tid == 0) sm.pub.n_cand = n_local;
+    if (tid == 0) {
+      sm.pub.n_cand = n_local;
+      sm.pub.above = packed_total >> 16;
+    }
     cluster_sync();
-    if (tid < 32) {  // lane r reads CTA r's count
+    if (tid < 32) {  // lane r reads CTA r's counts
       const uint32_t n = static_cast<uint32_t>(tid) < G ? ld_remote(&sm.pub.n_cand, tid) : 0u;
+      if (static_cast<uint32_t>(tid) < G) sm.above_r[tid] = ld_remote(&sm.pub.above, tid);
       const uint32_t inc = warp_inclusive_scan(n);
       const uint32_t big = __ballot_sync(0xFFFFFFFFu, n > static_cast<uint32_t>(kCandLocal));
       if (static_cast<uint32_t>(tid) < G) sm.cand_off[tid] = inc - n;
@@ -346,6 +376,8 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelParams p) 
         }
       }
       __syncthreads();
+      cluster_arrive();  // no remote reads from here on
+      fast = true;
       if (n_cand <= static_cast<uint32_t>(kRankMax)) {
         if (tid < static_cast<int>(n_cand)) {
           const uint32_t mine = sm.gathered[tid];
@@ -400,6 +432,28 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelParams p) 
           need = rem;
         }
       }
+      // every CTA's keys > T and == T: its count above the bin plus its
+      // candidates (gathered segment r is CTA r's list)
+      {
+        const int warp = tid >> 5, lane = tid & 31;
+        if (static_cast<uint32_t>(warp) < G) {
+          const uint32_t off = sm.cand_off[warp];
+          const uint32_t n = (warp + 1 < static_cast<int>(G) ? sm.cand_off[warp + 1] : n_cand) - off;
+          uint32_t gt = 0, eq = 0;
+          for (uint32_t i = lane; i < n; i += 32) {
+            const uint32_t kk = sm.gathered[off + i];
+            gt += kk > T;
+            eq += kk == T;
+          }
+          gt = warp_sum(gt);
+          eq = warp_sum(eq);
+          if (lane == 0) {
+            sm.cnt_gt[warp] = sm.above_r[warp] + gt;
+            sm.cnt_eq[warp] = eq;
+          }
+        }
+      }
+      __syncthreads();
     } else {
       // a bin too full to gather: cluster-wide radix levels over the
       // candidates' differing bits, each level one exchange of histograms
@@ -455,8 +509,22 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelParams p) 
     }
   };
 
-  // ---- 1. cluster-wide min / max / eligible count / NaN
-  {
+  // ---- 1. the row's key range (and eligible count): from the scorer's score
+  // bounds when given (the count then comes with the histogram), else a
+  // cluster-wide min / max / eligible count / NaN exchange
+  uint32_t kmin, kmax, n_elig = 0;
+  const bool elig_known = stp == nullptr;
+  if (stp) {
+    uint32_t bmax = st0.x, bmin = st0.y;
+    for (int i = tid + kThreads; i < n_spans; i += kThreads) {
+      const uint2 v = stp[i];
+      bmax = max(bmax, v.x);
+      bmin = min(bmin, v.y);
+    }
+    kmax = cta_max(sm, bmax);
+    kmin = cta_min(sm, bmin);
+    if (nanf) raise_status(p.status, LIDX_DEV_NAN);
+  } else {
     const int lane = tid & 31, warp = tid >> 5;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -515,14 +583,16 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelParams p) 
       }
     }
     __syncthreads();
+    kmin = sm.g[0];
+    kmax = sm.g[1];
+    n_elig = sm.g[2];
+    if (rank == 0 && tid == 0 && sm.g[3]) raise_status(p.status, LIDX_DEV_NAN);
   }
-  const uint32_t kmin = sm.g[0], kmax = sm.g[1], n_elig = sm.g[2];
-  if (rank == 0 && tid == 0 && sm.g[3]) raise_status(p.status, LIDX_DEV_NAN);
 
   // ---- 2./3. exact k-th key T and the number `need` of keys equal to T to take
-  if (n_elig > static_cast<uint32_t>(k)) {
+  if (elig_known ? n_elig > static_cast<uint32_t>(k) : kmax != 0u) {
     uint32_t rem = static_cast<uint32_t>(k);
-    if (kmin == kmax) {
+    if (elig_known && kmin == kmax) {
       T = kmax;
       need = rem;
     } else {
@@ -549,9 +619,17 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelParams p) 
       publish_hist(sm, 0);
       cluster_sync();
       cluster_find(sm, 0, 256, rem, G);
-      const uint32_t dbin = sm.digit;
-      rem -= sm.above;
-      resolve([&](int i) { return in_lin_bin(i, dbin); }, rem);
+      if (!elig_known && sm.total <= static_cast<uint32_t>(k)) {
+        // at most k eligible keys: take them all (T = 0)
+      } else if (!elig_known && kmin == kmax) {
+        T = kmax;  // every eligible key equals the row's only value
+        need = rem;
+      } else {
+        const uint32_t dbin = sm.digit;
+        rem -= sm.above;
+        resolve([&](int i) { return in_lin_bin(i, dbin); },
+                [&](int i) { return key[i] != 0u && ((pbin[i / 4] >> (8 * (i % 4))) & 0xFFu) > dbin; }, rem);
+      }
     }
   }
 
@@ -564,27 +642,42 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelParams p) 
   }
   uint32_t cta_tot;
   const uint32_t ex = cta_exclusive_scan(sm, (n_gt << 16) | n_eq, cta_tot);  // at most 32768 each
-  if (tid == 0) {
-    sm.pub.gt = cta_tot >> 16;
-    sm.pub.eq = cta_tot & 0xFFFFu;
-  }
-  cluster_sync();
-  if (tid < 32) {  // lane r reads CTA r's counts
-    const bool in = static_cast<uint32_t>(tid) < G;
-    const uint32_t g = in ? ld_remote(&sm.pub.gt, tid) : 0u, e = in ? ld_remote(&sm.pub.eq, tid) : 0u;
-    const uint32_t gi = warp_inclusive_scan(g), ei = warp_inclusive_scan(e);
-    if (static_cast<uint32_t>(tid) == rank) {
-      sm.g[0] = gi - g;
-      sm.g[1] = ei - e;
+  uint32_t gt_before = 0, eq_before = 0, gt_total = 0, eq_total = 0;
+  if (fast) {
+    for (uint32_t r = 0; r < G; r++) {
+      const uint32_t g = sm.cnt_gt[r], e = sm.cnt_eq[r];
+      if (r < rank) {
+        gt_before += g;
+        eq_before += e;
+      }
+      gt_total += g;
+      eq_total += e;
     }
-    if (tid == 31) {
-      sm.g[2] = gi;
-      sm.g[3] = ei;
+  } else {
+    if (tid == 0) {
+      sm.pub.gt = cta_tot >> 16;
+      sm.pub.eq = cta_tot & 0xFFFFu;
     }
+    cluster_sync();
+    if (tid < 32) {  // lane r reads CTA r's counts
+      const bool in = static_cast<uint32_t>(tid) < G;
+      const uint32_t g = in ? ld_remote(&sm.pub.gt, tid) : 0u, e = in ? ld_remote(&sm.pub.eq, tid) : 0u;
+      const uint32_t gi = warp_inclusive_scan(g), ei = warp_inclusive_scan(e);
+      if (static_cast<uint32_t>(tid) == rank) {
+        sm.g[0] = gi - g;
+        sm.g[1] = ei - e;
+      }
+      if (tid == 31) {
+        sm.g[2] = gi;
+        sm.g[3] = ei;
+      }
+    }
+    __syncthreads();
+    gt_before = sm.g[0];
+    eq_before = sm.g[1];
+    gt_total = sm.g[2];
+    eq_total = sm.g[3];
   }
-  __syncthreads();
-  uint32_t gt_before = sm.g[0], eq_before = sm.g[1];
-  const uint32_t gt_total = sm.g[2], eq_total = sm.g[3];
   gt_before += ex >> 16;
   eq_before += ex & 0xFFFFu;
   uint32_t out = gt_before + min(eq_before, need);
@@ -638,7 +731,11 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelParams p) 
       if ((p0 & 31) == 0 && wi < wmax) bw[wi] = word;
     }
   }
-  cluster_sync();  // keep this CTA's shared memory alive until every CTA has read it
+  // keep this CTA's shared memory alive until every CTA has read it
+  if (fast)
+    cluster_wait();
+  else
+    cluster_sync();
 }
 
 template <int C>

@@ -16,8 +16,8 @@ from typing import List, Optional, Sequence
 
 import torch
 
-from . import (AttnArgs, DeviceKV, ScoreArgs, TopkArgs, BF16, LAUNCH_PDL, OP_ATTN, OP_TOPK, LidxError, attn_args,
-               lib, topk_args, workspace, workspace_size)
+from . import (AttnArgs, DeviceKV, ScoreArgs, TopkArgs, BF16, LAUNCH_PDL, OP_ATTN, OP_TOPK, STATS_SPAN, LidxError,
+               attn_args, lib, topk_args, workspace, workspace_size)
 
 
 class LayerCache:
@@ -33,7 +33,7 @@ class LayerCache:
 
 class DecodeStep:
     def __init__(self, caches: Sequence[LayerCache], B: int, H: int, N: int, k: int, swa_len: int, scale: float,
-                 q_dtype=torch.bfloat16, device="cuda", pdl: bool = True):
+                 q_dtype=torch.bfloat16, device="cuda", pdl: bool = True, stats: bool = True):
         self.caches = list(caches)
         self.L, self.B, self.H, self.N, self.k, self.swa_len, self.scale = len(caches), B, H, N, k, swa_len, scale
         L = self.L
@@ -46,6 +46,10 @@ class DecodeStep:
         self.n_sel = torch.zeros((L, B, 1), dtype=torch.int32, device=dev)
         self.out = torch.zeros((L, B, H, 512), dtype=torch.float32, device=dev)
         self.lse = torch.zeros((L, B, H), dtype=torch.float32, device=dev)
+        # score bounds per span of entries (scorer -> top-k): the top-k reads
+        # the row's range instead of exchanging it among its CTAs
+        n_spans = (N + STATS_SPAN - 1) // STATS_SPAN
+        self.tile_stats = torch.zeros((L, B, 1, n_spans, 2), dtype=torch.int32, device=dev) if stats else None
         self._lib = lib()
         self._score, self._topk, self._attn, self._ws_topk, self._ws_attn = [], [], [], [], []
         # Programmatic dependent launch: each kernel may start while the previous
@@ -54,9 +58,10 @@ class DecodeStep:
         flags = LAUNCH_PDL if pdl else 0
         for l, c in enumerate(self.caches):
             qd = BF16 if q_dtype == torch.bfloat16 else 0
+            ts = self.tile_stats[l] if stats else None
             sa = ScoreArgs(B, 1, H, N, qd, self.q_idx[l].data_ptr(), self.w[l].data_ptr(), c.keys.args(),
-                           self.scores[l].data_ptr(), N, flags)
-            ta = topk_args(self.scores[l], k, None, self.ids[l], self.n_sel[l], flags=flags)
+                           self.scores[l].data_ptr(), N, flags, 0 if ts is None else ts.data_ptr())
+            ta = topk_args(self.scores[l], k, None, self.ids[l], self.n_sel[l], flags=flags, tile_stats=ts)
             aa = attn_args(self.q_attn[l], c.kv, N, self.ids[l][:, 0], self.n_sel[l][:, 0], c.swa, swa_len, scale,
                            self.out[l], self.lse[l], flags=flags)
             self._score.append(sa)
