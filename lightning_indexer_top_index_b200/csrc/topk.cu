@@ -10,18 +10,22 @@
 // the contiguous slice [r*S, r*S + S) of the row and thread t of it the
 // positions [t*C, (t+1)*C) of the slice, loaded by one bulk copy and held in
 // registers.  The CTAs exchange small summaries through distributed shared
-// memory between cluster barriers:
-//   1. min / max / count of eligible keys;
+// memory; each exchange pushes (remote stores into a slot per sender) before
+// a cluster barrier, so nobody waits on remote loads after it:
+//   1. the row's minimum and maximum key: read from the scorer's score
+//      bounds when the caller passes them, else exchanged (with the count of
+//      eligible keys);
 //   2. a histogram over 256 linear value bins between the row's minimum and
 //      maximum (the bin is a monotone function of the score, so the bin
 //      holding the k-th largest key, and the count above it, are exact; for
 //      score-like data that bin holds a few dozen keys);
-//   3. the keys of that bin: every CTA gathers all of them and resolves the
-//      k-th key T and how many keys equal to T are taken (rank counting, or a
-//      radix over the candidates' differing bits when there are many; a bin
-//      too full to gather is refined by cluster-wide radix levels);
-//   4. per-CTA counts of keys > T and == T, whose prefix gives every thread
-//      its output offset: ids come out ascending, ties to the lower index.
+//   3. the keys of that bin, with each CTA's count of keys above it: every
+//      CTA resolves the k-th key T and how many keys equal to T are taken
+//      (rank counting, or a radix over the candidates' differing bits when
+//      there are many; a bin too full to gather is refined by cluster-wide
+//      radix levels), and knows every CTA's count of keys > T and == T;
+//   4. those counts' prefix gives every thread its output offset: ids come
+//      out ascending, ties to the lower index.
 #include <algorithm>
 
 #include "kernels.cuh"
@@ -35,25 +39,27 @@ constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / 32;
 constexpr int kMaxItems = 32;
 constexpr int kMaxCluster = 8;
-constexpr int kCandLocal = 1024;   // candidates a CTA publishes
-constexpr int kGatherMax = 4096;   // candidates every CTA can gather
+constexpr int kSlot = 512;                       // candidates a CTA pushes to every CTA of its cluster
+constexpr int kGatherMax = kSlot * kMaxCluster;  // candidates every CTA can gather
 constexpr int kRankMax = 96;       // candidates resolved by direct rank counting (quadratic work)
 
 // Values other CTAs of the cluster read.
 struct Pub {
   uint32_t kmin, kmax, elig, nan;
   uint32_t cmin, cmax;
-  uint32_t n_cand, overflow;
-  uint32_t above;  // this CTA's keys above the threshold bin
   uint32_t gt, eq;
   uint32_t hist[2][256];
-  uint32_t cand[kCandLocal];
 };
 
 struct SelSmem {
   Pub pub;
   uint32_t whist[8][256];     // histograms shared by groups of four warps
   uint32_t hist[256];         // cluster-wide histogram
+  // written by the other CTAs of the cluster (remote stores before a cluster
+  // barrier), slot r by CTA r
+  uint32_t hist_in[kMaxCluster][256];
+  uint32_t landing[kMaxCluster][kSlot];
+  uint32_t cnt_in[kMaxCluster], above_in[kMaxCluster];
   uint32_t gathered[kGatherMax];
   uint32_t red_a[kWarps], red_b[kWarps];
   uint32_t red_tot;
@@ -77,13 +83,14 @@ __device__ __forceinline__ void cluster_sync_hw() {
   asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-// Split cluster barrier: arrive once this CTA reads no more remote shared
-// memory, wait before exiting (so no CTA leaves while others read it).
-__device__ __forceinline__ void cluster_arrive() {
-  if (gridDim.x > 1) asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+// Start barrier: every CTA arrives when it starts and waits before its first
+// access to another CTA's shared memory, which is only valid once all CTAs
+// of the cluster run.
+__device__ __forceinline__ void cluster_arrive_start() {
+  if (gridDim.x > 1) asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 }
-__device__ __forceinline__ void cluster_wait() {
-  if (gridDim.x > 1) asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+__device__ __forceinline__ void cluster_wait_start() {
+  if (gridDim.x > 1) asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
 }
 
 // Cluster barrier; a cluster of one CTA needs only the CTA barrier (no
@@ -93,6 +100,14 @@ __device__ __forceinline__ void cluster_sync() {
     __syncthreads();
   else
     cluster_sync_hw();
+}
+
+// Store a 32-bit word into CTA `rank`'s shared memory at the local address `p`
+// (the push side of an exchange: a cluster barrier makes it visible).
+__device__ __forceinline__ void st_remote(uint32_t *p, uint32_t rank, uint32_t v) {
+  uint32_t a;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(tc::smem_u32(p)), "r"(rank));
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
 }
 
 // Load a 32-bit word of CTA `rank`'s shared memory at the local address `p`.
@@ -132,15 +147,6 @@ __device__ __forceinline__ uint32_t cta_min(SelSmem &sm, uint32_t v) {
 }
 
 __device__ __forceinline__ uint32_t cta_max(SelSmem &sm, uint32_t v) { return ~cta_min(sm, ~v); }
-
-__device__ __forceinline__ uint32_t cta_sum(SelSmem &sm, uint32_t v) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  v = warp_sum(v);
-  __syncthreads();
-  if (lane == 0) sm.red_a[warp] = v;
-  __syncthreads();
-  return warp_sum(sm.red_a[lane]);
-}
 
 // Exclusive CTA scan of 32-bit values; *total gets the CTA sum.
 __device__ __forceinline__ uint32_t cta_exclusive_scan(SelSmem &sm, uint32_t v, uint32_t &total) {
@@ -223,6 +229,27 @@ __device__ __forceinline__ void cluster_find(SelSmem &sm, int buf, int nbins, ui
   find_bin(sm, nbins, rem);
 }
 
+// Push this CTA's histogram (the sum of its group histograms) into slot
+// `rank` of every CTA of the cluster; a cluster barrier must follow.
+__device__ __forceinline__ void push_hist(SelSmem &sm, uint32_t G, uint32_t rank) {
+  __syncthreads();
+  const int bin = threadIdx.x & 255;
+  uint32_t v = 0;
+#pragma unroll
+  for (int w = 0; w < 8; w++) v += sm.whist[w][bin];
+  for (uint32_t r = threadIdx.x >> 8; r < G; r += kThreads / 256) st_remote(&sm.hist_in[rank][bin], r, v);
+}
+
+// After the barrier: the cluster-wide histogram from the pushed slots, then find_bin.
+__device__ __forceinline__ void sum_pushed_hist(SelSmem &sm, uint32_t G, int nbins, uint32_t rem) {
+  if (threadIdx.x < 256) {
+    uint32_t v = 0;
+    for (uint32_t r = 0; r < G; r++) v += sm.hist_in[r][threadIdx.x];
+    sm.hist[threadIdx.x] = v;
+  }
+  find_bin(sm, nbins, rem);
+}
+
 struct SelParams {
   lidx_topk_args a;
   uint32_t *status;
@@ -231,8 +258,9 @@ struct SelParams {
 
 template <int C>
 __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelParams p) {
-  extern __shared__ __align__(16) float rowbuf[];
-  __shared__ SelSmem sm;
+  extern __shared__ __align__(16) uint8_t dyn_smem[];
+  SelSmem &sm = *reinterpret_cast<SelSmem *>(dyn_smem);
+  float *rowbuf = reinterpret_cast<float *>(dyn_smem + ((sizeof(SelSmem) + 15) & ~size_t(15)));
   const lidx_topk_args &a = p.a;
   const int tid = threadIdx.x;
   const int hg = (tid >> 5) & 7;
@@ -243,6 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelParams p) 
   const int s0 = static_cast<int>(rank) * p.slice;  // first position of this CTA's slice
   const int p0 = tid * C;                           // first position of this thread, within the slice
 
+  cluster_arrive_start();
   pdl_trigger();
   pdl_wait();  // the scores come from the previous kernel
 
@@ -339,22 +368,24 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelParams p) 
     uint32_t packed_total;
     uint32_t cpos = cta_exclusive_scan(sm, nc, packed_total) & 0xFFFFu;  // at most 32768 each
     const uint32_t n_local = packed_total & 0xFFFFu;
+    // push the candidates into slot `rank` of every CTA, with the counts
 #pragma unroll
     for (int i = 0; i < C; i++)
       if (in_bin(i)) {
-        if (cpos < kCandLocal) sm.pub.cand[cpos] = key[i];
+        if (cpos < static_cast<uint32_t>(kSlot))
+          for (uint32_t r = 0; r < G; r++) st_remote(&sm.landing[rank][cpos], r, key[i]);
         cpos++;
       }
-    if (tid == 0) {
-      sm.pub.n_cand = n_local;
-      sm.pub.above = packed_total >> 16;
+    if (static_cast<uint32_t>(tid) < G) {
+      st_remote(&sm.cnt_in[rank], tid, n_local);
+      st_remote(&sm.above_in[rank], tid, packed_total >> 16);
     }
     cluster_sync();
-    if (tid < 32) {  // lane r reads CTA r's counts
-      const uint32_t n = static_cast<uint32_t>(tid) < G ? ld_remote(&sm.pub.n_cand, tid) : 0u;
-      if (static_cast<uint32_t>(tid) < G) sm.above_r[tid] = ld_remote(&sm.pub.above, tid);
+    if (tid < 32) {  // every CTA's counts, now local
+      const uint32_t n = static_cast<uint32_t>(tid) < G ? sm.cnt_in[tid] : 0u;
+      if (static_cast<uint32_t>(tid) < G) sm.above_r[tid] = sm.above_in[tid];
       const uint32_t inc = warp_inclusive_scan(n);
-      const uint32_t big = __ballot_sync(0xFFFFFFFFu, n > static_cast<uint32_t>(kCandLocal));
+      const uint32_t big = __ballot_sync(0xFFFFFFFFu, n > static_cast<uint32_t>(kSlot));
       if (static_cast<uint32_t>(tid) < G) sm.cand_off[tid] = inc - n;
       if (tid == 31) {
         sm.cand_off[kMaxCluster] = inc;
@@ -364,20 +395,18 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelParams p) 
     __syncthreads();
     const uint32_t n_cand = sm.cand_off[kMaxCluster];
     const bool too_many = sm.g[0] != 0u;
-    if (!too_many && n_cand <= static_cast<uint32_t>(kGatherMax)) {
-      // gather every candidate of the cluster (the same list in every CTA):
-      // warp r copies CTA r's list
+    if (!too_many) {
+      // the same candidate list in every CTA: warp r compacts slot r
       {
         const int warp = tid >> 5, lane = tid & 31;
         if (static_cast<uint32_t>(warp) < G) {
           const uint32_t off = sm.cand_off[warp];
           const uint32_t n = (warp + 1 < static_cast<int>(G) ? sm.cand_off[warp + 1] : n_cand) - off;
-          for (uint32_t i = lane; i < n; i += 32) sm.gathered[off + i] = ld_remote(&sm.pub.cand[i], warp);
+          for (uint32_t i = lane; i < n; i += 32) sm.gathered[off + i] = sm.landing[warp][i];
         }
       }
       __syncthreads();
-      cluster_arrive();  // no remote reads from here on
-      fast = true;
+      fast = true;  // no cluster traffic from here on
       if (n_cand <= static_cast<uint32_t>(kRankMax)) {
         if (tid < static_cast<int>(n_cand)) {
           const uint32_t mine = sm.gathered[tid];
@@ -514,6 +543,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelParams p) 
   // cluster-wide min / max / eligible count / NaN exchange
   uint32_t kmin, kmax, n_elig = 0;
   const bool elig_known = stp == nullptr;
+  cluster_wait_start();
   if (stp) {
     uint32_t bmax = st0.x, bmin = st0.y;
     for (int i = tid + kThreads; i < n_spans; i += kThreads) {
@@ -521,8 +551,19 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelParams p) 
       bmax = max(bmax, v.x);
       bmin = min(bmin, v.y);
     }
-    kmax = cta_max(sm, bmax);
-    kmin = cta_min(sm, bmin);
+    // one block reduction for both bounds
+    {
+      const int lane = tid & 31, warp = tid >> 5;
+      bmax = __reduce_max_sync(0xFFFFFFFFu, bmax);
+      bmin = __reduce_min_sync(0xFFFFFFFFu, bmin);
+      if (lane == 0) {
+        sm.red_a[warp] = bmax;
+        sm.red_b[warp] = bmin;
+      }
+      __syncthreads();
+      kmax = __reduce_max_sync(0xFFFFFFFFu, sm.red_a[lane]);
+      kmin = __reduce_min_sync(0xFFFFFFFFu, sm.red_b[lane]);
+    }
     if (nanf) raise_status(p.status, LIDX_DEV_NAN);
   } else {
     const int lane = tid & 31, warp = tid >> 5;
@@ -616,9 +657,9 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelParams p) 
         pbin[i / 4] |= b << (8 * (i % 4));
       }
       auto in_lin_bin = [&](int i, uint32_t d) { return key[i] != 0u && ((pbin[i / 4] >> (8 * (i % 4))) & 0xFFu) == d; };
-      publish_hist(sm, 0);
+      push_hist(sm, G, rank);
       cluster_sync();
-      cluster_find(sm, 0, 256, rem, G);
+      sum_pushed_hist(sm, G, 256, rem);
       if (!elig_known && sm.total <= static_cast<uint32_t>(k)) {
         // at most k eligible keys: take them all (T = 0)
       } else if (!elig_known && kmin == kmax) {
@@ -731,16 +772,14 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelParams p) 
       if ((p0 & 31) == 0 && wi < wmax) bw[wi] = word;
     }
   }
-  // keep this CTA's shared memory alive until every CTA has read it
-  if (fast)
-    cluster_wait();
-  else
-    cluster_sync();
+  // keep this CTA's shared memory alive until every CTA has read it (the
+  // fast path reads no remote memory after its last barrier)
+  if (!fast) cluster_sync();
 }
 
 template <int C>
 cudaError_t launch_c(int G, int rows, const SelParams &p, cudaStream_t st, bool pdl) {
-  const size_t smem = (static_cast<size_t>(C) * kThreads + 4) * sizeof(float);
+  const size_t smem = ((sizeof(SelSmem) + 15) & ~size_t(15)) + (static_cast<size_t>(C) * kThreads + 4) * sizeof(float);
   cudaFuncSetAttribute(select_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(G, rows);
