@@ -14,15 +14,15 @@
 //      cp.async, one warp per row, straight into the 128-byte-swizzled
 //      K-major layout; E4M3 rows are converted in registers (times their
 //      power-of-two block scale; RoPE dims copied).
-//   2. MMA 1: S^T[row][head] = X . Q^T (M = 128, N = 16, K = 512) into TMEM.
-//      Rows 64..127 of the A operand run into the next panel (and, for the
-//      last panel, into the Q buffer): their S rows are never read.
-//   3. Softmax: 4 warps; thread = one row and 8 heads; per-head max and sum
-//      over the 64 rows by butterfly shuffles and a 2-warp exchange.  P^T is
-//      written to shared memory as bf16 hi and lo parts (p = hi + lo to ~16
-//      bits), K-major: one 128-byte swizzled line of 64 rows per head.
-//   4. MMA 2: O^T[d][head] = X^T . P^T, reading the same X tile as an
-//      MN-major operand (K = V), four 128-wide d tiles (N = 16) into TMEM.
+//   2. MMA 1: S^T[row][head] = X . Q^T (M = 64, N = 16, K = 512) into TMEM.
+//   3. Softmax: 8 warps; warp w takes rows 16(w&3).. (its TMEM lanes 0-15)
+//      and heads 8(w>>2)..; per-head max and sum over the 64 rows by
+//      butterfly shuffles and a 4-warp exchange.  P^T is written to shared
+//      memory as bf16 hi and lo parts (p = hi + lo to ~16 bits), K-major: one
+//      128-byte swizzled line of 64 rows per head, hi heads then lo heads.
+//   4. MMA 2: [O_hi | O_lo]^T[d][.] = X^T . [P_hi | P_lo]^T (N = 32),
+//      reading the same X tile as an MN-major operand (K = V), four 128-wide
+//      d tiles into TMEM; the epilogue adds the two parts.
 //   5. Each warp stores two d tiles, lanes = consecutive d: coalesced stores.
 // The partials are combined by the split-K merge kernel.
 #include "kernels.cuh"
@@ -46,7 +46,15 @@ constexpr int kXPanel = kRows * 128;         // 8 KB
 constexpr int kQBytes = kHG * kD * 2;        // 16 KB: 8 panels of [16 heads][128 B]
 constexpr int kQPanel = kHG * 128;           // 2 KB
 constexpr int kPBytes = kHG * kRows * 2;     // 2 KB: one bf16 P^T [16 heads][64 rows]
-constexpr uint32_t kTmemCols = 128;          // S^T at [0,16), O^T tile t at [32+16t, 48+16t)
+// TMEM: S^T as kS1 partial sums over K at columns [16i, 16i + 16) (M = 64:
+// row 16q + r in lane 32q + r), O^T tile t at [64 + 32t, 96 + 32t) as the
+// P_hi part (16 columns) then the P_lo part.  These MMAs are tiny, and each
+// costs its issuing thread a roughly fixed time: so MMA 1 is issued by kS1
+// threads over K quarters into separate partial sums, MMA 2 by four threads
+// (one d tile each) multiplying X^T by P_hi and P_lo at once (N = 32).
+constexpr int kS1 = 4;
+constexpr uint32_t kOCol = 64;
+constexpr uint32_t kTmemCols = 256;
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct __align__(8) AttnTcSmem {
@@ -57,7 +65,7 @@ struct __align__(8) AttnTcSmem {
   uint32_t abort;
   int64_t row_src[kRows];  // row index in its cache; -1 when empty
   int32_t row_kind[kRows]; // 0 none, 1 selected, 2 window
-  float red[2][2][8];      // per head half, per warp of the pair
+  float red[2][4][8];      // per head half, per row quarter
 };
 
 // smem: X (64 KB) | Q (16 KB) | P^T hi, lo (2 x 2 KB) | bookkeeping.  Q
@@ -100,8 +108,8 @@ __global__ void __launch_bounds__(kThreads, 2)
   const bool tma_window = !kFp8 && pure_window;  // 64 contiguous window rows
   if (tid == 0) {
     tc::mbar_init(&sm->q_full, 1);
-    tc::mbar_init(&sm->s_full, 1);
-    tc::mbar_init(&sm->o_full, 1);
+    tc::mbar_init(&sm->s_full, kS1);
+    tc::mbar_init(&sm->o_full, 4);
     sm->abort = 0;
     tc::fence_barrier_init();
     tc::tma_prefetch_desc(&tm_q);
@@ -207,37 +215,47 @@ __global__ void __launch_bounds__(kThreads, 2)
   tc::fence_proxy_async_smem();
   __syncthreads();
 
-  // ---- 2. S^T = X . Q^T
-  if (tid == 0) {
+  // ---- 2. S^T = X . Q^T: lane 0 of warp i < kS1 issues K steps [8i, 8i + 8)
+  // into partial sum i
+  if (warp < kS1 && lane == 0) {
     if (tc::mbar_wait(&sm->q_full, 0, abort_flag)) {
       tc::tc_fence_after();
-      const uint32_t idesc = tc::idesc_bf16(128, kHG);
+      const uint32_t idesc = tc::idesc_bf16(kRows, kHG);
       const uint32_t qs = tc::smem_u32(sQ);
 #pragma unroll
-      for (int k = 0; k < 32; k++) {
+      for (int kk = 0; kk < 32 / kS1; kk++) {
+        const int k = warp * (32 / kS1) + kk;
         const uint32_t ao = (k >> 2) * kXPanel + (k & 3) * 32;
         const uint32_t bo = (k >> 2) * kQPanel + (k & 3) * 32;
-        tc::mma_bf16(tmem, tc::desc_kmajor_sw128(xs + ao), tc::desc_kmajor_sw128(qs + bo), idesc, k > 0);
+        tc::mma_bf16(tmem + 16 * warp, tc::desc_kmajor_sw128(xs + ao), tc::desc_kmajor_sw128(qs + bo), idesc, kk > 0);
       }
       tc::mma_commit(&sm->s_full);
     }
   }
 
-  // ---- 3. softmax over the 64 rows, per head: warps 0,1 (heads 0-7) and
-  // 4,5 (heads 8-15); warp w reads TMEM lane quarter w&3 = rows 32(w&3)..
+  // ---- 3. softmax over the 64 rows, per head: warp w takes row quarter
+  // q = w&3 (rows 16q + lane, lanes 0-15; M = 64 puts them in TMEM lanes
+  // 32q..32q+15) and heads 8h.. with h = w>>2
   const int quarter = warp & 3, half = warp >> 2;
-  const bool smax_warp = quarter < 2 && half < 2;
   bool ready = false;
-  if (lane == 0) ready = smax_warp ? tc::mbar_wait(&sm->s_full, 0, abort_flag) : true;
+  if (lane == 0) ready = tc::mbar_wait(&sm->s_full, 0, abort_flag);
   ready = __shfl_sync(0xFFFFFFFFu, ready, 0);
   float mx[8];
-  if (smax_warp) {
-    const int r = quarter * 32 + lane;
-    const bool valid = sm->row_kind[r] != 0;
+  {
+    const int r = quarter * 16 + (lane & 15);
+    const bool valid = lane < 16 && sm->row_kind[r] != 0;
     float s[8];
     if (ready) {
       tc::tc_fence_after();
-      tc::tmem_ld8(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + half * 8, s);
+      const uint32_t ta = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + half * 8;
+      tc::tmem_ld8(ta, s);
+#pragma unroll
+      for (int i = 1; i < kS1; i++) {
+        float t8[8];
+        tc::tmem_ld8(ta + 16 * i, t8);
+#pragma unroll
+        for (int h = 0; h < 8; h++) s[h] += t8[h];
+      }
     }
     const float c2 = a.scale * kLog2e;
 #pragma unroll
@@ -246,75 +264,71 @@ __global__ void __launch_bounds__(kThreads, 2)
       mx[h] = s[h];
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
+    for (int o = 8; o > 0; o >>= 1)  // lanes 16-31 hold -inf copies: reduce within 16
 #pragma unroll
       for (int h = 0; h < 8; h++) mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xFFFFFFFFu, mx[h], o));
     if (lane == 0)
 #pragma unroll
       for (int h = 0; h < 8; h++) sm->red[half][quarter][h] = mx[h];
-    named_sync(1 + half, 64);
+    named_sync(1 + half, 128);
     float pv[8];
 #pragma unroll
     for (int h = 0; h < 8; h++) {
-      const float m = fmaxf(sm->red[half][0][h], sm->red[half][1][h]);
+      const float m = fmaxf(fmaxf(sm->red[half][0][h], sm->red[half][1][h]),
+                            fmaxf(sm->red[half][2][h], sm->red[half][3][h]));
       mx[h] = m;
       pv[h] = (m == -INFINITY || s[h] == -INFINITY) ? 0.f : exp2f(s[h] - m);
     }
     // P^T[head][row] as hi = bf16(p), lo = bf16(p - hi): head line h holds
     // rows in 16-byte chunks of 8, chunk index swizzled with h & 7
+    if (lane < 16) {
 #pragma unroll
-    for (int i = 0; i < 8; i++) {
-      const int h = half * 8 + i;
-      const __nv_bfloat16 ph = __float2bfloat16_rn(pv[i]);
-      const __nv_bfloat16 pl = __float2bfloat16_rn(pv[i] - __bfloat162float(ph));
-      const int off = h * 128 + ((((r >> 3) ^ (h & 7))) << 4) + (r & 7) * 2;
-      *reinterpret_cast<__nv_bfloat16 *>(sP + off) = ph;
-      *reinterpret_cast<__nv_bfloat16 *>(sP + kPBytes + off) = pl;
+      for (int i = 0; i < 8; i++) {
+        const int h = half * 8 + i;
+        const __nv_bfloat16 ph = __float2bfloat16_rn(pv[i]);
+        const __nv_bfloat16 pl = __float2bfloat16_rn(pv[i] - __bfloat162float(ph));
+        const int off = h * 128 + ((((r >> 3) ^ (h & 7))) << 4) + (r & 7) * 2;
+        *reinterpret_cast<__nv_bfloat16 *>(sP + off) = ph;
+        *reinterpret_cast<__nv_bfloat16 *>(sP + kPBytes + off) = pl;
+      }
     }
     float sum[8];
 #pragma unroll
-    for (int h = 0; h < 8; h++) sum[h] = pv[h];
+    for (int h = 0; h < 8; h++) sum[h] = lane < 16 ? pv[h] : 0.f;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
+    for (int o = 8; o > 0; o >>= 1)
 #pragma unroll
       for (int h = 0; h < 8; h++) sum[h] += __shfl_xor_sync(0xFFFFFFFFu, sum[h], o);
-    named_sync(1 + half, 64);  // both warps have read the maxima
+    named_sync(1 + half, 128);  // the four warps have read the maxima
     if (lane == 0)
 #pragma unroll
       for (int h = 0; h < 8; h++) sm->red[half][quarter][h] = sum[h];
-    named_sync(1 + half, 64);
+    named_sync(1 + half, 128);
   }
   if (pure_window) pdl_wait();  // no global write before the previous kernel is done
-  if (smax_warp) {
-    if (quarter == 0 && lane < 8) {
-      const float l = sm->red[half][0][lane] + sm->red[half][1][lane];
-      float m = mx[0];
+  if (quarter == 0 && lane < 8) {
+    const float l = (sm->red[half][0][lane] + sm->red[half][1][lane]) + (sm->red[half][2][lane] + sm->red[half][3][lane]);
+    float m = mx[0];
 #pragma unroll
-      for (int i = 1; i < 8; i++)
-        if (i == lane) m = mx[i];
-      part_ml[(static_cast<size_t>(b) * n_split + split) * kH + hg * kHG + half * 8 + lane] = make_float2(m, l);
-    }
+    for (int i = 1; i < 8; i++)
+      if (i == lane) m = mx[i];
+    part_ml[(static_cast<size_t>(b) * n_split + split) * kH + hg * kHG + half * 8 + lane] = make_float2(m, l);
   }
   tc::fence_proxy_async_smem();
   tc::tc_fence_before();
   __syncthreads();
 
-  // ---- 4. O^T = X^T . (P_hi + P_lo)^T
-  if (tid == 0 && !*abort_flag) {
+  // ---- 4. O^T = X^T . (P_hi + P_lo)^T: lane 0 of warp dt < 4 issues d tile dt
+  if (warp < 4 && lane == 0 && !*abort_flag) {
     tc::tc_fence_after();
-    const uint32_t idesc = tc::idesc_bf16(128, kHG, true, false);
+    const uint32_t idesc = tc::idesc_bf16(128, 2 * kHG, true, false);
     const uint32_t ps = tc::smem_u32(sP);
+    const int dt = warp;
 #pragma unroll
-    for (int dt = 0; dt < 4; dt++) {
-#pragma unroll
-      for (int part = 0; part < 2; part++) {
-#pragma unroll
-        for (int kk = 0; kk < kRows / 16; kk++) {
-          const uint64_t adesc = tc::desc_mnmajor_sw128(xs + 2 * dt * kXPanel + kk * 2048, kXPanel, 1024);
-          const uint64_t bdesc = tc::desc_kmajor_sw128(ps + part * kPBytes + kk * 32);
-          tc::mma_bf16(tmem + 32 + 16 * dt, adesc, bdesc, idesc, (part | kk) != 0);
-        }
-      }
+    for (int kk = 0; kk < kRows / 16; kk++) {
+      const uint64_t adesc = tc::desc_mnmajor_sw128(xs + 2 * dt * kXPanel + kk * 2048, kXPanel, 1024);
+      const uint64_t bdesc = tc::desc_kmajor_sw128(ps + kk * 32);  // 32 lines: hi heads, then lo heads
+      tc::mma_bf16(tmem + kOCol + 32 * dt, adesc, bdesc, idesc, kk > 0);
     }
     tc::mma_commit(&sm->o_full);
   }
@@ -331,10 +345,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     for (int j = 0; j < 2; j++) {
       const int dt = (warp >> 2) + 2 * j;
       const int d = dt * 128 + quarter * 32 + lane;
-      float v[16];
-      tc::tmem_ld16(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + 32 + 16 * dt, v);
+      float v[32];
+      tc::tmem_ld32(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + kOCol + 32 * dt, v);
 #pragma unroll
-      for (int h = 0; h < kHG; h++) po[h * kD + d] = v[h];
+      for (int h = 0; h < kHG; h++) po[h * kD + d] = v[h] + v[kHG + h];
     }
   }
   tc::tc_fence_before();

@@ -61,7 +61,7 @@ struct SelSmem {
   uint32_t landing[kMaxCluster][kSlot];
   uint32_t cnt_in[kMaxCluster], above_in[kMaxCluster];
   uint32_t gathered[kGatherMax];
-  uint32_t red_a[kWarps], red_b[kWarps];
+  uint32_t red_a[kWarps], red_b[kWarps], red_c[kWarps], red_d[kWarps];
   uint32_t red_tot;
   uint32_t digit, above, total;
   uint32_t T, need;
@@ -297,6 +297,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelParams p) 
       tc::mbar_init(&sm.bar, 1);
       tc::fence_barrier_init();
     }
+    clear_whist(sm);  // for the value histogram, off the critical path
     __syncthreads();
     if (tid == 0 && body > 0) {
       tc::mbar_arrive_expect_tx(&sm.bar, body * 4);
@@ -577,15 +578,15 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelParams p) 
     if (lane == 0) {
       sm.red_a[warp] = lo;
       sm.red_b[warp] = hi;
-      sm.whist[0][warp] = elig;
-      sm.whist[1][warp] = nanf;
+      sm.red_c[warp] = elig;
+      sm.red_d[warp] = nanf;
     }
     __syncthreads();
     if (warp == 0) {
       lo = sm.red_a[lane];
       hi = sm.red_b[lane];
-      elig = sm.whist[0][lane];
-      nanf = sm.whist[1][lane];
+      elig = sm.red_c[lane];
+      nanf = sm.red_d[lane];
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) {
         lo = min(lo, __shfl_xor_sync(0xFFFFFFFFu, lo, o));
@@ -642,8 +643,6 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelParams p) 
       const float scale0 = 256.f / range;
       const bool linear = isfinite(range) && range > 0.f && isfinite(scale0);
       const float scale = linear ? scale0 : 0.f;
-      clear_whist(sm);
-      __syncthreads();
       uint32_t pbin[(C + 3) / 4];
 #pragma unroll
       for (int i = 0; i < (C + 3) / 4; i++) pbin[i] = 0u;
