@@ -180,9 +180,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // Combine the split partials of one (b, h): base-2 log-sum-exp rescaling.
-// Thread t owns dims [4t, 4t+4).  Each batch of up to 8 splits issues its
+// Thread t owns dims [4t, 4t+4).  Each batch of up to 16 splits issues its
 // partial-O loads and its (m, l) loads together, then folds them in with a
-// running maximum, so a merge of <= 8 splits costs one memory round trip.
+// running maximum, so a merge of <= 16 splits costs one memory round trip.
 __global__ void __launch_bounds__(128) attn_merge_kernel(lidx_attn_args a, const float *part_o,
                                                           const float2 *part_ml, int n_split) {
   pdl_trigger();
@@ -193,18 +193,18 @@ __global__ void __launch_bounds__(128) attn_merge_kernel(lidx_attn_args a, const
   const size_t stride4 = static_cast<size_t>(H) * kD / 4;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   float M = -INFINITY, L = 0.f;
-  for (int s0 = 0; s0 < n_split; s0 += 8) {
-    float4 v[8];
-    float2 w[8];
+  for (int s0 = 0; s0 < n_split; s0 += 16) {
+    float4 v[16];
+    float2 w[16];
 #pragma unroll
-    for (int i = 0; i < 8; i++) {
+    for (int i = 0; i < 16; i++) {
       if (s0 + i < n_split) {
         w[i] = ml[static_cast<size_t>(s0 + i) * H];
         v[i] = po[(s0 + i) * stride4];
       }
     }
 #pragma unroll
-    for (int i = 0; i < 8; i++) {
+    for (int i = 0; i < 16; i++) {
       if (s0 + i < n_split && w[i].x != -INFINITY) {
         const float mn = fmaxf(M, w[i].x);
         const float c = exp2f(M - mn);  // 0 while M is -inf

@@ -196,20 +196,57 @@ __global__ void __launch_bounds__(kThreads, 2)
     pdl_wait();  // ids and n_sel come from the top-k kernel
     int n_b = a.n_ids;
     if (a.n_sel) n_b = min(max(a.n_sel[b], 0), a.n_ids);
-    if (tid < kRows) {
-      const int i = i0 + tid - swa_len;
+    // resolve the selected row of list entry i0 + r (row r of the chunk)
+    auto resolve_row = [&](int r, int &kind, int64_t &src) {
+      const int i = i0 + r - swa_len;
       if (i >= 0 && i < n_b) {
         const int id = a.ids[static_cast<int64_t>(b) * a.ld_ids + i];
         if (id >= 0 && id < a.N) {
-          sm->row_kind[tid] = 1;
-          sm->row_src[tid] = static_cast<int64_t>(b) * a.kv.batch_rows + id;
+          kind = 1;
+          src = static_cast<int64_t>(b) * a.kv.batch_rows + id;
+          sm->row_kind[r] = 1;
+          sm->row_src[r] = src;
         } else if (id != -1) {
           raise_status(status, LIDX_DEV_BOUNDS);
         }
       }
+    };
+    if (kFp8) {
+      if (tid < kRows) {
+        int kind;
+        int64_t src;
+        resolve_row(tid, kind, src);
+      }
+      __syncthreads();
+      load_rows(1);
+    } else {
+      // bf16: warp w gathers rows w + 8j; lane j resolves row w + 8j, so no
+      // block barrier stands between the ids and the gather
+      constexpr int kPerWarp = kRows / (kThreads / 32);
+      int kind = 0;
+      int64_t src = -1;
+      if (lane < kPerWarp) {
+        const int r = warp + (kThreads / 32) * lane;
+        kind = sm->row_kind[r];
+        src = sm->row_src[r];
+        resolve_row(r, kind, src);
+      }
+#pragma unroll
+      for (int j = 0; j < kPerWarp; j++) {
+        const int kj = __shfl_sync(0xFFFFFFFFu, kind, j);
+        const int64_t sj = __shfl_sync(0xFFFFFFFFu, src, j);
+        const int r = warp + (kThreads / 32) * j;
+        if (kj == 2) continue;  // window row: loaded in pass 0
+        if (kj == 1) {
+          const uint16_t *row = static_cast<const uint16_t *>(a.kv.data) + sj * a.kv.ld;
+          cp_async16(xs + x_off(r, lane), row + lane * 8);
+          cp_async16(xs + x_off(r, lane + 32), row + (lane + 32) * 8);
+        } else {
+          *reinterpret_cast<uint4 *>(sX + x_off(r, lane)) = make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4 *>(sX + x_off(r, lane + 32)) = make_uint4(0, 0, 0, 0);
+        }
+      }
     }
-    __syncthreads();
-    load_rows(1);
   }
   cp_async_wait_all();
   tc::fence_proxy_async_smem();
