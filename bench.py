@@ -5,7 +5,12 @@ attention) over a stack of CSA layers, on synthetic inputs shaped like the
 entries per layer, 64 heads, top-512, 128-row window, bf16).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl lidx|reference]
-                    [--workload decode-64k|decode-128k-b32|decode-500k-b4]
+                    [--workload decode-64k|decode-128k-b32|decode-500k-b4|eval-window]
+
+The eval-window workload times one tau-window of the selection evaluation
+(64 queries x 21 layers x 32768 entries: native scores and top-512, golden
+dense-attention probabilities, top-p 0.6, the 3-of-21 vote and window union,
+the gate, overlap counts) in windows/s.
 
 Prints one JSON line (rank 0).  With --gpus N > 1 under torchrun every rank
 runs an independent replica of the workload on its own GPU (the path does not
@@ -71,8 +76,9 @@ def peaks() -> dict:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         d = json.load(open(p))
-        return dict(hbm_gbs=float(d["hbm_gbs"]), source="measured")
-    return dict(hbm_gbs=6650.0, source="fallback")
+        return dict(hbm_gbs=float(d["hbm_gbs"]), bf16_tflops=float(d["bf16_tflops"]),
+                    bf16_tflops_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
 
 
 # source files of each library call's kernels
@@ -358,17 +364,183 @@ def run_lidx(args, spec, cfg, rank, world, local_rank):
         dist.destroy_process_group()
 
 
+# ------------------------------------------------------------- eval window
+EVAL_METRIC = "selection-eval windows/s (64 queries x 21 layers x 32K entries; golden TFLOP/s vs peak)"
+EVAL_STAGES = ("score", "topk", "golden", "gold_topk", "vote", "gate", "overlap")
+
+
+def eval_inputs(spec):
+    layers = [synth.eval_layer(spec, l) for l in range(spec.L)]
+    return layers, synth.eval_gate(spec)
+
+
+def oracle_eval_sample(spec, layers, gate):
+    """The oracle on a bounded sample of a window: golden probabilities of one
+    query of one layer (all 64 heads, all N entries), its top-p set and top-k;
+    returns (seconds, windows the sample stands for)."""
+    import oracle
+    x = layers[0]
+    t0 = time.perf_counter()
+    p = oracle.golden(x["qa"][:1], x["kv"], 1, spec.H, spec.N, spec.scale)
+    oracle.topp(p[0])
+    oracle.topk(p[0], spec.k)
+    dt = time.perf_counter() - t0
+    return dt, 1.0 / (spec.L * spec.T)
+
+
+def run_eval(args, cfg, rank, world, local_rank, reference=False):
+    spec = synth.C5
+    if reference:
+        layers, gate = eval_inputs(synth.scaled(spec, L=1))
+        for _ in range(args.warmup):
+            oracle_eval_sample(spec, layers, gate)
+        t, w = 0.0, 0.0
+        for _ in range(args.steps):
+            dt, dw = oracle_eval_sample(spec, layers, gate)
+            t, w = t + dt, w + dw
+        v = w / t
+        sample = ("golden probabilities, top-p and top-k of one query of one layer per step "
+                  f"(1/{spec.L * spec.T} of a window), single thread")
+        print(json.dumps({"metric": EVAL_METRIC, "value": v, "unit": "windows/s", "n_gpus": args.gpus,
+                          "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / v,
+                          "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                          "data": "synthetic", "config": cfg, "impl": "reference",
+                          "cpu_baseline": {"value": v, "unit": "windows/s", "cores": 1, "kind": "oracle",
+                                           "sample": sample},
+                          "e2e": {"value": v, "unit": "windows/s", "h2d_bytes_per_step": 0,
+                                  "d2h_bytes_per_step": 0}}), flush=True)
+        return
+    import torch
+    import lightning_indexer_top_index_b200 as L
+    from lightning_indexer_top_index_b200.evalwin import EvalWindow
+
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    layers, gate = eval_inputs(spec)
+
+    def bf(a):
+        return torch.from_numpy(np.ascontiguousarray(a)).view(torch.int16).view(torch.bfloat16)
+
+    keys = [L.DeviceKV.from_arrays("bf16", 128, x["keys"].data, batch_rows=spec.N, device=device) for x in layers]
+    kv_all = L.DeviceKV.from_arrays("bf16", 512, np.concatenate([x["kv"].data for x in layers]),
+                                    batch_rows=spec.N, device=device)
+    q_idx_h = torch.stack([bf(x["q_idx"]) for x in layers])
+    w_h = torch.stack([torch.from_numpy(x["w"]) for x in layers])
+    qa_h = torch.stack([bf(x["qa"]) for x in layers])
+    gq_h, gu_h = bf(gate["g"]), torch.from_numpy(gate["u"])
+    q_idx, w, qa, gq, gu = (t.to(device) for t in (q_idx_h, w_h, qa_h, gq_h, gu_h))
+    win = EvalWindow(keys, kv_all, q_idx, w, qa, gq, gu, spec.gate_layers, spec.N, spec.k,
+                     (spec.top_p_num, spec.top_p_den), spec.min_votes, spec.scale)
+    for _ in range(args.warmup):
+        win.enqueue()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        win.enqueue()
+    e1.record()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    if dist:
+        t = torch.tensor([ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    # per-stage times (events between stages)
+    ev = {n: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for n in EVAL_STAGES}
+    stage_ms = {n: 0.0 for n in EVAL_STAGES}
+    reps = max(1, min(args.steps, 5))
+    for _ in range(reps):
+        win.enqueue(events=ev)
+        torch.cuda.synchronize()
+        for n in EVAL_STAGES:
+            stage_ms[n] += ev[n][0].elapsed_time(ev[n][1]) / reps
+    # end to end: the window's queries in from pinned host memory, counts back
+    pins = [t.pin_memory() for t in (q_idx_h, w_h, qa_h, gq_h, gu_h)]
+    outs = [torch.empty(c.shape, dtype=c.dtype).pin_memory()
+            for c in (win.counts_nat_gold, win.counts_nat_f, win.counts_g_f)]
+    dsts = (win.q_idx, win.w, win.qa, gq, gu)
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record()
+    for _ in range(args.steps):
+        for d, hsrc in zip(dsts, pins):
+            d.copy_(hsrc, non_blocking=True)
+        win.enqueue()
+        for o, c in zip(outs, (win.counts_nat_gold, win.counts_nat_f, win.counts_g_f)):
+            o.copy_(c, non_blocking=True)
+    f1.record()
+    torch.cuda.synchronize()
+    e2e_ms = f0.elapsed_time(f1) / args.steps
+    if dist:
+        t = torch.tensor([e2e_ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    if rank == 0:
+        pk = peaks()
+        gflops = win.golden_flops()
+        achieved = gflops / (stage_ms["golden"] * 1e-3) / 1e12
+        peak = pk["bf16_tflops_sustained"]
+        line = {
+            "metric": EVAL_METRIC, "value": world * 1e3 / ms, "unit": "windows/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": None, "kernel": "lidx_selection_eval (golden)",
+                         "peak_source": pk["source"] + " bf16, sustained", "flops_per_launch": gflops,
+                         "avg_launch_us": stage_ms["golden"] * 1e3},
+            "stages_ms": stage_ms,
+            "score_tflops": win.score_flops() / (stage_ms["score"] * 1e-3) / 1e12,
+            "e2e": {"value": world * 1e3 / e2e_ms, "unit": "windows/s",
+                    "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in pins),
+                    "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in outs)},
+            "gpu_launches": None,
+            "clocks": clk,
+        }
+        if world == 1:
+            dt, dw = oracle_eval_sample(spec, layers, gate)
+            line["cpu_baseline"] = {"value": dw / dt, "unit": "windows/s", "cores": 1, "kind": "oracle",
+                                    "sample": "golden probabilities, top-p and top-k of one query of one "
+                                              f"layer (1/{spec.L * spec.T} of a window), single thread"}
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="lidx", choices=["lidx", "reference"])
-    ap.add_argument("--workload", default="decode-64k", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="decode-64k", choices=sorted(WORKLOADS) + ["eval-window"])
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.workload == "eval-window":
+        e = synth.C5
+        cfg = {"workload": e.name, "layers": e.L, "queries": e.T, "heads": e.H, "entries": e.N, "top_k": e.k,
+               "top_p": f"{e.top_p_num}/{e.top_p_den}", "min_votes": e.min_votes,
+               "gate_layers": list(e.gate_layers), "l2": "inputs larger than L2 (704 MB of attention rows)",
+               "parallelism": f"replicas x{world}"}
+        if args.impl == "reference":
+            if rank == 0:
+                run_eval(args, cfg, rank, world, local_rank, reference=True)
+            return
+        run_eval(args, cfg, rank, world, local_rank)
+        return
     spec = WORKLOADS[args.workload]
     ab = algorithmic_bytes(spec)
     cfg = {"workload": spec.name, "layers": spec.layers, "batch": spec.B, "entries": spec.N, "heads": spec.H,

@@ -251,7 +251,7 @@ def topk_args(scores, k, allowed=None, ids=None, n_sel=None, mask=None, mask_bit
 
 
 def topk_select(scores: torch.Tensor, k: int, allowed: torch.Tensor = None, *, want_mask=False,
-                want_bits=False, ids=None, n_sel=None, ws=None, stream=None, tile_stats=None):
+                want_bits=False, ids=None, n_sel=None, ws=None, stream=None, tile_stats=None, bits=None):
     """Top-k row ids of scores [B][Q][N] (N = scores.shape[2]).
 
     Returns (ids int32 [B][Q][k] ascending with -1 padding, n_sel int32 [B][Q],
@@ -262,7 +262,8 @@ def topk_select(scores: torch.Tensor, k: int, allowed: torch.Tensor = None, *, w
     ids = torch.empty((B, Q, k), dtype=torch.int32, device=dev) if ids is None else ids
     n_sel = torch.empty((B, Q), dtype=torch.int32, device=dev) if n_sel is None else n_sel
     mask = torch.empty((B, Q, N), dtype=torch.uint8, device=dev) if want_mask else None
-    bits = torch.empty((B, Q, (N + 31) // 32), dtype=torch.int32, device=dev) if want_bits else None
+    if bits is None and want_bits:
+        bits = torch.empty((B, Q, (N + 31) // 32), dtype=torch.int32, device=dev)
     a = topk_args(scores, k, allowed, ids, n_sel, mask, bits, tile_stats=tile_stats)
     if ws is None:
         ws = workspace(workspace_size(OP_TOPK, a), dev)

@@ -312,7 +312,7 @@ size_t vote_bytes(const lidx_eval_args &a) {
 
 size_t eval_workspace(const lidx_eval_args &a) {
   size_t n = LIDX_WS_HEADER;
-  if (a.ops & LIDX_EVAL_GOLDEN) n += lse_bytes(a);
+  if (a.ops & LIDX_EVAL_GOLDEN) n += golden_tc_supported(a) ? golden_tc_workspace(a) : lse_bytes(a);
   if ((a.ops & LIDX_EVAL_VOTE) && !a.vote_bits) n += vote_bytes(a);
   return n;
 }
@@ -321,7 +321,10 @@ cudaError_t launch_eval(const lidx_eval_args &a, void *ws, cudaStream_t st) {
   uint32_t *status = static_cast<uint32_t *>(ws);
   char *cur = static_cast<char *>(ws) + LIDX_WS_HEADER;
   cudaError_t e;
-  if (a.ops & LIDX_EVAL_GOLDEN) {
+  if ((a.ops & LIDX_EVAL_GOLDEN) && golden_tc_supported(a)) {
+    if ((e = launch_golden_tc(a, cur, status, st)) != cudaSuccess) return e;
+    cur += golden_tc_workspace(a);
+  } else if (a.ops & LIDX_EVAL_GOLDEN) {
     float *lse2 = reinterpret_cast<float *>(cur);
     cur += lse_bytes(a);
     const size_t smem = (static_cast<size_t>(a.H) * kD + a.H) * sizeof(float);

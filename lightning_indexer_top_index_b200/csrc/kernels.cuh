@@ -30,6 +30,9 @@ size_t attn_workspace(const lidx_attn_args &a);
 cudaError_t launch_attn(const lidx_attn_args &a, void *ws, cudaStream_t st);
 
 // ---- selection evaluation
+bool golden_tc_supported(const lidx_eval_args &a);
+size_t golden_tc_workspace(const lidx_eval_args &a);
+cudaError_t launch_golden_tc(const lidx_eval_args &a, void *scratch, uint32_t *status, cudaStream_t st);
 size_t eval_workspace(const lidx_eval_args &a);
 cudaError_t launch_eval(const lidx_eval_args &a, void *ws, cudaStream_t st);
 

@@ -236,6 +236,23 @@ def test_golden_probs_parity():
         np.testing.assert_allclose(got[l], ref, rtol=1e-4, atol=1e-10)
 
 
+@pytest.mark.parametrize("T,N", [(3, 1100), (2, 256), (5, 2000)])
+def test_golden_probs_tensor_core(T, N):
+    """64 heads, bf16: the tcgen05 path (two queries per 128-row tile, 256-key
+    blocks); odd T leaves padding rows in the last tile, N a partial block."""
+    spec = synth.scaled(synth.C5, L=2, T=T, H=64, N=N)
+    qa = np.stack([synth.eval_layer(spec, l)["qa"] for l in range(spec.L)])
+    kvs = [synth.eval_layer(spec, l)["kv"] for l in range(spec.L)]
+    kv = synth.concat_kv(kvs)
+    probs = torch.full((spec.L, spec.T, spec.N), -1.0, device="cuda")
+    L.selection_eval(L.EVAL_GOLDEN, L=spec.L, T=spec.T, H=spec.H, N=spec.N, qa=dev_q(qa, "bf16"),
+                     kv=dev_kv(kv, batch_rows=spec.N), scale=spec.scale, probs=probs)
+    got = probs.cpu().numpy()
+    for l in range(spec.L):
+        ref = oracle.golden(qa[l], kvs[l], spec.T, spec.H, spec.N, spec.scale)
+        np.testing.assert_allclose(got[l], ref, rtol=1e-4, atol=1e-10)
+
+
 @pytest.mark.parametrize("N,conc", [(1, 1.0), (100, 0.5), (4097, 2.0), (32768, 1.0), (32768, 6.0)])
 def test_topp_bit_exact(N, conc):
     rows = 4
