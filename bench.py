@@ -366,7 +366,7 @@ def run_lidx(args, spec, cfg, rank, world, local_rank):
 
 # ------------------------------------------------------------- eval window
 EVAL_METRIC = "selection-eval windows/s (64 queries x 21 layers x 32K entries; golden TFLOP/s vs peak)"
-EVAL_STAGES = ("score", "topk", "golden", "gold_topk", "vote", "gate", "overlap")
+EVAL_STAGES = ("score", "topk", "golden", "topp", "gold_topk", "vote", "gate", "overlap")
 
 
 def eval_inputs(spec):

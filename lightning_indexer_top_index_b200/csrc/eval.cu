@@ -121,17 +121,28 @@ struct ToppSmem {
   uint32_t bad;
 };
 
+// The row is staged in shared memory once when it fits (kStage); every pass
+// then reads it from there.  The radix starts at the highest bit in which the
+// row's keys differ, and each thread folds runs of equal digits before its
+// atomic add, so rows whose probabilities share an exponent (one hot bin)
+// do not serialise on a single shared-memory address.
+template <bool kStage>
 __global__ void __launch_bounds__(kT, 1) topp_kernel(lidx_eval_args a, uint32_t *status) {
+  extern __shared__ float prow[];  // [N] when staged
   __shared__ ToppSmem sm;
+  __shared__ uint32_t red_lo[32], red_hi[32];
   const int row = blockIdx.x;
-  const float *p = a.probs + static_cast<size_t>(row) * a.N;
+  const float *gp = a.probs + static_cast<size_t>(row) * a.N;
   const int N = a.N, tid = threadIdx.x;
   const uint32_t lane = lane_id(), warp = tid >> 5;
   if (tid == 0) {
     sm.total = 0;
     sm.bad = 0;
   }
+  if (kStage)
+    for (int j = tid; j < N; j += kT) prow[j] = gp[j];
   __syncthreads();
+  const float *p = kStage ? prow : gp;
   auto key_mass = [&](int j, uint32_t &key, uint64_t &m) {
     const float x = p[j];
     if (!(x >= 0.f) || x > 1.f) {  // negative, > 1 or NaN: excluded
@@ -143,17 +154,31 @@ __global__ void __launch_bounds__(kT, 1) topp_kernel(lidx_eval_args a, uint32_t 
     key = order_key(x);
     m = mass_of(x);
   };
+  // total mass, and the range of keys that carry mass
   unsigned long long tot = 0;
+  uint32_t klo = 0xFFFFFFFFu, khi = 0u;
   for (int j = tid; j < N; j += kT) {
     uint32_t k;
     uint64_t m;
     key_mass(j, k, m);
     tot += m;
+    if (m) {
+      klo = min(klo, k);
+      khi = max(khi, k);
+    }
   }
   tot = warp_sum(tot);
-  if (lane == 0) atomicAdd(&sm.total, tot);
+  klo = __reduce_min_sync(0xFFFFFFFFu, klo);
+  khi = __reduce_max_sync(0xFFFFFFFFu, khi);
+  if (lane == 0) {
+    atomicAdd(&sm.total, tot);
+    red_lo[warp] = klo;
+    red_hi[warp] = khi;
+  }
   __syncthreads();
   if (tid == 0 && sm.bad) raise_status(status, LIDX_DEV_NAN);
+  klo = __reduce_min_sync(0xFFFFFFFFu, red_lo[lane]);
+  khi = __reduce_max_sync(0xFFFFFFFFu, red_hi[lane]);
   const uint64_t M = sm.total;
   const uint64_t q1 = M / a.top_p_den, r1 = M % a.top_p_den;
   const uint64_t rr = r1 * a.top_p_num;
@@ -162,34 +187,51 @@ __global__ void __launch_bounds__(kT, 1) topp_kernel(lidx_eval_args a, uint32_t 
   uint32_t T = 0xFFFFFFFFu;  // threshold key; nothing selected when Tm == 0
   uint32_t take_eq = 0;
   if (Tm > 0) {
-    uint32_t prefix = 0u, pmask = 0u;
+    // keys with mass share the bits above the highest differing one
+    const int bits_left = khi == klo ? 0 : 32 - __clz(klo ^ khi);
+    uint32_t pmask = bits_left >= 32 ? 0u : ~((1u << bits_left) - 1u);
+    uint32_t prefix = khi & pmask;
     uint64_t rem = Tm;
-    for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int hi = bits_left; hi > 0; hi -= 8) {
+      const int w = min(8, hi), shift = hi - w;
+      const uint32_t dmask = (1u << w) - 1u;
       if (tid < 256) sm.hist[tid] = 0ull;
       __syncthreads();
+      uint32_t run_d = 0xFFFFFFFFu;
+      unsigned long long run_m = 0;
       for (int j = tid; j < N; j += kT) {
         uint32_t k;
         uint64_t m;
         key_mass(j, k, m);
-        if (k != 0u && (k & pmask) == prefix && m) atomicAdd(&sm.hist[(k >> shift) & 0xFFu], (unsigned long long)m);
+        if (m && (k & pmask) == prefix) {
+          const uint32_t d = (k >> shift) & dmask;
+          if (d != run_d) {
+            if (run_m) atomicAdd(&sm.hist[run_d], run_m);
+            run_d = d;
+            run_m = 0;
+          }
+          run_m += m;
+        }
       }
+      if (run_m) atomicAdd(&sm.hist[run_d], run_m);
       __syncthreads();
+      const int nb = 1 << w;
       if (tid < 256) {
-        const unsigned long long v = sm.hist[255 - tid];
+        const unsigned long long v = tid < nb ? sm.hist[nb - 1 - tid] : 0ull;
         unsigned long long inc = warp_inclusive_scan(v);
         if (lane == 31) sm.warp_m[warp] = inc;
         asm volatile("bar.sync 1, 256;");
         unsigned long long before = 0;
-        for (int w = 0; w < static_cast<int>(warp); w++) before += sm.warp_m[w];
+        for (int ww = 0; ww < static_cast<int>(warp); ww++) before += sm.warp_m[ww];
         inc += before;
-        if (inc >= rem && inc - v < rem) {
-          sm.digit = 255u - tid;
+        if (tid < nb && inc >= rem && inc - v < rem) {
+          sm.digit = static_cast<uint32_t>(nb - 1 - tid);
           sm.above = inc - v;
         }
       }
       __syncthreads();
       prefix |= sm.digit << shift;
-      pmask |= 0xFFu << shift;
+      pmask |= dmask << shift;
       rem -= sm.above;
       __syncthreads();
     }
@@ -349,7 +391,13 @@ cudaError_t launch_eval(const lidx_eval_args &a, void *ws, cudaStream_t st) {
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   if (a.ops & LIDX_EVAL_TOPP) {
-    topp_kernel<<<a.L * a.T, kT, 0, st>>>(a, status);
+    const size_t row_bytes = static_cast<size_t>(a.N) * sizeof(float);
+    if (row_bytes <= 200u * 1024u) {
+      cudaFuncSetAttribute(topp_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(row_bytes));
+      topp_kernel<true><<<a.L * a.T, kT, row_bytes, st>>>(a, status);
+    } else {
+      topp_kernel<false><<<a.L * a.T, kT, 0, st>>>(a, status);
+    }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   const int Wn = (a.N + 31) / 32;

@@ -11,16 +11,23 @@
 //   pass 2  2^(c*logit - lse2) per element, then the mean over the H = 64
 //           heads of each query.
 // Tile: 128 rows (two queries x 64 heads) x 256 keys, K = 512 in eight
-// 64-wide panels.  Persistent CTAs walk a contiguous range of (layer, row
-// block, key block) units, key block fastest:
+// 64-wide panels.  Persistent CTAs take the (layer, key block, row block)
+// units round-robin, row block fastest: at any time all CTAs work on one
+// layer and a few key blocks, so each 256-key block is fetched from HBM once
+// and reused from L2 by the layer's row blocks (ranges per CTA would spread
+// the CTAs over every layer and re-read the keys once per row block):
 //   warp 0      TMA producer: per panel the 128 x 64 query box and the
-//               256 x 64 key box (128-byte swizzled) into a 3-stage ring
+//               256 x 64 key box (128-byte swizzled) into a 4-stage ring
 //   warp 1      TMEM allocation; one lane issues 4 MMAs per panel
 //               (M = 128, N = 256) into one of two TMEM accumulators
-//   warps 2-5   epilogue, thread = one row (its TMEM lane)
+//   warps 2-17  epilogue: warp w reads TMEM lane quarter w&3 (32 rows) and
+//               64 of the 256 columns, thread = one row; four warps per
+//               quarter keep the exponentials (one SFU op per element) and
+//               their latencies spread over the SM
 // Pass 2 sums over the 64 rows of a query with a transposed warp reduction
 // (each lane ends with one column's sum over the warp's 32 rows) and one
-// shared-memory exchange between the two warps of the query.
+// shared-memory exchange between the two warps of the query that share the
+// columns.
 #include <algorithm>
 
 #include "kernels.cuh"
@@ -35,11 +42,14 @@ constexpr int kHeads = 64;          // rows of a query
 constexpr int kTM = 128;            // rows per tile (two queries)
 constexpr int kTN = 256;            // keys per tile
 constexpr int kPanels = kD / 64;
-constexpr int kStages = 3;
+constexpr int kStages = 4;
 constexpr int kABytes = kTM * 128;  // one 64-wide panel of the query rows
 constexpr int kBBytes = kTN * 128;  // one 64-wide panel of the keys
 constexpr int kStageBytes = kABytes + kBBytes;
 constexpr uint32_t kTmemCols = 512;  // two 256-column accumulators
+constexpr int kEpiWarps = 16;        // 4 lane quarters x 4 column groups
+constexpr int kCG = kTN / 4;         // columns per epilogue warp
+constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct GoldenParams {
@@ -49,7 +59,7 @@ struct GoldenParams {
   long long units;
   int64_t key_rows;  // rows between layers in the key tensor map
   float c;           // scale * log2(e)
-  float2 *part;      // pass 1: [L][rows][n_kb]
+  float2 *part;      // pass 1: [L][rows][n_kb][4 column groups]
   const float *lse2; // pass 2: [L][rows]
   float *probs;      // pass 2: [L][T][N]
 };
@@ -68,10 +78,10 @@ constexpr size_t golden_smem_bytes() {
 }
 
 __device__ __forceinline__ void unit_coords(const GoldenParams &p, long long u, int &l, int &rb, int &kb) {
-  kb = static_cast<int>(u % p.n_kb);
-  const long long r = u / p.n_kb;
-  rb = static_cast<int>(r % p.n_rb);
-  l = static_cast<int>(r / p.n_rb);
+  rb = static_cast<int>(u % p.n_rb);
+  const long long r = u / p.n_rb;
+  kb = static_cast<int>(r % p.n_kb);
+  l = static_cast<int>(r / p.n_kb);
 }
 
 __device__ __forceinline__ void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n)); }
@@ -94,7 +104,7 @@ __device__ __forceinline__ float transpose_sum32(float (&v)[32]) {
 }
 
 template <int kPass>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     golden_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const GoldenParams p, uint32_t *status) {
   extern __shared__ uint8_t smem_raw[];
@@ -103,7 +113,7 @@ __global__ void __launch_bounds__(192, 1)
   GoldenBars *bar = reinterpret_cast<GoldenBars *>(sRed + 2 * kTN);
   volatile uint32_t *abort_flag = &bar->abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long u0 = blockIdx.x * p.units / gridDim.x, u1 = (blockIdx.x + 1) * p.units / gridDim.x;
+  const long long u0 = blockIdx.x, ustep = gridDim.x;  // units u0, u0 + ustep, ...
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; s++) {
@@ -112,7 +122,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int a = 0; a < 2; a++) {
       tc::mbar_init(&bar->tfull[a], 1);
-      tc::mbar_init(&bar->tempty[a], 4);
+      tc::mbar_init(&bar->tempty[a], kEpiWarps);
     }
     bar->abort = 0;
     tc::fence_barrier_init();
@@ -132,7 +142,7 @@ __global__ void __launch_bounds__(192, 1)
       uint32_t phase = 0;
       uint32_t last_par[kStages] = {};
       bool used[kStages] = {};
-      for (long long u = u0; u < u1 && !*abort_flag; u++) {
+      for (long long u = u0; u < p.units && !*abort_flag; u += ustep) {
         int l, rb, kb;
         unit_coords(p, u, l, rb, kb);
         const int qrow = l * p.rows + rb * kTM;
@@ -163,7 +173,7 @@ __global__ void __launch_bounds__(192, 1)
       uint32_t phase = 0, acc_par = 0;
       const uint32_t idesc = tc::idesc_bf16(kTM, kTN);
       const uint32_t base = tc::smem_u32(smem);
-      for (long long u = u0; u < u1; u++) {
+      for (long long u = u0; u < p.units; u += ustep) {
         if (!tc::mbar_wait(&bar->tempty[acc], acc_par ^ 1, abort_flag)) break;
         tc::tc_fence_after();
         const uint32_t d = tmem + acc * kTN;
@@ -196,10 +206,11 @@ __global__ void __launch_bounds__(192, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     const int quarter = warp & 3;  // TMEM lane quarter = rows [32q, 32q+32) of the tile
+    const int cg = (warp - 2) >> 2;  // column group: columns [64cg, 64cg + 64)
     const int trow = quarter * 32 + lane;
     int acc = 0;
     uint32_t acc_par = 0;
-    for (long long u = u0; u < u1; u++) {
+    for (long long u = u0; u < p.units; u += ustep) {
       int l, rb, kb;
       unit_coords(p, u, l, rb, kb);
       const int row = rb * kTM + trow;  // row of the layer: t * 64 + h
@@ -209,11 +220,11 @@ __global__ void __launch_bounds__(192, 1)
       ready = __shfl_sync(0xFFFFFFFFu, ready, 0);
       if (ready) {
         tc::tc_fence_after();
-        const uint32_t tbase = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + acc * kTN;
-        const int j0 = kb * kTN;
+        const uint32_t tbase = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + acc * kTN + cg * kCG;
+        const int j0 = kb * kTN + cg * kCG;
         if (kPass == 1) {
           float m = -INFINITY, s = 0.f;
-          for (int c0 = 0; c0 < kTN; c0 += 32) {
+          for (int c0 = 0; c0 < kCG; c0 += 32) {
             float v[32];
             tc::tmem_ld32(tbase + c0, v);
             float cm = -INFINITY;
@@ -231,34 +242,36 @@ __global__ void __launch_bounds__(192, 1)
               m = mn;
             }
           }
-          if (row_ok) p.part[(static_cast<size_t>(l) * p.rows + row) * p.n_kb + kb] = make_float2(m, s);
+          if (row_ok) p.part[((static_cast<size_t>(l) * p.rows + row) * p.n_kb + kb) * 4 + cg] = make_float2(m, s);
         } else {
           const float lse = row_ok ? p.lse2[static_cast<size_t>(l) * p.rows + row] : INFINITY;
           const int q = quarter >> 1;       // query of the tile
           const int t = rb * 2 + q;         // query of the layer
-          for (int c0 = 0; c0 < kTN; c0 += 32) {
+          const int bar_id = 1 + q * 4 + cg;  // the two warps of query q on these columns
+          for (int c0 = 0; c0 < kCG; c0 += 32) {
             float v[32];
             tc::tmem_ld32(tbase + c0, v);
 #pragma unroll
             for (int i = 0; i < 32; i++) v[i] = row_ok ? exp2f(v[i] * p.c - lse) : 0.f;
             const float colsum = transpose_sum32(v);  // column c0 + lane, this warp's 32 heads
-            if (quarter & 1) sRed[q * kTN + c0 + lane] = colsum;
-            named_sync(1 + q, 64);
+            float *red = sRed + q * kTN + cg * kCG + c0;
+            if (quarter & 1) red[lane] = colsum;
+            named_sync(bar_id, 64);
             if (!(quarter & 1)) {
               const int j = j0 + c0 + lane;
-              const float tot = colsum + sRed[q * kTN + c0 + lane];
+              const float tot = colsum + red[lane];
               if (t < p.T && j < p.N)
                 p.probs[(static_cast<size_t>(l) * p.T + t) * p.N + j] = tot * (1.f / kHeads);
             }
-            named_sync(1 + q, 64);  // the partner may overwrite sRed
+            named_sync(bar_id, 64);  // the partner may overwrite sRed
           }
         }
       } else if (kPass == 2) {
         // keep the named barriers of the pair matched on a give-up
-        const int q = quarter >> 1;
-        for (int c0 = 0; c0 < kTN; c0 += 32) {
-          named_sync(1 + q, 64);
-          named_sync(1 + q, 64);
+        const int bar_id = 1 + (quarter >> 1) * 4 + cg;
+        for (int c0 = 0; c0 < kCG; c0 += 32) {
+          named_sync(bar_id, 64);
+          named_sync(bar_id, 64);
         }
       }
       tc::tc_fence_before();
@@ -280,7 +293,7 @@ __global__ void __launch_bounds__(192, 1)
   if (threadIdx.x == 0 && bar->abort) raise_status(status, LIDX_DEV_TIMEOUT);
 }
 
-// lse2[l][row] = log2 sum over the key blocks' partials.
+// lse2[l][row] = log2 sum over the partials (key blocks x column groups).
 __global__ void golden_lse_merge_kernel(const float2 *part, int n, int n_kb, float *lse2) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= n) return;
@@ -317,7 +330,7 @@ bool golden_tc_supported(const lidx_eval_args &a) {
 size_t golden_tc_workspace(const lidx_eval_args &a) {
   const size_t rows = static_cast<size_t>(a.L) * a.T * a.H;
   const size_t n_kb = (a.N + kTN - 1) / kTN;
-  return ((rows * n_kb * sizeof(float2) + 255) / 256) * 256 + ((rows * sizeof(float) + 255) / 256) * 256;
+  return ((rows * n_kb * 4 * sizeof(float2) + 255) / 256) * 256 + ((rows * sizeof(float) + 255) / 256) * 256;
 }
 
 cudaError_t launch_golden_tc(const lidx_eval_args &a, void *scratch, uint32_t *status, cudaStream_t st) {
@@ -334,7 +347,7 @@ cudaError_t launch_golden_tc(const lidx_eval_args &a, void *scratch, uint32_t *s
   const size_t rows = static_cast<size_t>(a.L) * p.rows;
   p.part = static_cast<float2 *>(scratch);
   float *lse2 = reinterpret_cast<float *>(static_cast<char *>(scratch) +
-                                          ((rows * p.n_kb * sizeof(float2) + 255) / 256) * 256);
+                                          ((rows * p.n_kb * 4 * sizeof(float2) + 255) / 256) * 256);
   p.lse2 = lse2;
   p.probs = a.probs;
 
@@ -349,13 +362,13 @@ cudaError_t launch_golden_tc(const lidx_eval_args &a, void *scratch, uint32_t *s
   const int grid = static_cast<int>(std::min<long long>(p.units, sm_count()));
   cudaFuncSetAttribute(golden_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   cudaFuncSetAttribute(golden_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-  golden_tc_kernel<1><<<grid, 192, smem, st>>>(tm_q, tm_k, p, status);
+  golden_tc_kernel<1><<<grid, kThreads, smem, st>>>(tm_q, tm_k, p, status);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int n = static_cast<int>(rows);
-  golden_lse_merge_kernel<<<(n + 255) / 256, 256, 0, st>>>(p.part, n, p.n_kb, lse2);
+  golden_lse_merge_kernel<<<(n + 255) / 256, 256, 0, st>>>(p.part, n, p.n_kb * 4, lse2);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  golden_tc_kernel<2><<<grid, 192, smem, st>>>(tm_q, tm_k, p, status);
+  golden_tc_kernel<2><<<grid, kThreads, smem, st>>>(tm_q, tm_k, p, status);
   return cudaGetLastError();
 }
 

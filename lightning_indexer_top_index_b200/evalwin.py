@@ -74,8 +74,8 @@ class EvalWindow:
     def enqueue(self, stream=None, events: Optional[Dict] = None):
         """Issue the window's calls on `stream` (default: current).  With
         `events` (name -> (start, end) CUDA events) the stages "score",
-        "topk", "golden", "gold_topk", "vote", "gate" and "overlap" are
-        bracketed for timing."""
+        "topk", "golden", "topp", "gold_topk", "vote", "gate" and "overlap"
+        are bracketed for timing."""
         L, T, H, N, k = self.L, self.T, self.H, self.N, self.k
         st = stream or torch.cuda.current_stream()
 
@@ -94,9 +94,13 @@ class EvalWindow:
                         bits=self.nat_bits[l], ws=self.ws_topk_nat, stream=st)
         mark("topk", 1)
         mark("golden", 0)
-        selection_eval(EVAL_GOLDEN | EVAL_TOPP, L=L, T=T, H=H, N=N, qa=self.qa, kv=self.kv_all, scale=self.scale,
-                       probs=self.probs, top_p=self.top_p, topp_bits=self.topp_bits, ws=self.ws_golden, stream=st)
+        selection_eval(EVAL_GOLDEN, L=L, T=T, H=H, N=N, qa=self.qa, kv=self.kv_all, scale=self.scale,
+                       probs=self.probs, ws=self.ws_golden, stream=st)
         mark("golden", 1)
+        mark("topp", 0)
+        selection_eval(EVAL_TOPP, L=L, T=T, N=N, probs=self.probs, top_p=self.top_p, topp_bits=self.topp_bits,
+                       ws=self.ws_small, stream=st)
+        mark("topp", 1)
         mark("gold_topk", 0)
         topk_select(self.probs.view(L * T, 1, N), k, want_bits=True, ids=self.gold_ids, n_sel=self.gold_n,
                     bits=self.gold_bits, ws=self.ws_topk_gold, stream=st)
