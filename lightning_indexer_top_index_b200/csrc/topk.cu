@@ -62,6 +62,8 @@ struct SelSmem {
   uint32_t cnt_in[kMaxCluster], above_in[kMaxCluster];
   uint32_t gathered[kGatherMax];
   uint32_t red_a[kWarps], red_b[kWarps], red_c[kWarps], red_d[kWarps];
+  uint32_t scan[2][kWarps];
+  uint32_t cand_count;
   uint32_t red_tot;
   uint32_t digit, above, total;
   uint32_t T, need;
@@ -83,11 +85,12 @@ __device__ __forceinline__ void cluster_sync_hw() {
   asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-// Start barrier: every CTA arrives when it starts and waits before its first
-// access to another CTA's shared memory, which is only valid once all CTAs
-// of the cluster run.
+// Start barrier: every CTA arrives when it starts (after zeroing the slots
+// others add into; arrive releases, wait acquires) and waits before its first
+// access to another CTA's shared memory, which is only valid once all CTAs of
+// the cluster run.
 __device__ __forceinline__ void cluster_arrive_start() {
-  if (gridDim.x > 1) asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+  if (gridDim.x > 1) asm volatile("barrier.cluster.arrive.aligned;" ::: "memory");
 }
 __device__ __forceinline__ void cluster_wait_start() {
   if (gridDim.x > 1) asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
@@ -108,6 +111,13 @@ __device__ __forceinline__ void st_remote(uint32_t *p, uint32_t rank, uint32_t v
   uint32_t a;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(tc::smem_u32(p)), "r"(rank));
   asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
+}
+
+// Add to a 32-bit word of CTA `rank`'s shared memory.
+__device__ __forceinline__ void add_remote(uint32_t *p, uint32_t rank, uint32_t v) {
+  uint32_t a;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(tc::smem_u32(p)), "r"(rank));
+  asm volatile("red.shared::cluster.add.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
 }
 
 // Load a 32-bit word of CTA `rank`'s shared memory at the local address `p`.
@@ -149,21 +159,20 @@ __device__ __forceinline__ uint32_t cta_min(SelSmem &sm, uint32_t v) {
 __device__ __forceinline__ uint32_t cta_max(SelSmem &sm, uint32_t v) { return ~cta_min(sm, ~v); }
 
 // Exclusive CTA scan of 32-bit values; *total gets the CTA sum.
-__device__ __forceinline__ uint32_t cta_exclusive_scan(SelSmem &sm, uint32_t v, uint32_t &total) {
+// One barrier: every warp scans the 32 warp totals itself.  `buf` alternates
+// between two scratch rows, so a scan never overwrites totals the previous
+// scan's slower warps may still read (two scans apart there is a barrier).
+__device__ __forceinline__ uint32_t cta_exclusive_scan(SelSmem &sm, uint32_t v, uint32_t &total, int &buf) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const uint32_t inc = warp_inclusive_scan(v);
+  if (lane == 31) sm.scan[buf][warp] = inc;
   __syncthreads();
-  if (lane == 31) sm.red_a[warp] = inc;
-  __syncthreads();
-  if (warp == 0) {
-    const uint32_t x = sm.red_a[lane];
-    const uint32_t xi = warp_inclusive_scan(x);
-    sm.red_b[lane] = xi - x;
-    if (lane == 31) sm.red_tot = xi;
-  }
-  __syncthreads();
-  total = sm.red_tot;
-  return sm.red_b[warp] + inc - v;
+  const uint32_t x = sm.scan[buf][lane];
+  const uint32_t xi = warp_inclusive_scan(x);
+  total = __shfl_sync(0xFFFFFFFFu, xi, 31);
+  const uint32_t before = __shfl_sync(0xFFFFFFFFu, xi - x, warp);
+  buf ^= 1;
+  return before + inc - v;
 }
 
 // Merge the per-group histograms into pub.hist[buf].
@@ -271,6 +280,11 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelParams p) 
   const int s0 = static_cast<int>(rank) * p.slice;  // first position of this CTA's slice
   const int p0 = tid * C;                           // first position of this thread, within the slice
 
+  if (tid < kMaxCluster) {
+    sm.cnt_in[tid] = 0u;
+    sm.above_in[tid] = 0u;
+  }
+  if (tid == 0) sm.cand_count = 0u;
   cluster_arrive_start();
   pdl_trigger();
   pdl_wait();  // the scores come from the previous kernel
@@ -362,24 +376,31 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelParams p) 
   // exchange; this CTA has arrived on the final cluster barrier
   bool fast = false;
   auto resolve = [&](auto in_bin, auto above_bin, uint32_t rem) {
-    // this CTA's keys of the threshold bin (low 16 bits) and above it (high)
-    uint32_t nc = 0;
+    // push this CTA's keys of the threshold bin into slot `rank` of every CTA
+    // (positions from a CTA counter: order within a slot does not matter),
+    // and add its counts of those keys and of keys above the bin into every
+    // CTA's slot; the cluster barrier publishes both, no block barrier needed
+    const int lane = tid & 31;
+    uint32_t w_in = 0, w_above = 0;
 #pragma unroll
-    for (int i = 0; i < C; i++) nc += in_bin(i) ? 1u : above_bin(i) ? 0x10000u : 0u;
-    uint32_t packed_total;
-    uint32_t cpos = cta_exclusive_scan(sm, nc, packed_total) & 0xFFFFu;  // at most 32768 each
-    const uint32_t n_local = packed_total & 0xFFFFu;
-    // push the candidates into slot `rank` of every CTA, with the counts
-#pragma unroll
-    for (int i = 0; i < C; i++)
-      if (in_bin(i)) {
-        if (cpos < static_cast<uint32_t>(kSlot))
-          for (uint32_t r = 0; r < G; r++) st_remote(&sm.landing[rank][cpos], r, key[i]);
-        cpos++;
+    for (int i = 0; i < C; i++) {
+      const bool in = in_bin(i);
+      w_above += __popc(__ballot_sync(0xFFFFFFFFu, !in && above_bin(i)));
+      const uint32_t m = __ballot_sync(0xFFFFFFFFu, in);
+      if (m == 0u) continue;
+      uint32_t base = 0;
+      if (lane == 0) base = atomicAdd(&sm.cand_count, static_cast<uint32_t>(__popc(m)));
+      base = __shfl_sync(0xFFFFFFFFu, base, 0);
+      w_in += __popc(m);
+      if (in) {
+        const uint32_t pos = base + __popc(m & ((1u << lane) - 1u));
+        if (pos < static_cast<uint32_t>(kSlot))
+          for (uint32_t r = 0; r < G; r++) st_remote(&sm.landing[rank][pos], r, key[i]);
       }
-    if (static_cast<uint32_t>(tid) < G) {
-      st_remote(&sm.cnt_in[rank], tid, n_local);
-      st_remote(&sm.above_in[rank], tid, packed_total >> 16);
+    }
+    if (static_cast<uint32_t>(lane) < G) {
+      if (w_in) add_remote(&sm.cnt_in[rank], lane, w_in);
+      if (w_above) add_remote(&sm.above_in[rank], lane, w_above);
     }
     cluster_sync();
     if (tid < 32) {  // every CTA's counts, now local
@@ -681,7 +702,8 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelParams p) 
     n_eq += T != 0u && key[i] == T;
   }
   uint32_t cta_tot;
-  const uint32_t ex = cta_exclusive_scan(sm, (n_gt << 16) | n_eq, cta_tot);  // at most 32768 each
+  int scan_buf = 0;
+  const uint32_t ex = cta_exclusive_scan(sm, (n_gt << 16) | n_eq, cta_tot, scan_buf);  // at most 32768 each
   uint32_t gt_before = 0, eq_before = 0, gt_total = 0, eq_total = 0;
   if (fast) {
     for (uint32_t r = 0; r < G; r++) {
