@@ -77,11 +77,14 @@ constexpr size_t golden_smem_bytes() {
   return 1024 + static_cast<size_t>(kStages) * kStageBytes + 2 * kTN * sizeof(float) + sizeof(GoldenBars);
 }
 
+// 32-bit arithmetic (units < 2^31 is checked at launch): a 64-bit division
+// is a long software sequence.
 __device__ __forceinline__ void unit_coords(const GoldenParams &p, long long u, int &l, int &rb, int &kb) {
-  rb = static_cast<int>(u % p.n_rb);
-  const long long r = u / p.n_rb;
-  kb = static_cast<int>(r % p.n_kb);
-  l = static_cast<int>(r / p.n_kb);
+  const uint32_t uu = static_cast<uint32_t>(u), nrb = static_cast<uint32_t>(p.n_rb), nkb = static_cast<uint32_t>(p.n_kb);
+  rb = static_cast<int>(uu % nrb);
+  const uint32_t r = uu / nrb;
+  kb = static_cast<int>(r % nkb);
+  l = static_cast<int>(r / nkb);
 }
 
 __device__ __forceinline__ void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n)); }
@@ -324,7 +327,8 @@ bool golden_tc_supported(const lidx_eval_args &a) {
   if ((a.kv.ld * 2) % 16 != 0) return false;
   const int64_t qrows = static_cast<int64_t>(a.L) * a.T * a.H;
   const int64_t krows = static_cast<int64_t>(a.L - 1) * (a.L > 1 ? a.kv.batch_rows : 0) + a.N;
-  return qrows < (1ll << 31) && krows < (1ll << 31);
+  const int64_t units = static_cast<int64_t>(a.L) * ((a.T * kHeads + kTM - 1) / kTM) * ((a.N + kTN - 1) / kTN);
+  return qrows < (1ll << 31) && krows < (1ll << 31) && units < (1ll << 31);
 }
 
 size_t golden_tc_workspace(const lidx_eval_args &a) {

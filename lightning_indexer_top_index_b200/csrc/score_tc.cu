@@ -12,10 +12,14 @@
 //               through a kStages-deep ring of shared-memory stages
 //   warp 1      allocates TMEM; one lane issues the MMAs (K = 128 in steps of
 //               16) into one of two TMEM accumulators and commits
-//   warps 2-5   epilogue: each thread owns one key row (its TMEM lane), loads
-//               the H head dots of each query and reduces sum_h w_h max(x,0)
-//               in registers; 128 consecutive scores per query are stored
-//   warps 6-9   (E4M3 keys only) convert the FP8 non-RoPE half of each key
+//   warps 2-9   epilogue, two groups of four warps taking alternate tiles
+//               (group k reduces accumulator k): each thread owns one key row
+//               (its TMEM lane), loads the H head dots of each query and
+//               reduces sum_h w_h max(x,0) in registers; 128 consecutive
+//               scores per query are stored.  Two groups keep the reduction,
+//               which one warp per SM sub-partition cannot hide, off the
+//               critical path.
+//   warps 10-13 (E4M3 keys only) convert the FP8 non-RoPE half of each key
 //               tile to bf16 in the 128-byte-swizzled layout the MMA reads;
 //               the RoPE half arrives by TMA directly.  The power-of-two
 //               block scale is applied in the epilogue to a separate
@@ -35,6 +39,8 @@ constexpr int kTileM = 128;
 constexpr int kTileBytes = kTileM * 128 * 2;  // bf16 [128][128] as two 64-wide swizzled panels
 constexpr int kPanelBytes = kTileBytes / 2;
 constexpr int kF8Bytes = kTileM * 64;         // raw E4M3 half-tile
+constexpr int kEpiGroups = 2;                 // epilogue groups of four warps
+constexpr int kConvWarp0 = 2 + 4 * kEpiGroups;  // first FP8 converter warp
 
 struct TcParams {
   int B, Q, H, N;
@@ -68,20 +74,37 @@ struct __align__(8) TcBarriers {
 
 __host__ __device__ constexpr size_t tc_smem_bytes(int NM, bool fp8) {
   return 1024 + static_cast<size_t>(kStages) * kTileBytes + 2ull * NM * 128 + (fp8 ? kStages * kF8Bytes : 0) +
-         256 * sizeof(float) + sizeof(TcBarriers);
+         kEpiGroups * 256 * sizeof(float) + sizeof(TcBarriers);
 }
 
-__device__ __forceinline__ void unit_coords(const TcParams &p, long long u, int &b, int &g, int &t, long long &bg) {
-  bg = u / p.n_tiles;
-  t = static_cast<int>(u % p.n_tiles);
-  b = static_cast<int>(bg / p.n_groups);
-  g = static_cast<int>(bg % p.n_groups);
-}
+// Coordinates (sequence b, query group g, key tile t; bg = b * n_groups + g)
+// of consecutive units, t fastest.  Only `init` divides: 64-bit divisions are
+// long software sequences, too slow to repeat per tile in the pipeline roles.
+struct UnitCursor {
+  int b, g, t;
+  long long bg;
+  __device__ __forceinline__ void init(const TcParams &p, long long u) {
+    bg = u / p.n_tiles;
+    t = static_cast<int>(u % p.n_tiles);
+    b = static_cast<int>(bg / p.n_groups);
+    g = static_cast<int>(bg % p.n_groups);
+  }
+  __device__ __forceinline__ void next(const TcParams &p) {
+    if (++t == p.n_tiles) {
+      t = 0;
+      ++bg;
+      if (++g == p.n_groups) {
+        g = 0;
+        ++b;
+      }
+    }
+  }
+};
 
 __device__ __forceinline__ void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n)); }
 
 template <bool kFp8>
-__global__ void __launch_bounds__(kFp8 ? 320 : 192, 1)
+__global__ void __launch_bounds__(kFp8 ? 32 * kConvWarp0 + 128 : 32 * kConvWarp0, 1)
     score_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_rope,
                     const __grid_constant__ CUtensorMap tm_q, const TcParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -90,7 +113,7 @@ __global__ void __launch_bounds__(kFp8 ? 320 : 192, 1)
   uint8_t *sB = sA + kStages * kTileBytes;
   uint8_t *sF8 = sB + 2 * p.NM * 128;
   float *sW = reinterpret_cast<float *>(sF8 + (kFp8 ? kStages * kF8Bytes : 0));
-  TcBarriers *bar = reinterpret_cast<TcBarriers *>(sW + 256);
+  TcBarriers *bar = reinterpret_cast<TcBarriers *>(sW + kEpiGroups * 256);
   volatile uint32_t *abort_flag = &bar->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -99,11 +122,8 @@ __global__ void __launch_bounds__(kFp8 ? 320 : 192, 1)
   // Key tiles of the first kStages units: cache-side data, issued before the
   // block sync and before waiting for the previous kernel on the stream.
   const long long n_pre = min(static_cast<long long>(kStages), u1 - u0);
-  auto issue_a = [&](long long u, int stage) {
-    int b, g, t;
-    long long bg;
-    unit_coords(p, u, b, g, t, bg);
-    const int row = static_cast<int>(b * p.key_batch_rows + static_cast<int64_t>(t) * kTileM);
+  auto issue_a = [&](const UnitCursor &c, int stage) {
+    const int row = static_cast<int>(c.b * p.key_batch_rows + static_cast<int64_t>(c.t) * kTileM);
     uint8_t *a = sA + stage * kTileBytes;
     if (kFp8) {
       tc::mbar_arrive_expect_tx(&bar->full[stage], kF8Bytes + kPanelBytes);
@@ -132,7 +152,9 @@ __global__ void __launch_bounds__(kFp8 ? 320 : 192, 1)
     tc::tma_prefetch_desc(&tm_a);
     tc::tma_prefetch_desc(&tm_q);
     if (kFp8) tc::tma_prefetch_desc(&tm_rope);
-    for (long long i = 0; i < n_pre; i++) issue_a(u0 + i, static_cast<int>(i));
+    UnitCursor c;
+    c.init(p, u0);
+    for (long long i = 0; i < n_pre; i++, c.next(p)) issue_a(c, static_cast<int>(i));
   }
   if (warp == 1) tc::tmem_alloc(&bar->tmem_base, p.tmem_cols);
   tc::tc_fence_before();
@@ -157,10 +179,11 @@ __global__ void __launch_bounds__(kFp8 ? 320 : 192, 1)
       uint32_t bfull_last = 0;
       long long prev_bg = -1;
       pdl_wait();  // queries and weights may come from the previous kernel
-      for (long long u = u0; u < u1; u++) {
-        int b, g, t;
-        long long bg;
-        unit_coords(p, u, b, g, t, bg);
+      UnitCursor c;
+      c.init(p, u0);
+      for (long long u = u0; u < u1; u++, c.next(p)) {
+        const int b = c.b, g = c.g;
+        const long long bg = c.bg;
         if (bg != prev_bg) {
           if (prev_bg != -1) {
             if (!tc::mbar_wait(&bar->bempty, bempty_par, abort_flag)) break;
@@ -176,7 +199,7 @@ __global__ void __launch_bounds__(kFp8 ? 320 : 192, 1)
         }
         if (u - u0 < n_pre) continue;  // key tile already in flight
         if (!tc::mbar_wait(&bar->empty[stage], phase ^ 1, abort_flag)) break;
-        issue_a(u, stage);
+        issue_a(c, stage);
         last_par[stage] = phase;
         used[stage] = true;
         if (++stage == kStages) {
@@ -198,10 +221,10 @@ __global__ void __launch_bounds__(kFp8 ? 320 : 192, 1)
       long long prev_bg = -1;
       const uint32_t idesc = tc::idesc_bf16(kTileM, kFp8 ? p.H : p.NM);
       const uint32_t a_base = tc::smem_u32(sA), b_base = tc::smem_u32(sB);
-      for (long long u = u0; u < u1; u++) {
-        int b, g, t;
-        long long bg;
-        unit_coords(p, u, b, g, t, bg);
+      UnitCursor c;
+      c.init(p, u0);
+      for (long long u = u0; u < u1; u++, c.next(p)) {
+        const long long bg = c.bg;
         if (bg != prev_bg) {
           if (prev_bg != -1) tc::mma_commit(&bar->bempty);
           if (!tc::mbar_wait(&bar->bfull, bfull_par, abort_flag)) break;
@@ -241,26 +264,32 @@ __global__ void __launch_bounds__(kFp8 ? 320 : 192, 1)
         }
       }
     }
-  } else if (warp < 6) {
+  } else if (warp < kConvWarp0) {
     // ------------------------------------------------------------ epilogue
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
-    const int etid = threadIdx.x - 64;
+    const int grp = (warp - 2) >> 2;             // takes units u0 + grp, u0 + grp + 2, ...
+    const int etid = threadIdx.x - 64 - 128 * grp;
+    float *gW = sW + grp * 256;                   // this group's head weights
     pdl_wait();  // head weights may come from the previous kernel
-    int acc = 0;
+    const int acc = grp;
     uint32_t acc_par = 0;
     long long prev_bg = -1;
     // E4M3 block scales of this thread's key row, loaded two units ahead so
     // that their latency hides behind the tiles in between
-    auto load_scale = [&](long long u) -> float {
-      if (!kFp8 || u >= u1) return 0.f;
-      int b, g, t;
-      long long bg;
-      unit_coords(p, u, b, g, t, bg);
-      const int j = t * kTileM + row;
-      return j < p.N ? e8m0_to_f32(p.scale[(b * p.key_batch_rows + j) * p.ld_scale]) : 0.f;
+    auto load_scale = [&](const UnitCursor &cu, bool valid) -> float {
+      if (!kFp8 || !valid) return 0.f;
+      const int j = cu.t * kTileM + row;
+      return j < p.N ? e8m0_to_f32(p.scale[(cu.b * p.key_batch_rows + j) * p.ld_scale]) : 0.f;
     };
-    float sc_next0 = load_scale(u0), sc_next1 = load_scale(u0 + 1);
+    UnitCursor cs;  // runs two of this group's units ahead of the tile being reduced
+    cs.init(p, u0 + grp);
+    float sc_next0 = load_scale(cs, u0 + grp < u1);
+    cs.next(p);
+    cs.next(p);
+    float sc_next1 = load_scale(cs, u0 + grp + 2 < u1);
+    cs.next(p);
+    cs.next(p);
     // Score bounds of this warp's 32 keys of a tile (one span record), for the
     // top-k: the largest and the smallest non-NaN order key.  Called by whole
     // warps.
@@ -272,19 +301,22 @@ __global__ void __launch_bounds__(kFp8 ? 320 : 192, 1)
       if (lane == 0 && j0 < p.N)
         reinterpret_cast<uint2 *>(p.stats)[static_cast<size_t>(srow) * p.n_spans + j0 / 32] = make_uint2(mx, mn);
     };
-    for (long long u = u0; u < u1; u++) {
-      int b, g, t;
-      long long bg;
-      unit_coords(p, u, b, g, t, bg);
+    UnitCursor c;
+    c.init(p, u0 + grp);
+    for (long long u = u0 + grp; u < u1; u += kEpiGroups, c.next(p), c.next(p)) {
+      const int b = c.b, g = c.g, t = c.t;
+      const long long bg = c.bg;
       const float sc = sc_next0;
       sc_next0 = sc_next1;
-      sc_next1 = load_scale(u + 2);
+      sc_next1 = load_scale(cs, u + 4 < u1);
+      cs.next(p);
+      cs.next(p);
       if (bg != prev_bg) {
-        named_sync(2, 128);
+        named_sync(2 + grp, 128);
         const int nq = min(p.QG, p.Q - g * p.QG);
         for (int i = etid; i < p.QG * p.H; i += 128)
-          sW[i] = (i / p.H) < nq ? p.w[static_cast<int64_t>(b * p.Q + g * p.QG) * p.H + i] : 0.f;
-        named_sync(2, 128);
+          gW[i] = (i / p.H) < nq ? p.w[static_cast<int64_t>(b * p.Q + g * p.QG) * p.H + i] : 0.f;
+        named_sync(2 + grp, 128);
         prev_bg = bg;
       }
       // lane 0 waits, the warp follows its verdict; after a give-up the
@@ -304,7 +336,7 @@ __global__ void __launch_bounds__(kFp8 ? 320 : 192, 1)
             tc::tmem_ld32(base + c0, v);
             tc::tmem_ld32(base + p.H + c0, r);
 #pragma unroll
-            for (int i = 0; i < 32; i++) s = fmaf(sW[c0 + i], fmaxf(fmaf(sc, v[i], r[i]), 0.f), s);
+            for (int i = 0; i < 32; i++) s = fmaf(gW[c0 + i], fmaxf(fmaf(sc, v[i], r[i]), 0.f), s);
           }
           if (j < p.N) p.scores[static_cast<int64_t>(b * p.Q + g) * p.ld_scores + j] = s;
           if (p.stats) span_stats(s, j < p.N, b * p.Q + g, t);
@@ -314,7 +346,7 @@ __global__ void __launch_bounds__(kFp8 ? 320 : 192, 1)
             for (int c0 = 0; c0 < p.H; c0 += 32) {
               tc::tmem_ld32(base + qi * p.H + c0, v);
 #pragma unroll
-              for (int i = 0; i < 32; i++) s = fmaf(sW[qi * p.H + c0 + i], fmaxf(v[i], 0.f), s);
+              for (int i = 0; i < 32; i++) s = fmaf(gW[qi * p.H + c0 + i], fmaxf(v[i], 0.f), s);
             }
             const int qq = g * p.QG + qi;
             if (j < p.N && qq < p.Q) p.scores[static_cast<int64_t>(b * p.Q + qq) * p.ld_scores + j] = s;
@@ -325,10 +357,7 @@ __global__ void __launch_bounds__(kFp8 ? 320 : 192, 1)
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0 && ready) tc::mbar_arrive(&bar->tempty[acc]);
-      if (++acc == 2) {
-        acc = 0;
-        acc_par ^= 1;
-      }
+      acc_par ^= 1;
     }
   } else if (kFp8) {
     // ------------------------------------------------------------ FP8 -> bf16
@@ -336,7 +365,7 @@ __global__ void __launch_bounds__(kFp8 ? 320 : 192, 1)
     // each 8-lane phase reads 128 contiguous bytes of the raw half-tile and
     // writes 8 distinct 16-byte slots of the swizzled panel (no bank
     // conflicts either way).
-    const int t = threadIdx.x - 192;
+    const int t = threadIdx.x - 32 * kConvWarp0;
     int stage = 0;
     uint32_t phase = 0;
     for (long long u = u0; u < u1; u++) {
@@ -450,10 +479,12 @@ cudaError_t launch_score_tc(const lidx_score_args &a, cudaStream_t st) {
   const int grid = static_cast<int>(std::min<long long>(p.units, sm_count()));
   if (fp8) {
     cudaFuncSetAttribute(score_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    return launch_kernel(score_tc_kernel<true>, dim3(grid), dim3(320), smem, st, pdl, tm_a, tm_rope, tm_q, p);
+    return launch_kernel(score_tc_kernel<true>, dim3(grid), dim3(32 * kConvWarp0 + 128), smem, st, pdl, tm_a, tm_rope,
+                         tm_q, p);
   } else {
     cudaFuncSetAttribute(score_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    return launch_kernel(score_tc_kernel<false>, dim3(grid), dim3(192), smem, st, pdl, tm_a, tm_rope, tm_q, p);
+    return launch_kernel(score_tc_kernel<false>, dim3(grid), dim3(32 * kConvWarp0), smem, st, pdl, tm_a, tm_rope, tm_q,
+                         p);
   }
 }
 
