@@ -110,6 +110,37 @@ def profiled_traffic(workload: str, call: str):
     return d.get("dram_bytes_per_launch")
 
 
+def init_group(world: int, device=None, backend: str = "nccl"):
+    """The process group of a `world`-rank run (rank and rendezvous from the
+    environment torchrun sets), or None for one rank.  Replicas exchange
+    nothing on the data path: the group carries barriers and the timing
+    reduction only."""
+    if world <= 1:
+        return None
+    import datetime
+    import torch.distributed as dist
+    kw = {} if device is None else {"device_id": device}
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
+    return dist
+
+
+def job_rate(units_per_rank: float, world: int, ms: float) -> float:
+    """Whole-job throughput per second: the units every rank processed over
+    the slowest rank's time per step."""
+    return world * units_per_rank * 1e3 / ms
+
+
+def max_over_ranks(x: float, dist, device=None) -> float:
+    """The largest value over the ranks of the process group (the job's time
+    is its slowest replica's); `x` itself without a process group."""
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 # --------------------------------------------------------------------- clocks
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -243,11 +274,7 @@ def run_lidx(args, spec, cfg, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     device = torch.device("cuda", local_rank)
-    dist = None
-    if world > 1:
-        import torch.distributed as dist
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    dist = init_group(world, device)
 
     layers_inp = [synth.decode_layer(spec, l) for l in range(spec.layers)]
     ab = algorithmic_bytes(spec)
@@ -277,11 +304,8 @@ def run_lidx(args, spec, cfg, rank, world, local_rank):
     e1.record()
     torch.cuda.synchronize()
     clk = clocks.stop()
-    ms = e0.elapsed_time(e1) / args.steps
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dist, device)
     if dist:
-        t = torch.tensor([ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
         dist.barrier()
 
     # ---- live per-call timing: the same step with external events around
@@ -323,11 +347,7 @@ def run_lidx(args, spec, cfg, rank, world, local_rank):
         out_p.copy_(s.out, non_blocking=True)
     f1.record()
     torch.cuda.synchronize()
-    e2e_ms = f0.elapsed_time(f1) / args.steps
-    if dist:
-        t = torch.tensor([e2e_ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1) / args.steps, dist, device)
     h2d = sum(x.numel() * x.element_size() for x in (q_idx_p, w_p, q_attn_p))
     d2h = out_p.numel() * out_p.element_size()
 
@@ -336,7 +356,7 @@ def run_lidx(args, spec, cfg, rank, world, local_rank):
         dom = max(calls, key=lambda c: call_ms[c])
         achieved = ab["per_call"][dom] / (call_ms[dom] * 1e-3) / 1e9
         line = {
-            "metric": METRIC, "value": world * 1e3 / ms, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "metric": METRIC, "value": job_rate(1, world, ms), "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16" if spec.key_dtype == "bf16" else spec.key_dtype,
             "data": "synthetic", "config": cfg,
@@ -347,7 +367,7 @@ def run_lidx(args, spec, cfg, rank, world, local_rank):
                          "bytes_per_launch": ab["per_call"][dom], "avg_launch_us": call_ms[dom] * 1e3},
             "calls": {CALL_NAMES[c]: {"avg_launch_us": call_ms[c] * 1e3, "bytes_per_launch": ab["per_call"][c],
                                       "gbs": ab["per_call"][c] / (call_ms[c] * 1e-3) / 1e9} for c in calls},
-            "e2e": {"value": world * 1e3 / e2e_ms, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "e2e": {"value": job_rate(1, world, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": args.steps * steps[0].kernel_launches(),
             "clocks": clk,
         }
@@ -416,11 +436,7 @@ def run_eval(args, cfg, rank, world, local_rank, reference=False):
 
     torch.cuda.set_device(local_rank)
     device = torch.device("cuda", local_rank)
-    dist = None
-    if world > 1:
-        import torch.distributed as dist
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    dist = init_group(world, device)
     layers, gate = eval_inputs(spec)
 
     def bf(a):
@@ -452,11 +468,7 @@ def run_eval(args, cfg, rank, world, local_rank, reference=False):
     e1.record()
     torch.cuda.synchronize()
     clk = clocks.stop()
-    ms = e0.elapsed_time(e1) / args.steps
-    if dist:
-        t = torch.tensor([ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dist, device)
     # per-stage times (events between stages)
     ev = {n: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for n in EVAL_STAGES}
     stage_ms = {n: 0.0 for n in EVAL_STAGES}
@@ -481,18 +493,14 @@ def run_eval(args, cfg, rank, world, local_rank, reference=False):
             o.copy_(c, non_blocking=True)
     f1.record()
     torch.cuda.synchronize()
-    e2e_ms = f0.elapsed_time(f1) / args.steps
-    if dist:
-        t = torch.tensor([e2e_ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1) / args.steps, dist, device)
     if rank == 0:
         pk = peaks()
         gflops = win.golden_flops()
         achieved = gflops / (stage_ms["golden"] * 1e-3) / 1e12
         peak = pk["bf16_tflops_sustained"]
         line = {
-            "metric": EVAL_METRIC, "value": world * 1e3 / ms, "unit": "windows/s", "n_gpus": world,
+            "metric": EVAL_METRIC, "value": job_rate(1, world, ms), "unit": "windows/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
@@ -501,7 +509,7 @@ def run_eval(args, cfg, rank, world, local_rank, reference=False):
                          "avg_launch_us": stage_ms["golden"] * 1e3},
             "stages_ms": stage_ms,
             "score_tflops": win.score_flops() / (stage_ms["score"] * 1e-3) / 1e12,
-            "e2e": {"value": world * 1e3 / e2e_ms, "unit": "windows/s",
+            "e2e": {"value": job_rate(1, world, e2e_ms), "unit": "windows/s",
                     "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in pins),
                     "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in outs)},
             "gpu_launches": None,
