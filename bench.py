@@ -512,7 +512,7 @@ def run_eval(args, cfg, rank, world, local_rank, reference=False):
             "e2e": {"value": job_rate(1, world, e2e_ms), "unit": "windows/s",
                     "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in pins),
                     "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in outs)},
-            "gpu_launches": None,
+            "gpu_launches": args.steps * win.kernel_launches(),
             "clocks": clk,
         }
         if world == 1:

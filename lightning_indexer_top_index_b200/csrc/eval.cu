@@ -110,8 +110,16 @@ __device__ __forceinline__ uint64_t mass_of(float p) {
   return __float2ull_rd(p * 1099511627776.0f);
 }
 
+// Digit masses are kept as two 32-bit sums, mass = hi * 2^kLoBits + lo, which
+// the shared-memory atomic units add natively.  Exact whenever the row's total
+// mass is below 2^(32 + kLoBits) (every hi sum is at most total >> kLoBits)
+// and N < 2^(32 - kLoBits) (every lo sum is below 2^kLoBits per run); other
+// rows take 64-bit adds.
+constexpr int kLoBits = 11;
+
 struct ToppSmem {
   unsigned long long hist[256];
+  uint32_t hist_hi[256], hist_lo[256];
   unsigned long long warp_m[32];
   uint32_t warp_a[32];
   unsigned long long total;
@@ -180,6 +188,15 @@ __global__ void __launch_bounds__(kT, 1) topp_kernel(lidx_eval_args a, uint32_t 
   klo = __reduce_min_sync(0xFFFFFFFFu, red_lo[lane]);
   khi = __reduce_max_sync(0xFFFFFFFFu, red_hi[lane]);
   const uint64_t M = sm.total;
+  const bool split = M < (1ull << (32 + kLoBits)) && N < (1 << (32 - kLoBits));
+  auto add_mass = [&](uint32_t d, unsigned long long m) {
+    if (split) {
+      atomicAdd(&sm.hist_hi[d], static_cast<uint32_t>(m >> kLoBits));
+      atomicAdd(&sm.hist_lo[d], static_cast<uint32_t>(m & ((1u << kLoBits) - 1u)));
+    } else {
+      atomicAdd(&sm.hist[d], m);
+    }
+  };
   const uint64_t q1 = M / a.top_p_den, r1 = M % a.top_p_den;
   const uint64_t rr = r1 * a.top_p_num;
   const uint64_t Tm = q1 * a.top_p_num + rr / a.top_p_den + (rr % a.top_p_den != 0);
@@ -195,7 +212,11 @@ __global__ void __launch_bounds__(kT, 1) topp_kernel(lidx_eval_args a, uint32_t 
     for (int hi = bits_left; hi > 0; hi -= 8) {
       const int w = min(8, hi), shift = hi - w;
       const uint32_t dmask = (1u << w) - 1u;
-      if (tid < 256) sm.hist[tid] = 0ull;
+      if (tid < 256) {
+        sm.hist[tid] = 0ull;
+        sm.hist_hi[tid] = 0u;
+        sm.hist_lo[tid] = 0u;
+      }
       __syncthreads();
       uint32_t run_d = 0xFFFFFFFFu;
       unsigned long long run_m = 0;
@@ -206,18 +227,22 @@ __global__ void __launch_bounds__(kT, 1) topp_kernel(lidx_eval_args a, uint32_t 
         if (m && (k & pmask) == prefix) {
           const uint32_t d = (k >> shift) & dmask;
           if (d != run_d) {
-            if (run_m) atomicAdd(&sm.hist[run_d], run_m);
+            if (run_m) add_mass(run_d, run_m);
             run_d = d;
             run_m = 0;
           }
           run_m += m;
         }
       }
-      if (run_m) atomicAdd(&sm.hist[run_d], run_m);
+      if (run_m) add_mass(run_d, run_m);
       __syncthreads();
       const int nb = 1 << w;
       if (tid < 256) {
-        const unsigned long long v = tid < nb ? sm.hist[nb - 1 - tid] : 0ull;
+        const int x = nb - 1 - tid;
+        const unsigned long long v =
+            tid >= nb ? 0ull
+            : split   ? (static_cast<unsigned long long>(sm.hist_hi[x]) << kLoBits) + sm.hist_lo[x]
+                      : sm.hist[x];
         unsigned long long inc = warp_inclusive_scan(v);
         if (lane == 31) sm.warp_m[warp] = inc;
         asm volatile("bar.sync 1, 256;");

@@ -297,16 +297,38 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // lse2[l][row] = log2 sum over the partials (key blocks x column groups).
+// One warp per row: the lanes read the row's (max, sum) pairs two at a time
+// with coalesced 16-byte loads in a single pass, keep an online (max, sum),
+// and fold the 32 lane states with shuffles.  n_kb is a multiple of 4 and
+// the partials are 16-byte aligned.
+__device__ __forceinline__ void lse_fold(float &M, float &S, float m, float s) {
+  if (m == -INFINITY) return;
+  if (m > M) {
+    S = S * exp2f(M - m) + s;
+    M = m;
+  } else {
+    S += s * exp2f(m - M);
+  }
+}
+
 __global__ void golden_lse_merge_kernel(const float2 *part, int n, int n_kb, float *lse2) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  const int lane = threadIdx.x & 31;
+  const int i = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (i >= n) return;
-  const float2 *pp = part + static_cast<size_t>(i) * n_kb;
-  float M = -INFINITY;
-  for (int b = 0; b < n_kb; b++) M = fmaxf(M, pp[b].x);
-  float S = 0.f;
-  if (M != -INFINITY)
-    for (int b = 0; b < n_kb; b++) S += pp[b].x == -INFINITY ? 0.f : pp[b].y * exp2f(pp[b].x - M);
-  lse2[i] = M + log2f(S);
+  const float4 *pp = reinterpret_cast<const float4 *>(part + static_cast<size_t>(i) * n_kb);
+  float M = -INFINITY, S = 0.f;
+  for (int b = lane; b < (n_kb >> 1); b += 32) {
+    const float4 v = __ldcs(pp + b);
+    lse_fold(M, S, v.x, v.y);
+    lse_fold(M, S, v.z, v.w);
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    const float m2 = __shfl_xor_sync(0xffffffffu, M, o);
+    const float s2 = __shfl_xor_sync(0xffffffffu, S, o);
+    lse_fold(M, S, m2, s2);
+  }
+  if (lane == 0) lse2[i] = M + log2f(S);
 }
 
 int sm_count() {
@@ -370,7 +392,7 @@ cudaError_t launch_golden_tc(const lidx_eval_args &a, void *scratch, uint32_t *s
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int n = static_cast<int>(rows);
-  golden_lse_merge_kernel<<<(n + 255) / 256, 256, 0, st>>>(p.part, n, p.n_kb * 4, lse2);
+  golden_lse_merge_kernel<<<(n + 7) / 8, 256, 0, st>>>(p.part, n, p.n_kb * 4, lse2);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   golden_tc_kernel<2><<<grid, kThreads, smem, st>>>(tm_q, tm_k, p, status);
   return cudaGetLastError();

@@ -125,6 +125,15 @@ class EvalWindow:
                        n_pairs=1, counts=self.counts_g_f, ws=self.ws_small, stream=st)
         mark("overlap", 1)
 
+    def kernel_launches(self) -> int:
+        """Kernels one window launches: per layer a scorer and a top-k, the
+        golden probabilities (two tensor-core passes around the lse merge on
+        the tcgen05 path, else the lse and probability kernels), top-p, the
+        golden top-k, the vote and its union, a scorer per gate layer and the
+        gate OR, and three overlap counts."""
+        golden = 3 if self.H == 64 and self.qa.dtype == torch.bfloat16 and self.kv_all.dtype == BF16 else 2
+        return 2 * self.L + golden + 1 + 1 + 2 + len(self.gate_layers) + 1 + 3
+
     def golden_flops(self) -> float:
         """Tensor FLOPs of the golden passes: two GEMMs of (T*H) x N x 512 per layer."""
         return 2.0 * self.L * 2.0 * self.T * self.H * self.N * 512

@@ -74,3 +74,30 @@ def topk_sets_equivalent(ids_gpu, ids_ref, scores_ref, bound=None, rtol=1e-6):
 
 def score_bound(ref, cond):
     return SCORE_RTOL * np.abs(np.asarray(ref, dtype=np.float64)) + SCORE_CTOL * cond
+
+
+def graph_kernel_count(enqueue):
+    """Kernels one call of `enqueue(stream)` launches: the call is captured
+    into a CUDA graph (after one warm call outside capture) and the graph's
+    kernel nodes are counted."""
+    from cuda.bindings import runtime as rt
+
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        enqueue(s)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph(keep_graph=True)
+    with torch.cuda.graph(g):
+        enqueue(torch.cuda.current_stream())
+    raw = rt.cudaGraph_t(init_value=int(g.raw_cuda_graph()))
+    err, _, n = rt.cudaGraphGetNodes(raw, 0)
+    assert err == rt.cudaError_t.cudaSuccess, err
+    err, nodes, n = rt.cudaGraphGetNodes(raw, n)
+    assert err == rt.cudaError_t.cudaSuccess, err
+    kinds = [rt.cudaGraphNodeGetType(x)[1] for x in nodes[:n]]
+    count = sum(k == rt.cudaGraphNodeType.cudaGraphNodeTypeKernel for k in kinds)
+    torch.cuda.synchronize()
+    del g
+    return count

@@ -9,7 +9,7 @@ import torch
 import lightning_indexer_top_index_b200 as L
 import oracle
 import synth
-from _helpers import assert_attn_close, assert_scores_close, score_bound, topk_sets_equivalent
+from _helpers import assert_attn_close, assert_scores_close, graph_kernel_count, score_bound, topk_sets_equivalent
 from lightning_indexer_top_index_b200.decode import DecodeStep, LayerCache
 
 pytestmark = pytest.mark.gpu
@@ -69,3 +69,10 @@ def test_decode_step_fp8_batched(cuda_device):
                                 swa=x["swa"].slice(b * spec.swa, (b + 1) * spec.swa), swa_len=spec.swa,
                                 scale=spec.scale)
             assert_attn_close(out[l, b], ro)
+
+
+@pytest.mark.parametrize("pdl", [True, False])
+def test_decode_step_kernel_count(cuda_device, pdl):
+    spec = synth.scaled(synth.C2, N=4099, layers=3)
+    _, st = _step(spec, 3, pdl)
+    assert graph_kernel_count(st.enqueue) == st.kernel_launches()

@@ -9,14 +9,13 @@ import torch
 import lightning_indexer_top_index_b200 as L
 import oracle
 import synth
-from _helpers import assert_scores_close, dev_kv, dev_q
+from _helpers import assert_scores_close, dev_kv, dev_q, graph_kernel_count
 from lightning_indexer_top_index_b200.evalwin import EvalWindow
 
 pytestmark = pytest.mark.gpu
 
 
-def test_eval_window_against_oracle(cuda_device):
-    spec = synth.scaled(synth.C5, L=4, T=3, N=1100, k=64, gate_layers=(0, 1, 3))
+def _window(spec):
     layers = [synth.eval_layer(spec, l) for l in range(spec.L)]
     gate = synth.eval_gate(spec)
     keys = [dev_kv(x["keys"], batch_rows=spec.N) for x in layers]
@@ -26,6 +25,18 @@ def test_eval_window_against_oracle(cuda_device):
     qa = torch.stack([dev_q(x["qa"], "bf16") for x in layers])
     win = EvalWindow(keys, kv_all, q_idx, w, qa, dev_q(gate["g"], "bf16"), torch.from_numpy(gate["u"]).cuda(),
                      spec.gate_layers, spec.N, spec.k, (spec.top_p_num, spec.top_p_den), spec.min_votes, spec.scale)
+    return layers, gate, win
+
+
+def test_eval_window_kernel_count(cuda_device):
+    spec = synth.scaled(synth.C5, L=4, T=3, N=1100, k=64, gate_layers=(0, 1, 3))
+    _, _, win = _window(spec)
+    assert graph_kernel_count(win.enqueue) == win.kernel_launches()
+
+
+def test_eval_window_against_oracle(cuda_device):
+    spec = synth.scaled(synth.C5, L=4, T=3, N=1100, k=64, gate_layers=(0, 1, 3))
+    layers, gate, win = _window(spec)
     win.enqueue()
     win.enqueue()  # a second window on the same buffers
     torch.cuda.synchronize()

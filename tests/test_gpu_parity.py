@@ -253,12 +253,34 @@ def test_golden_probs_tensor_core(T, N):
         np.testing.assert_allclose(got[l], ref, rtol=1e-4, atol=1e-10)
 
 
-@pytest.mark.parametrize("N,conc", [(1, 1.0), (100, 0.5), (4097, 2.0), (32768, 1.0), (32768, 6.0)])
+@pytest.mark.parametrize("N,conc", [(1, 1.0), (100, 0.5), (4097, 2.0), (32768, 1.0), (32768, 6.0), (60000, 1.0)])
 def test_topp_bit_exact(N, conc):
     rows = 4
     p = synth.random_probs(41, rows, N, conc)
     W = (N + 31) // 32
     bits = torch.zeros((rows, W), dtype=torch.int32, device="cuda")
+    L.selection_eval(L.EVAL_TOPP, L=rows, T=1, N=N, probs=torch.from_numpy(p).cuda(), topp_bits=bits)
+    got = bits.cpu().numpy().view(np.uint32)
+    for r in range(rows):
+        ref, _ = oracle.topp(p[r])
+        assert np.array_equal(got[r], ref), f"row {r}"
+
+
+@pytest.mark.parametrize("case", ["uniform", "just_below_split", "at_split"])
+def test_topp_unnormalised_rows(case):
+    """Rows whose entries lie in [0, 1] but do not sum to 1: a total mass of
+    2^43 or more takes the 64-bit digit sums, below it the split 32-bit sums."""
+    rng = np.random.default_rng(7)
+    if case == "uniform":
+        p = rng.random((3, 4097), dtype=np.float32)
+    elif case == "just_below_split":
+        p = np.full((2, 10), 0.79, dtype=np.float32)
+        p[1, 3] = 0.5
+    else:
+        p = np.full((2, 16), 0.5, dtype=np.float32)
+        p[1, ::3] = 0.25
+    rows, N = p.shape
+    bits = torch.zeros((rows, (N + 31) // 32), dtype=torch.int32, device="cuda")
     L.selection_eval(L.EVAL_TOPP, L=rows, T=1, N=N, probs=torch.from_numpy(p).cuda(), topp_bits=bits)
     got = bits.cpu().numpy().view(np.uint32)
     for r in range(rows):
