@@ -86,6 +86,7 @@ CALL_SOURCES = {
     "score": ("score_tc.cu", "score_cc.cu"),
     "topk": ("topk.cu",),
     "attn": ("attn.cu", "attn_tc.cu"),
+    "golden": ("golden_tc.cu", "eval.cu"),
 }
 CALL_NAMES = {"score": "lidx_index_score", "topk": "lidx_topk_select", "attn": "lidx_sparse_attn_decode"}
 
@@ -504,7 +505,8 @@ def run_eval(args, cfg, rank, world, local_rank, reference=False):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                         "frac": achieved / peak, "traffic": None, "kernel": "lidx_selection_eval (golden)",
+                         "frac": achieved / peak, "traffic": profiled_traffic("eval-window", "golden"),
+                         "kernel": "lidx_selection_eval (golden)",
                          "peak_source": pk["source"] + " bf16, sustained", "flops_per_launch": gflops,
                          "avg_launch_us": stage_ms["golden"] * 1e3},
             "stages_ms": stage_ms,
