@@ -24,6 +24,7 @@ import json
 import math
 import os
 import statistics
+import tempfile
 import subprocess
 import sys
 import time
@@ -151,7 +152,7 @@ class ClockSampler:
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_{os.getpid()}.csv")
+        self.path = os.path.join(tempfile.gettempdir(), f"lidx_clocks_{os.getpid()}.csv")
 
     def start(self):
         try:

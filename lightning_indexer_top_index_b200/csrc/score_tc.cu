@@ -341,16 +341,43 @@ __global__ void __launch_bounds__(kFp8 ? 32 * kConvWarp0 + 128 : 32 * kConvWarp0
           if (j < p.N) p.scores[static_cast<int64_t>(b * p.Q + g) * p.ld_scores + j] = s;
           if (p.stats) span_stats(s, j < p.N, b * p.Q + g, t);
         } else {
-          for (int qi = 0; qi < p.QG; qi++) {
-            float s = 0.f;
-            for (int c0 = 0; c0 < p.H; c0 += 32) {
-              tc::tmem_ld32(base + qi * p.H + c0, v);
+          // The QG x H accumulator columns in chunks of 32, two register
+          // buffers deep: chunk c+1 loads from TMEM while chunk c is reduced.
+          // A query's score is complete after its last chunk.
+          const int nch = (p.QG * p.H) >> 5;
+          uint32_t ra[32], rb[32];
+          float s = 0.f;
+          auto reduce = [&](const uint32_t (&rr)[32], int c) {
+            const float4 *w4 = reinterpret_cast<const float4 *>(gW + 32 * c);
+            float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-              for (int i = 0; i < 32; i++) s = fmaf(gW[qi * p.H + c0 + i], fmaxf(v[i], 0.f), s);
+            for (int i = 0; i < 8; i++) {
+              const float4 wv = w4[i];
+              s4[0] = fmaf(wv.x, fmaxf(__uint_as_float(rr[4 * i + 0]), 0.f), s4[0]);
+              s4[1] = fmaf(wv.y, fmaxf(__uint_as_float(rr[4 * i + 1]), 0.f), s4[1]);
+              s4[2] = fmaf(wv.z, fmaxf(__uint_as_float(rr[4 * i + 2]), 0.f), s4[2]);
+              s4[3] = fmaf(wv.w, fmaxf(__uint_as_float(rr[4 * i + 3]), 0.f), s4[3]);
             }
-            const int qq = g * p.QG + qi;
-            if (j < p.N && qq < p.Q) p.scores[static_cast<int64_t>(b * p.Q + qq) * p.ld_scores + j] = s;
-            if (p.stats && qq < p.Q) span_stats(s, j < p.N, b * p.Q + qq, t);
+            s += (s4[0] + s4[1]) + (s4[2] + s4[3]);
+            if (((c + 1) << 5) % p.H == 0) {  // last chunk of query qi
+              const int qq = g * p.QG + ((c << 5) / p.H);
+              if (j < p.N && qq < p.Q) p.scores[static_cast<int64_t>(b * p.Q + qq) * p.ld_scores + j] = s;
+              if (p.stats && qq < p.Q) span_stats(s, j < p.N, b * p.Q + qq, t);
+              s = 0.f;
+            }
+          };
+          tc::tmem_ld32_issue(base, ra);
+          for (int c = 0; c < nch; c += 2) {
+            tc::tmem_ld_wait();
+            tc::tmem_ld32_pin(ra);
+            if (c + 1 < nch) tc::tmem_ld32_issue(base + 32 * (c + 1), rb);
+            reduce(ra, c);
+            if (c + 1 < nch) {
+              tc::tmem_ld_wait();
+              tc::tmem_ld32_pin(rb);
+              if (c + 2 < nch) tc::tmem_ld32_issue(base + 32 * (c + 2), ra);
+              reduce(rb, c + 1);
+            }
           }
         }
       }
