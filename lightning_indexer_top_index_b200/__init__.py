@@ -51,6 +51,25 @@ def csa_stack_index(model_layer: int) -> int:
 
 
 GATE_LAYERS = tuple(csa_stack_index(l) for l in GATE_MODEL_LAYERS)
+MODEL_LAYERS = 43
+SWA_ROWS = 128
+
+
+def logical_kv_bytes(tokens: int, elem_bytes: int = 4) -> dict:
+    """Logical KV-cache size of the 43-layer stack at a context of `tokens`
+    (architecture post, section (A)), `elem_bytes` per element:
+
+      CSA  per layer tokens/4 entries, each a 512-wide attention row and a
+           128-d index key
+      HCA  per layer tokens/128 entries of a 512-wide row (no index keys)
+      SWA  a 128-row window of 512-wide rows in every layer
+
+    The post's ~871 MiB at 64K comes out with 4-byte elements, the logical
+    (host-side) cache it names; the stored FP8 rows are smaller."""
+    csa = len(CSA_LAYERS) * (tokens // 4) * (512 + 128) * elem_bytes
+    hca = len(HCA_LAYERS) * (tokens // 128) * 512 * elem_bytes
+    swa = MODEL_LAYERS * min(SWA_ROWS, tokens) * 512 * elem_bytes
+    return {"csa": csa, "hca": hca, "swa": swa, "total": csa + hca + swa}
 
 
 class LidxError(RuntimeError):

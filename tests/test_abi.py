@@ -123,6 +123,23 @@ def test_schedule_constants():
     assert len(L.CSA_LAYERS) + len(L.HCA_LAYERS) + len(facts["swa_layers"]["value"]) == facts["model_layers"]["value"]
 
 
+def test_logical_kv_size_at_64k():
+    """The architecture post's ~871 MiB of KV at 64K: 21 CSA layers of 16384
+    entries x (512 + 128) fp32, 20 HCA layers of 512 entries x 512, and a
+    128-row window of 512 in each of the 43 layers."""
+    import json
+    facts = json.load(open(os.path.join(ROOT, "tests", "golden", "page_facts.json")))
+    kv = L.logical_kv_bytes(65536)
+    mib = 1 << 20
+    assert kv["csa"] == 840 * mib
+    assert kv["hca"] == 20 * mib
+    assert kv["swa"] == 10.75 * mib
+    assert abs(kv["total"] / mib - facts["kv_logical_mib_at_64k"]["value"]) < 0.5
+    # entries per layer at 64K as the post gives them
+    assert kv["csa"] // (len(L.CSA_LAYERS) * 640 * 4) == facts["csa_entries_at_64k"]["value"]
+    assert kv["hca"] // (len(L.HCA_LAYERS) * 512 * 4) == facts["hca_entries_at_64k"]["value"]
+
+
 def test_oracle_and_product_share_nothing():
     """The oracle and the CUDA path import / include nothing of each other."""
     pkg = os.path.join(ROOT, "lightning_indexer_top_index_b200")
