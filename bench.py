@@ -40,9 +40,9 @@ METRIC = "CSA decode steps/s (score+top-k+sparse attn) at 64K; HBM GB/s vs peak"
 UNIT = "steps/s"
 
 WORKLOADS = {
-    "decode-64k": synth.C2,
-    "decode-128k-b32": synth.C3,
-    "decode-500k-b4": synth.C4,
+    "decode-64k": synth.DECODE_64K,
+    "decode-128k-b32": synth.DECODE_128K_B32,
+    "decode-500k-b4": synth.DECODE_500K_FP8,
 }
 
 KEY_ROW_BYTES = {"f32": 512, "bf16": 256, "e4m3": 64 + 1 + 128}
@@ -411,7 +411,7 @@ def oracle_eval_sample(spec, layers, gate):
 
 
 def run_eval(args, cfg, rank, world, local_rank, reference=False):
-    spec = synth.C5
+    spec = synth.EVAL_WINDOW
     if reference:
         layers, gate = eval_inputs(synth.scaled(spec, L=1))
         for _ in range(args.warmup):
@@ -541,7 +541,7 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.workload == "eval-window":
-        e = synth.C5
+        e = synth.EVAL_WINDOW
         cfg = {"workload": e.name, "layers": e.L, "queries": e.T, "heads": e.H, "entries": e.N, "top_k": e.k,
                "top_p": f"{e.top_p_num}/{e.top_p_den}", "min_votes": e.min_votes,
                "gate_layers": list(e.gate_layers), "l2": "inputs larger than L2 (704 MB of attention rows)",

@@ -12,8 +12,8 @@
  *        s[b,t,j] = sum_h w[b,t,h] * max(q[b,t,h,:] . k[b,j,:], 0)
  *        (lightning indexer: DeepSeek-V4-Flash architecture post, section
  *        (B); "native ReLU-MQA" and the head-fused gate form in the
- *        FlashMemory-DeepSeek-V4 write-up, reply #2; the rule itself is
- *        fixed by the build's specification because the pages leave it open)
+ *        FlashMemory-DeepSeek-V4 write-up, reply #2; the pages name the rule
+ *        but print no formula, and this is its plainest reading)
  *  - orc_topk          the k largest scores, ties to the lower index
  *        (n_indexer_top_k = 512 / 1024: architecture post, section (B))
  *  - orc_attn          softmax attention of one decode query over the

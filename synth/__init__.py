@@ -199,13 +199,14 @@ class DecodeSpec:
         return 1.0 / math.sqrt(self.D_attn)
 
 
-# The five workloads of the benchmark definition, in its order.
-C1 = DecodeSpec("tiny-1k-f32", seed=0, B=1, N=1024, H=16, k=64, key_dtype="f32",
-                q_dtype="f32", kv_dtype="f32")
-C2 = DecodeSpec("decode-64k-b1-x21", seed=1, B=1, N=16384, H=64, k=512, layers=21)
-C3 = DecodeSpec("decode-128k-b32-planted", seed=2, B=32, N=32768, H=64, k=512, plant=True)
-C4 = DecodeSpec("decode-500k-b4-pro-fp8", seed=3, B=4, N=125000, H=64, k=1024,
-                key_dtype="e4m3", kv_dtype="e4m3")
+# The workloads: a tiny fp32 parity case, one 64K decode token over 21 CSA
+# layers, a planted 128K batch of 32, and the 500K Pro batch of 4 in FP8.
+TINY_1K_F32 = DecodeSpec("tiny-1k-f32", seed=0, B=1, N=1024, H=16, k=64, key_dtype="f32",
+                         q_dtype="f32", kv_dtype="f32")
+DECODE_64K = DecodeSpec("decode-64k-b1-x21", seed=1, B=1, N=16384, H=64, k=512, layers=21)
+DECODE_128K_B32 = DecodeSpec("decode-128k-b32-planted", seed=2, B=32, N=32768, H=64, k=512, plant=True)
+DECODE_500K_FP8 = DecodeSpec("decode-500k-b4-pro-fp8", seed=3, B=4, N=125000, H=64, k=1024,
+                             key_dtype="e4m3", kv_dtype="e4m3")
 
 
 @dataclasses.dataclass
@@ -233,7 +234,7 @@ class EvalSpec:
         return 1.0 / math.sqrt(self.D_attn)
 
 
-C5 = EvalSpec()
+EVAL_WINDOW = EvalSpec()
 
 
 def scaled(spec, **kw):

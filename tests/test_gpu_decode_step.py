@@ -42,7 +42,7 @@ def _step(spec, layers, pdl):
 
 @pytest.mark.parametrize("pdl", [True, False])
 def test_decode_step_against_oracle(cuda_device, pdl):
-    spec = synth.scaled(synth.C2, N=4099, layers=3)
+    spec = synth.scaled(synth.DECODE_64K, N=4099, layers=3)
     inp, st = _step(spec, 3, pdl)
     scores, ids, n_sel = st.scores.cpu().numpy(), st.ids.cpu().numpy(), st.n_sel.cpu().numpy()
     out = st.out.cpu().numpy()
@@ -59,7 +59,7 @@ def test_decode_step_against_oracle(cuda_device, pdl):
 
 
 def test_decode_step_fp8_batched(cuda_device):
-    spec = synth.scaled(synth.C4, N=5000, B=2, layers=2)
+    spec = synth.scaled(synth.DECODE_500K_FP8, N=5000, B=2, layers=2)
     inp, st = _step(spec, 2, True)
     ids, out = st.ids.cpu().numpy(), st.out.cpu().numpy()
     for l, x in enumerate(inp):
@@ -73,6 +73,6 @@ def test_decode_step_fp8_batched(cuda_device):
 
 @pytest.mark.parametrize("pdl", [True, False])
 def test_decode_step_kernel_count(cuda_device, pdl):
-    spec = synth.scaled(synth.C2, N=4099, layers=3)
+    spec = synth.scaled(synth.DECODE_64K, N=4099, layers=3)
     _, st = _step(spec, 3, pdl)
     assert graph_kernel_count(st.enqueue) == st.kernel_launches()

@@ -29,13 +29,13 @@ def _window(spec):
 
 
 def test_eval_window_kernel_count(cuda_device):
-    spec = synth.scaled(synth.C5, L=4, T=3, N=1100, k=64, gate_layers=(0, 1, 3))
+    spec = synth.scaled(synth.EVAL_WINDOW, L=4, T=3, N=1100, k=64, gate_layers=(0, 1, 3))
     _, _, win = _window(spec)
     assert graph_kernel_count(win.enqueue) == win.kernel_launches()
 
 
 def test_eval_window_against_oracle(cuda_device):
-    spec = synth.scaled(synth.C5, L=4, T=3, N=1100, k=64, gate_layers=(0, 1, 3))
+    spec = synth.scaled(synth.EVAL_WINDOW, L=4, T=3, N=1100, k=64, gate_layers=(0, 1, 3))
     layers, gate, win = _window(spec)
     win.enqueue()
     win.enqueue()  # a second window on the same buffers

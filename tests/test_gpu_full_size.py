@@ -50,7 +50,7 @@ def _check_layer(spec, x, scores, ids, n_sel, out, b, ranges=None):
 
 def test_decode_64k_full_step(cuda_device):
     """21 layers x 16384 entries, bf16: three layers checked whole."""
-    spec = synth.C2
+    spec = synth.DECODE_64K
     layers, st = _bench_step(spec)
     scores, ids, n_sel, out = (t.cpu().numpy() for t in (st.scores, st.ids, st.n_sel, st.out))
     for l in (0, 10, 20):
@@ -61,7 +61,7 @@ def test_decode_500k_fp8_full_step(cuda_device):
     """B=4 x 125000 entries, E4M3 keys and rows, top-1024: every sequence's
     top-k and attention; scores on the first and the last 2048 entries (the
     ragged tail tile)."""
-    spec = synth.C4
+    spec = synth.DECODE_500K_FP8
     layers, st = _bench_step(spec)
     scores, ids, n_sel, out = (t.cpu().numpy() for t in (st.scores, st.ids, st.n_sel, st.out))
     N = spec.N
@@ -73,7 +73,7 @@ def test_decode_500k_fp8_full_step(cuda_device):
 def test_decode_128k_b32_planted_full_step(cuda_device):
     """B=32 x 32768 entries: every sequence's top-512 is its planted set;
     two sequences checked whole."""
-    spec = synth.C3
+    spec = synth.DECODE_128K_B32
     layers, st = _bench_step(spec)
     scores, ids, n_sel, out = (t.cpu().numpy() for t in (st.scores, st.ids, st.n_sel, st.out))
     x = layers[0]
@@ -92,7 +92,7 @@ def test_eval_window_full_size(cuda_device):
     import lightning_indexer_top_index_b200 as L
     from lightning_indexer_top_index_b200.evalwin import EvalWindow
 
-    spec = synth.C5
+    spec = synth.EVAL_WINDOW
     layers, gate = bench.eval_inputs(spec)
 
     def bf(a):

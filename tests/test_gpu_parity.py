@@ -35,12 +35,12 @@ def _score_case(spec, layer=0):
 
 
 @pytest.mark.parametrize("spec", [
-    synth.C1,
-    synth.scaled(synth.C2, N=1000),
-    synth.scaled(synth.C2, N=16384),
-    synth.scaled(synth.C2, N=4099, B=3, H=32),
-    synth.scaled(synth.C4, N=3001, B=2),
-    synth.scaled(synth.C3, N=2500, B=2, k=64),
+    synth.TINY_1K_F32,
+    synth.scaled(synth.DECODE_64K, N=1000),
+    synth.scaled(synth.DECODE_64K, N=16384),
+    synth.scaled(synth.DECODE_64K, N=4099, B=3, H=32),
+    synth.scaled(synth.DECODE_500K_FP8, N=3001, B=2),
+    synth.scaled(synth.DECODE_128K_B32, N=2500, B=2, k=64),
 ], ids=lambda s: f"{s.name}-N{s.N}-B{s.B}-H{s.H}")
 def test_score_parity(spec):
     _, got, ref, cond = _score_case(spec)
@@ -50,7 +50,7 @@ def test_score_parity(spec):
 @pytest.mark.parametrize("T,N,H", [(64, 700, 64), (5, 1029, 64), (3, 300, 16)])
 def test_score_batched_queries(T, N, H):
     """Prefill-style: many queries of one layer scored against the same keys."""
-    spec = synth.scaled(synth.C5, T=T, N=N, H=H, L=2)
+    spec = synth.scaled(synth.EVAL_WINDOW, T=T, N=N, H=H, L=2)
     B = 2
     qs, ws, ks = [], [], []
     for l in range(B):
@@ -68,7 +68,7 @@ def test_score_batched_queries(T, N, H):
 
 def test_score_signed_weights_and_ld():
     """Signed head weights (gate use) and a padded score row stride."""
-    spec = synth.scaled(synth.C2, N=777)
+    spec = synth.scaled(synth.DECODE_64K, N=777)
     inp = synth.decode_layer(spec)
     w = (np.random.default_rng(3).random((1, 64)) * 2 - 1).astype(np.float32)
     scores = torch.full((1, 1, 800), 7.0, device="cuda")
@@ -82,7 +82,7 @@ def test_score_signed_weights_and_ld():
 
 
 def test_score_f16_refused():
-    spec = synth.scaled(synth.C2, N=64)
+    spec = synth.scaled(synth.DECODE_64K, N=64)
     inp = synth.decode_layer(spec)
     keys = dev_kv(inp["keys"])
     keys.dtype = L.F16
@@ -168,28 +168,28 @@ def _attn_case(spec, n_sel=None, swa_len=None, ids=None, layer=0):
 
 
 @pytest.mark.parametrize("spec", [
-    synth.C1,
-    synth.scaled(synth.C2, N=3000),
-    synth.scaled(synth.C4, N=5000, B=2),
-    synth.scaled(synth.C3, N=4000, B=3, plant=False),
+    synth.TINY_1K_F32,
+    synth.scaled(synth.DECODE_64K, N=3000),
+    synth.scaled(synth.DECODE_500K_FP8, N=5000, B=2),
+    synth.scaled(synth.DECODE_128K_B32, N=4000, B=3, plant=False),
 ], ids=lambda s: s.name)
 def test_attn_parity(spec):
     _attn_case(spec)
 
 
 def test_attn_partial_selection_and_short_window():
-    spec = synth.scaled(synth.C2, N=2000, B=3, k=512)
+    spec = synth.scaled(synth.DECODE_64K, N=2000, B=3, k=512)
     _attn_case(spec, n_sel=[512, 100, 0], swa_len=37)
 
 
 def test_attn_no_window_and_empty():
-    spec = synth.scaled(synth.C2, N=900, B=2, k=64)
+    spec = synth.scaled(synth.DECODE_64K, N=900, B=2, k=64)
     _attn_case(spec, swa_len=0)
     _attn_case(spec, n_sel=[0, 3], swa_len=0)
 
 
 def test_attn_out_of_range_id_flags_bounds():
-    spec = synth.scaled(synth.C2, N=500, B=1, k=8)
+    spec = synth.scaled(synth.DECODE_64K, N=500, B=1, k=8)
     inp = synth.decode_layer(spec)
     ids = np.array([[1, 5, 499, 500, 7, -1, 1000, 2]], dtype=np.int32)
     kv, swa = dev_kv(inp["kv"]), dev_kv(inp["swa"])
@@ -206,8 +206,9 @@ def test_attn_out_of_range_id_flags_bounds():
 
 # ------------------------------------------------------------- end to end
 def test_chain_tiny_config():
-    """C1 end to end: score -> top-64 -> attention, against the oracle chain."""
-    spec = synth.C1
+    """The tiny fp32 case end to end: score -> top-64 -> attention, against the
+    oracle chain."""
+    spec = synth.TINY_1K_F32
     inp, got, ref, cond = _score_case(spec)
     scores = torch.from_numpy(got).cuda()
     ids, n_sel, _, _ = L.topk_select(scores, spec.k)
@@ -223,7 +224,7 @@ def test_chain_tiny_config():
 
 # ------------------------------------------------------------------- eval
 def test_golden_probs_parity():
-    spec = synth.scaled(synth.C5, L=2, T=3, H=8, N=1100)
+    spec = synth.scaled(synth.EVAL_WINDOW, L=2, T=3, H=8, N=1100)
     qa = np.stack([synth.eval_layer(spec, l)["qa"][:, :spec.H] for l in range(spec.L)])
     kvs = [synth.eval_layer(spec, l)["kv"] for l in range(spec.L)]
     kv = synth.concat_kv(kvs)
@@ -240,7 +241,7 @@ def test_golden_probs_parity():
 def test_golden_probs_tensor_core(T, N):
     """64 heads, bf16: the tcgen05 path (two queries per 128-row tile, 256-key
     blocks); odd T leaves padding rows in the last tile, N a partial block."""
-    spec = synth.scaled(synth.C5, L=2, T=T, H=64, N=N)
+    spec = synth.scaled(synth.EVAL_WINDOW, L=2, T=T, H=64, N=N)
     qa = np.stack([synth.eval_layer(spec, l)["qa"] for l in range(spec.L)])
     kvs = [synth.eval_layer(spec, l)["kv"] for l in range(spec.L)]
     kv = synth.concat_kv(kvs)

@@ -105,11 +105,11 @@ def test_topk_wrong_bounds_stay_in_bounds():
 
 
 @pytest.mark.parametrize("spec", [
-    synth.C1,
-    synth.scaled(synth.C2, N=5000),
-    synth.scaled(synth.C2, N=16384),
-    synth.scaled(synth.C2, N=3001, B=3, H=32),
-    synth.scaled(synth.C4, N=3001, B=2),
+    synth.TINY_1K_F32,
+    synth.scaled(synth.DECODE_64K, N=5000),
+    synth.scaled(synth.DECODE_64K, N=16384),
+    synth.scaled(synth.DECODE_64K, N=3001, B=3, H=32),
+    synth.scaled(synth.DECODE_500K_FP8, N=3001, B=2),
 ], ids=lambda s: f"{s.name}-N{s.N}-B{s.B}-H{s.H}")
 def test_scorer_bounds_then_topk(spec):
     """The scorer's bounds describe exactly its own scores; the top-k that
@@ -130,7 +130,7 @@ def test_scorer_bounds_then_topk(spec):
 
 def test_scorer_bounds_batched_queries():
     """Several queries per key tile."""
-    spec = synth.scaled(synth.C5, T=7, N=3000, H=64, L=1)
+    spec = synth.scaled(synth.EVAL_WINDOW, T=7, N=3000, H=64, L=1)
     inp = synth.eval_layer(spec, 0)
     T, H, N = spec.T, spec.H, spec.N
     keys = dev_kv(inp["keys"], batch_rows=N)

@@ -170,7 +170,7 @@ def test_score_batch_and_query_indexing():
 def test_planted_rows_are_the_topk():
     """The +3 sigma planted rows of the 128K batched workload dominate the noise
     (planted scores ~8 vs noise ~1.1 +- 0.24), so the top-k is the planted set."""
-    spec = synth.scaled(synth.C3, B=2, N=2048, k=64)
+    spec = synth.scaled(synth.DECODE_128K_B32, B=2, N=2048, k=64)
     inp = synth.decode_layer(spec)
     for b in range(spec.B):
         s = oracle.index_score(inp["q_idx"][b][None], inp["w"][b][None],
@@ -248,7 +248,7 @@ def test_attn_equal_logits_is_the_mean():
 def test_attn_matches_library_softmax():
     """Small case against scipy's softmax and numpy matmul on decoded rows."""
     g = np.random.default_rng(8)
-    spec = synth.scaled(synth.C2, N=300, H=8, swa=16)
+    spec = synth.scaled(synth.DECODE_64K, N=300, H=8, swa=16)
     inp = synth.decode_layer(spec)
     ids = np.sort(g.choice(300, 40, replace=False)).astype(np.int32)
     out, lse = oracle.attn(inp["q_attn"][0], inp["kv"], 300, ids, swa=inp["swa"], swa_len=16,
@@ -289,7 +289,7 @@ def test_attn_empty_and_padding():
 
 # ---------------------------------------------------------------------- golden
 def test_golden_rows_sum_to_one_and_single_head():
-    spec = synth.scaled(synth.C5, N=200, T=3, H=4)
+    spec = synth.scaled(synth.EVAL_WINDOW, N=200, T=3, H=4)
     inp = synth.eval_layer(spec, 0)
     p = oracle.golden(inp["qa"], inp["kv"], spec.T, spec.H, spec.N, spec.scale)
     np.testing.assert_allclose(p.sum(axis=1), 1.0, rtol=2e-6)
@@ -302,7 +302,7 @@ def test_golden_rows_sum_to_one_and_single_head():
 def test_golden_agrees_with_attention_lse():
     """p_h(j) = exp(logit_hj - lse_h): the golden probabilities and the
     attention log-sum-exp over all entries describe the same softmax."""
-    spec = synth.scaled(synth.C5, N=150, T=1, H=1)
+    spec = synth.scaled(synth.EVAL_WINDOW, N=150, T=1, H=1)
     inp = synth.eval_layer(spec, 1)
     p = oracle.golden(inp["qa"], inp["kv"], 1, 1, spec.N, spec.scale)[0]
     _, lse = oracle.attn(inp["qa"][0], inp["kv"], spec.N, np.arange(spec.N, dtype=np.int32),

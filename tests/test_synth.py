@@ -7,7 +7,7 @@ import synth
 
 
 def test_deterministic_and_slice_independent():
-    spec = synth.scaled(synth.C2, N=256, layers=2)
+    spec = synth.scaled(synth.DECODE_64K, N=256, layers=2)
     a = synth.decode_layer(spec, 1)
     b = synth.decode_layer(spec, 1)
     for key in ("q_idx", "w", "q_attn"):

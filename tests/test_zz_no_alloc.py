@@ -37,7 +37,7 @@ def test_noalloc_matches_workspace_entry_point(cuda_device):
     fn = lib.lidx_sparse_attn_decode_noalloc
     fn.restype = C.c_int
     fn.argtypes = [C.POINTER(L.AttnArgs), C.c_void_p, C.c_void_p]
-    spec = synth.scaled(synth.C2, N=3000, B=2, k=256)
+    spec = synth.scaled(synth.DECODE_64K, N=3000, B=2, k=256)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     for call, (layer, seed) in enumerate([(0, 5), (1, 6)]):
         q, kv, swa, ids = _case(spec, layer, seed)
@@ -59,7 +59,7 @@ def test_noalloc_matches_workspace_entry_point(cuda_device):
 def test_noalloc_rejects_oversized_requests(cuda_device):
     """A request whose split-K scratch exceeds the fixed array is refused
     before anything is enqueued."""
-    spec = synth.scaled(synth.C2, N=600, B=1, k=512)
+    spec = synth.scaled(synth.DECODE_64K, N=600, B=1, k=512)
     q, kv, swa, ids = _case(spec, 0, 7)
     big_b = 64  # 64 sequences x 20 splits x 64 heads x 514 floats > 16 MiB
     qb = q.expand(big_b, -1, -1).contiguous()
