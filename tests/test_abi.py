@@ -34,6 +34,25 @@ def test_exports_every_declared_symbol(lib):
     assert lib.lidx_abi_version() == int(re.search(r"#define LIDX_ABI_VERSION (\d+)", hdr).group(1))
 
 
+@pytest.mark.parametrize("compiler,flags", [("gcc", ["-x", "c", "-std=c11", "-pedantic"]),
+                                            ("g++", ["-x", "c++", "-std=c++17"])])
+def test_plain_c_consumer(lib, tmp_path, compiler, flags):
+    """include/lidx.h compiles as strict C11 and as C++ without CUDA or torch
+    headers, links against liblidx.so, and agrees with the library's struct
+    layouts and host-only calls."""
+    import shutil
+    import subprocess
+    if shutil.which(compiler) is None:
+        pytest.skip(f"no {compiler}")
+    pkg = os.path.dirname(L.__file__)
+    exe = str(tmp_path / "consumer")
+    subprocess.run([compiler, *flags, "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "abi_consumer.c"), "-x", "none", "-L", pkg, "-llidx",
+                    f"-Wl,-rpath,{pkg}", "-o", exe], check=True, capture_output=True, text=True)
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0 and r.stdout.strip() == "OK", r.stdout + r.stderr
+
+
 def test_struct_sizes_match(lib):
     for i, s in enumerate(L._STRUCTS):
         assert lib.lidx_struct_size(i) == C.sizeof(s)
