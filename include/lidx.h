@@ -257,7 +257,9 @@ LIDX_API lidx_status lidx_sparse_attn_decode_noalloc(const lidx_attn_args *args,
  *     per row (l,t): with m_j = floor(probs_j * 2^40) and M = sum m_j, the
  *     shortest prefix of the ranking (probs descending, ties to the lower
  *     index) whose mass reaches ceil(M * top_p_num / top_p_den)
- *     -> topp_bits[l][t][W].
+ *     -> topp_bits[l][t][W].  Rows need not sum to 1; a value outside
+ *     [0, 1] or NaN carries no mass and sets LIDX_DEV_NAN.  N above 2^23
+ *     (where the masses could overflow 64 bits) is LIDX_ERR_UNSUPPORTED.
  *  LIDX_EVAL_VOTE    (write-up 3.2 step 3)
  *     vote_bits[t] = { j : #{l : j in topp_bits[l][t]} >= min_votes },
  *     window_bits = union over t of vote_bits[t].
