@@ -53,6 +53,17 @@ def test_plain_c_consumer(lib, tmp_path, compiler, flags):
     assert r.returncode == 0 and r.stdout.strip() == "OK", r.stdout + r.stderr
 
 
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    """Without liblidx.so every call raises: there is no fallback path."""
+    import torch
+    monkeypatch.setattr(L, "LIB_PATH", str(tmp_path / "liblidx.so"))
+    monkeypatch.setattr(L, "_lib", None)
+    with pytest.raises(ImportError):
+        L.lib()
+    with pytest.raises(ImportError):
+        L.topk_select(torch.zeros(1, 1, 8), 2)
+
+
 def test_struct_sizes_match(lib):
     for i, s in enumerate(L._STRUCTS):
         assert lib.lidx_struct_size(i) == C.sizeof(s)
