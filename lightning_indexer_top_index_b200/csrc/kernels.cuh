@@ -14,6 +14,10 @@ struct WsHeader {
   uint32_t pad[63];
 };
 
+// LIDX_OK when the current device is an sm_100 part, else UNSUPPORTED (or
+// CUDA when the device cannot be queried); leaves no pending CUDA error.
+lidx_status check_device_sm100();
+
 // ---- index score
 cudaError_t launch_score_cc(const lidx_score_args &a, cudaStream_t st);
 // tcgen05 scorer; returns cudaErrorNotSupported when the shape is not covered.

@@ -14,12 +14,18 @@ std::mutex g_dev_mu;
 
 lidx_status check_device() {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return LIDX_ERR_CUDA;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return LIDX_ERR_CUDA;
+  }
   if (dev < 0 || dev >= kMaxDevices) return LIDX_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lk(g_dev_mu);
   if (g_dev_ok[dev] == 0) {
     int major = 0;
-    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return LIDX_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return LIDX_ERR_CUDA;
+    }
     g_dev_ok[dev] = major == 10 ? 1 : 2;
   }
   return g_dev_ok[dev] == 1 ? LIDX_OK : LIDX_ERR_UNSUPPORTED;
@@ -128,6 +134,10 @@ lidx_status check_ws(void *ws, size_t have, size_t need) {
 }
 
 }  // namespace
+
+namespace lidx {
+lidx_status check_device_sm100() { return check_device(); }
+}  // namespace lidx
 
 extern "C" {
 

@@ -58,7 +58,7 @@ def _load():
                 "orc_decode_e4m3": (C.c_double, [C.c_uint8]),
                 "orc_decode_e8m0": (C.c_double, [C.c_uint8]),
                 "orc_decode_rows": (I, [RP, I64, P]),
-                "orc_index_score": (I, [I, I, I, I, RP, P, RP, I64, P, I64, P]),
+                "orc_index_score": (I, [I, I, I, I, RP, P, RP, I64, P, I64, P, P]),
                 "orc_topk": (I, [I, I, P, P, P, P, P]),
                 "orc_attn": (I, [I, RP, RP, I, P, I, RP, I, D, P, P]),
                 "orc_golden": (I, [I, I, I, RP, RP, D, P]),
@@ -132,8 +132,11 @@ def decode_rows(kv) -> np.ndarray:
 
 
 # ----------------------------------------------------------------- the path
-def index_score(q, w, keys, B, Q, H, N, key_batch_rows=None, want_cond=False):
-    """scores float32 [B][Q][N] (and cond float64 [B][Q][N] if requested).
+def index_score(q, w, keys, B, Q, H, N, key_batch_rows=None, want_cond=False, want_mag=False):
+    """scores float32 [B][Q][N], plus, if requested, float64 [B][Q][N] arrays:
+    cond = sum_h |w_h| |q_h . k_j| (the absolute floor of the score tolerance)
+    and mag = sum_h |w_h| sum_d |q_hd k_jd| (what a rounding-error bound of
+    the sums scales with).  Returns s, (s, cond), (s, mag) or (s, cond, mag).
 
     q: [B][Q][H][D] (float32 or bf16 bits) or [B][H][D] when Q == 1;
     w: float32 [B][Q][H] / [B][H]; keys: KV with rows b*key_batch_rows + j."""
@@ -142,10 +145,12 @@ def index_score(q, w, keys, B, Q, H, N, key_batch_rows=None, want_cond=False):
     w = np.ascontiguousarray(np.asarray(w, dtype=np.float32).reshape(B, Q, H))
     s = np.empty((B, Q, N), dtype=np.float32)
     cond = np.empty((B, Q, N), dtype=np.float64) if want_cond else None
+    mag = np.empty((B, Q, N), dtype=np.float64) if want_mag else None
     kbr = N if key_batch_rows is None else key_batch_rows
     _check(_load().orc_index_score(B, Q, H, N, C.byref(qr), _ptr(w), C.byref(kr), kbr,
-                                   _ptr(s), N, _ptr(cond)))
-    return (s, cond) if want_cond else s
+                                   _ptr(s), N, _ptr(mag), _ptr(cond)))
+    out = (s,) + ((cond,) if want_cond else ()) + ((mag,) if want_mag else ())
+    return out if len(out) > 1 else s
 
 
 def topk(scores, k, allowed=None):

@@ -140,10 +140,14 @@ int orc_decode_rows(const orc_rows *r, int64_t n, double *out)
  * scores: float [B][Q][N] (row stride ld_s)
  * cond (optional): double [B][Q][N], sum_h |w_h| * sum_d |q_hd k_jd| -- the
  *   magnitude a rounding-error bound of the score scales with.
+ * cond_dot (optional): double [B][Q][N], sum_h |w_h| * |q_h . k_j| -- the
+ *   absolute floor of the score tolerance (the scores must agree to 1e-5
+ *   relative; this term only keeps that bar finite where the head terms
+ *   cancel to near zero).
  */
 int orc_index_score(int B, int Q, int H, int N, const orc_rows *q, const float *w,
                     const orc_rows *keys, int64_t key_batch_rows, float *scores,
-                    int64_t ld_s, double *cond)
+                    int64_t ld_s, double *cond, double *cond_dot)
 {
     int D = keys->dim;
     if (q->dim != D || B < 0 || Q < 0 || H < 1 || N < 0) return ORC_EINVAL;
@@ -156,7 +160,7 @@ int orc_index_score(int B, int Q, int H, int N, const orc_rows *q, const float *
             const float *wt = w + ((int64_t)b * Q + t) * H;
             for (int j = 0; j < N; j++) {
                 decode_row(keys, (int64_t)b * key_batch_rows + j, kv);
-                double s = 0.0, c = 0.0;
+                double s = 0.0, c = 0.0, cd = 0.0;
                 for (int h = 0; h < H; h++) {
                     double dot = 0.0, mag = 0.0;
                     for (int d = 0; d < D; d++) {
@@ -166,9 +170,11 @@ int orc_index_score(int B, int Q, int H, int N, const orc_rows *q, const float *
                     double relu = dot > 0.0 ? dot : 0.0;
                     s += (double)wt[h] * relu;
                     c += fabs((double)wt[h]) * mag;
+                    cd += fabs((double)wt[h]) * fabs(dot);
                 }
                 scores[((int64_t)b * Q + t) * ld_s + j] = (float)s;
                 if (cond) cond[((int64_t)b * Q + t) * N + j] = c;
+                if (cond_dot) cond_dot[((int64_t)b * Q + t) * N + j] = cd;
             }
         }
     free(qv);

@@ -1,8 +1,10 @@
 """Shared helpers of the GPU parity tests: move synthetic inputs to the device
 and apply the parity rules.
 
-Tolerances (derived in the design doc from fp32 accumulation):
-  scores     |g - o| <= 1e-5 |o| + 1e-6 * sum_h |w_h| sum_d |q_hd k_jd|
+Tolerances (fp32 accumulation of exact bf16 / E4M3 products):
+  scores     |g - o| <= 1e-5 |o| + 1e-6 * sum_h |w_h| |q_h . k_j|
+             (1e-5 relative; the absolute term only keeps the bar finite
+             where the head terms cancel to near zero)
   attention  max_d |g - o| / max_d |o| <= 2e-3 per (b, h)
   sets       bit-exact on identical inputs; end to end, differences only for
              entries tied with the k-th score within 1e-6 relative
@@ -30,7 +32,19 @@ def dev_q(q, dtype):
     return t.cuda().contiguous()
 
 
+def score_rel_err(got, ref):
+    """Largest |g - o| / |o| over the entries with |o| > 1e-3 max |o| (the
+    relative error away from the near-zero scores)."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    big = np.abs(ref) > 1e-3 * np.abs(ref).max()
+    if not big.any():
+        return 0.0
+    return float((np.abs(got - ref)[big] / np.abs(ref)[big]).max())
+
+
 def assert_scores_close(got, ref, cond):
+    """Element-wise score check; returns (and prints) score_rel_err."""
     got = np.asarray(got, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
     err = np.abs(got - ref)
@@ -38,6 +52,9 @@ def assert_scores_close(got, ref, cond):
     bad = err > bound
     assert not bad.any(), (f"{bad.sum()} scores outside tolerance; worst err {err.max():.3e} "
                            f"bound there {bound.ravel()[np.argmax(err)]:.3e}")
+    rel = score_rel_err(got, ref)
+    print(f"score max rel err {rel:.3e} over {ref.size} entries")
+    return rel
 
 
 def assert_attn_close(got, ref):

@@ -143,12 +143,34 @@ def test_score_all_negative_dots_is_zero_and_cond():
     q = -np.abs(g.standard_normal((H, 128)))
     keys = synth.encode_rows(k, "f32")
     w = np.ones(H, dtype=np.float32)
-    s, cond = oracle.index_score(q.astype(np.float32)[None], w[None], keys, 1, 1, H, N, want_cond=True)
+    s, cond, mag = oracle.index_score(q.astype(np.float32)[None], w[None], keys, 1, 1, H, N, want_cond=True,
+                                      want_mag=True)
     assert np.all(s == 0.0)
-    # all products nonnegative -> sum |q k| equals q . k, so cond == score
-    s2, cond2 = oracle.index_score((-q).astype(np.float32)[None], w[None], keys, 1, 1, H, N,
-                                   want_cond=True)
-    np.testing.assert_allclose(cond2[0, 0], s2[0, 0], rtol=1e-6)
+    # every dot is negative: |q_h . k| = sum_d |q_hd k_d| = -(q_h . k), so both
+    # tolerance terms equal the score of -q
+    s2 = oracle.index_score((-q).astype(np.float32)[None], w[None], keys, 1, 1, H, N)
+    np.testing.assert_allclose(cond[0, 0], s2[0, 0], rtol=1e-6)
+    np.testing.assert_allclose(mag[0, 0], s2[0, 0], rtol=1e-6)
+
+
+@pytest.mark.parametrize("ex", HAND["score"])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_score_signed_weight_hand_examples(ex, dtype):
+    """Signed head weights multiply the ReLU of each head's dot product (the
+    weight sits outside the ReLU).  Key k = e_0 and q_h = dot_h e_0 give the
+    dots exactly; the expected scores were worked by hand."""
+    w = np.array(ex["w"], dtype=np.float32)
+    H = len(w)
+    q = np.zeros((H, 128))
+    q[:, 0] = ex["q_dot_k"]
+    k = np.zeros((3, 128))
+    k[:, 0] = 1.0
+    k[1, 0] = 2.0  # entry 1 doubles every dot, and the score with it
+    qs = synth.bf16_bits(q) if dtype == "bf16" else q.astype(np.float32)
+    s, cond = oracle.index_score(qs[None], w[None], synth.encode_rows(k, dtype), 1, 1, H, 3, want_cond=True)
+    assert s[0, 0, 0] == ex["score"] and s[0, 0, 2] == ex["score"]
+    assert s[0, 0, 1] == 2 * ex["score"]
+    assert cond[0, 0, 0] == sum(abs(a) * abs(b) for a, b in zip(ex["w"], ex["q_dot_k"]))
 
 
 def test_score_batch_and_query_indexing():

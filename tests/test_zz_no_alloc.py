@@ -5,7 +5,8 @@ scratch allocator, a serving loop that forbids cudaMalloc after start-up).
 It is called through the C ABI, twice in a row on different inputs (the
 shared scratch array keeps the previous call's contents), and each result is
 checked against lidx_sparse_attn_decode on the same inputs within the
-attention tolerance.  This file is collected last on purpose."""
+attention tolerance.  The second call must leave the device's free memory
+unchanged.  This file is collected last on purpose."""
 import ctypes as C
 
 import numpy as np
@@ -47,8 +48,15 @@ def test_noalloc_matches_workspace_entry_point(cuda_device):
         lse = torch.full_like(ref_lse, float("nan"))
         a = L.attn_args(q, kv, spec.N, ids, None, swa, swa_len, spec.scale, out, lse)
         st = C.c_void_p(torch.cuda.current_stream().cuda_stream)
+        torch.cuda.synchronize()
+        free0, torch0 = torch.cuda.mem_get_info()[0], torch.cuda.memory_allocated()
         assert fn(C.byref(a), C.c_void_p(status.data_ptr()), st) == L.OK
         torch.cuda.synchronize()
+        if call > 0:
+            # the first call has loaded the library's module (and its array);
+            # from then on a call takes no device memory at all
+            assert torch.cuda.mem_get_info()[0] == free0, "the call changed the device's free memory"
+            assert torch.cuda.memory_allocated() == torch0
         r, o = ref.cpu().numpy().astype(np.float64), out.cpu().numpy().astype(np.float64)
         rel = np.abs(o - r).max(axis=-1) / np.abs(r).max(axis=-1)
         assert rel.max() <= ATTN_TOL, f"call {call}: max relative difference {rel.max():.3e}"
