@@ -39,7 +39,7 @@
 extern "C" {
 #endif
 
-#define LIDX_ABI_VERSION 3
+#define LIDX_ABI_VERSION 4
 
 #if defined(__GNUC__)
 #define LIDX_API __attribute__((visibility("default")))
@@ -67,6 +67,10 @@ typedef enum lidx_status {
                               * E8M0 scales, attention queries); everything else is read, and every
                               * global write is made, after the wait.  So with this flag the cache-side
                               * inputs must not be written by kernels that may still be running. */
+
+#define LIDX_LAUNCH_TEST_LOST_ARRIVAL 0x80000000u /* test hook of lidx_decode_layer: one score CTA
+                              * withholds its arrival and the cross-CTA waits give up after about 2 ms;
+                              * the call must then finish and report LIDX_DEV_TIMEOUT */
 
 /* Storage formats. */
 #define LIDX_F32 0
@@ -147,8 +151,13 @@ LIDX_API lidx_status lidx_index_score(const lidx_score_args *args, void *stream)
  * lidx_topk_select -- top-k row ids (architecture post, section (B):
  * n_indexer_top_k, and the comp_allowed row set).
  *
- * For each (b,t): the k largest scores[b,t,0..N) among entries with
- * allowed[b][j] != 0 (all entries when allowed is NULL).  Equal scores
+ * For each (b,t): the k largest scores[b,t,0..N) among the eligible
+ * entries: those with allowed[b][j] != 0 when `allowed` is given, and with
+ * bit j%32 of allowed_bits[b][j/32] set when `allowed_bits` is given (all
+ * entries when neither is).  allowed_bits takes the fetched set of the
+ * memory-indexer gate (lidx_selection_eval, LIDX_EVAL_LSA) as it is: the
+ * native indexer then keeps its top-k inside the fetched set
+ * (FlashMemory-vs-native post, "The setup"; write-up, reply #2).  Equal scores
  * (+0 and -0 included) are ranked by index, lower first; NaN scores are
  * never selected and set LIDX_DEV_NAN.
  *
@@ -173,6 +182,8 @@ typedef struct lidx_topk_args {
     uint32_t *mask_bits;
     uint32_t flags;             /* LIDX_LAUNCH_* */
     const uint32_t *tile_stats; /* optional score bounds, see LIDX_STATS_SPAN */
+    const uint32_t *allowed_bits; /* optional [B][ld_allowed_bits] bit set, shared by the Q queries */
+    int64_t ld_allowed_bits;      /* words between sequences, >= ceil(N/32) */
 } lidx_topk_args;
 
 LIDX_API lidx_status lidx_topk_select(const lidx_topk_args *args, void *ws, size_t ws_bytes, void *stream);
@@ -183,13 +194,17 @@ LIDX_API lidx_status lidx_topk_select(const lidx_topk_args *args, void *ws, size
  * sections (A)-(B)).  K = V = the full 512-wide row.
  *
  *   R_b  = { kv row ids[b][i] : i < n_b, ids[b][i] >= 0 } U { swa rows 0..swa_len-1 }
- *          with n_b = n_sel[b] if n_sel is given, else n_ids
+ *          with n_b = n_sel[b] if n_sel is given, else n_ids.
+ *          ids NULL means ids[b][i] = i: the rows 0..n_b-1 are read whole, with
+ *          no top-k (the HCA layers of the architecture post, section (A):
+ *          128:1 compression, every entry attended); n_ids <= N then.
  *   out[b,h,:] = sum_{r in R_b} softmax_r(scale * q[b,h,:] . x_r) x_r
  *   lse[b,h]   = log sum_{r in R_b} exp(scale * q[b,h,:] . x_r)   (optional)
  *
  *   q     [B][H][512], LIDX_F32 (with F32 rows) or LIDX_BF16
  *   kv    comp_kv rows, dim 512, N entries per sequence
- *   ids   [B][ld_ids] int32 (ascending not required; duplicates count twice)
+ *   ids   [B][ld_ids] int32 (ascending not required; duplicates count twice),
+ *         or NULL for the dense rows 0..n_b-1
  *   swa   sliding-window rows, dim 512, same dtype as kv (swa_len may be 0)
  *   out   [B][H][512] fp32
  * Ids outside [-1, N) are skipped and set LIDX_DEV_BOUNDS.  Empty R gives
@@ -216,6 +231,57 @@ typedef struct lidx_attn_args {
 
 LIDX_API lidx_status lidx_sparse_attn_decode(const lidx_attn_args *args, void *ws, size_t ws_bytes,
                                     void *stream);
+
+/* ------------------------------------------------------------------------
+ * lidx_decode_layer -- one CSA layer of decode in a single launch: index
+ * scores -> top-k -> sparse MQA attention over the selected rows plus the
+ * window (architecture post, section (B): the indexer scores every compressed
+ * entry, keeps the top k, and attention reads those attn_comp_kv rows and the
+ * 128-row window).  Same results as lidx_index_score, lidx_topk_select (on
+ * the scores it computes) and lidx_sparse_attn_decode (on those ids) in
+ * sequence, with Q = 1 query per sequence.
+ *
+ *   q_idx [B][H][128] bf16, w [B][H] fp32, keys bf16 dim 128
+ *   q_attn [B][64][512] bf16, kv and swa bf16 dim 512 (64 query heads)
+ *   out [B][64][512] fp32, lse [B][64] (optional)
+ *   scores [B][ld_scores] fp32 (optional), ids [B][k] int32 ascending with -1
+ *           padding (optional), n_sel [B] (optional): the intermediate
+ *           results, written when given
+ *   prefetch[i], prefetch_bytes[i] (optional): device ranges to pull into L2
+ *           while this layer runs, e.g. the next layer's index keys and window
+ *           rows, which are known before its query is (a hint; no result
+ *           depends on it).  16-byte aligned, sizes multiples of 16.
+ *
+ * Supported: bf16 keys, rows and queries, H a multiple of 32 up to 128,
+ * N <= 32768, and B * ceil((swa_len + k) / 64) * 4 <= the device's SM count
+ * (every attention unit runs concurrently); otherwise LIDX_ERR_UNSUPPORTED
+ * (use the three calls).  The workspace (lidx_workspace_size(LIDX_OP_DECODE))
+ * must be zeroed before its first use; every call leaves its control words
+ * zeroed again.  One workspace serves one call at a time.
+ * ------------------------------------------------------------------------ */
+typedef struct lidx_decode_args {
+    int32_t B, H, N, k;
+    const void *q_idx;
+    const float *w;
+    lidx_kv keys;
+    int32_t H_attn;        /* must be 64 */
+    const void *q_attn;
+    lidx_kv kv;
+    lidx_kv swa;
+    int32_t swa_len;
+    float scale;
+    float *out;
+    float *lse;
+    float *scores;
+    int64_t ld_scores;
+    int32_t *ids;
+    int32_t *n_sel;
+    const void *prefetch[2];
+    uint64_t prefetch_bytes[2];
+    uint32_t flags;        /* LIDX_LAUNCH_* */
+} lidx_decode_args;
+
+LIDX_API lidx_status lidx_decode_layer(const lidx_decode_args *args, void *ws, size_t ws_bytes, void *stream);
 
 /* ------------------------------------------------------------------------
  * lidx_sparse_attn_decode_noalloc -- lidx_sparse_attn_decode without a
@@ -321,6 +387,7 @@ LIDX_API lidx_status lidx_selection_eval(const lidx_eval_args *args, void *ws, s
 #define LIDX_OP_TOPK 1
 #define LIDX_OP_ATTN 2
 #define LIDX_OP_EVAL 3
+#define LIDX_OP_DECODE 4
 
 /* Bytes of workspace call `op` needs for `args` (a pointer to the matching
  * *_args struct, host memory).  Score needs none (0). */
@@ -337,7 +404,7 @@ LIDX_API const char *lidx_status_string(lidx_status s);
 LIDX_API int lidx_abi_version(void);
 
 /* sizeof() of the argument structs as compiled into the library, for binding
- * checks: which = 0 lidx_kv, 1 score, 2 topk, 3 attn, 4 eval. */
+ * checks: which = 0 lidx_kv, 1 score, 2 topk, 3 attn, 4 eval, 5 decode. */
 LIDX_API size_t lidx_struct_size(int which);
 
 #ifdef __cplusplus

@@ -30,10 +30,11 @@ DTYPES = {"f32": F32, "bf16": BF16, "e4m3": E4M3, "f16": F16}
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_WORKSPACE = 0, 1, 2, 3, 4
 DEV_BOUNDS, DEV_NAN, DEV_TIMEOUT = 0x1, 0x2, 0x4
 LAUNCH_PDL = 0x1
+LAUNCH_TEST_LOST_ARRIVAL = 0x80000000
 STATS_SPAN = 32  # entries per score-bounds record (optional scorer output, top-k input)
 
 EVAL_GOLDEN, EVAL_TOPP, EVAL_VOTE, EVAL_LSA, EVAL_OVERLAP = 0x1, 0x2, 0x4, 0x8, 0x10
-OP_SCORE, OP_TOPK, OP_ATTN, OP_EVAL = 0, 1, 2, 3
+OP_SCORE, OP_TOPK, OP_ATTN, OP_EVAL, OP_DECODE = 0, 1, 2, 3, 4
 
 # Layer schedule of DeepSeek-V4-Flash (architecture post, section (A) table):
 # layers 0-1 sliding window only, even layers 2..42 CSA (4:1 + top-k), odd
@@ -95,7 +96,8 @@ class TopkArgs(C.Structure):
     _fields_ = [("B", C.c_int32), ("Q", C.c_int32), ("N", C.c_int32), ("k", C.c_int32),
                 ("scores", C.c_void_p), ("ld_scores", C.c_int64), ("allowed", C.c_void_p),
                 ("ld_allowed", C.c_int64), ("ids", C.c_void_p), ("n_sel", C.c_void_p), ("mask", C.c_void_p),
-                ("mask_bits", C.c_void_p), ("flags", C.c_uint32), ("tile_stats", C.c_void_p)]
+                ("mask_bits", C.c_void_p), ("flags", C.c_uint32), ("tile_stats", C.c_void_p),
+                ("allowed_bits", C.c_void_p), ("ld_allowed_bits", C.c_int64)]
 
 
 class AttnArgs(C.Structure):
@@ -116,10 +118,19 @@ class EvalArgs(C.Structure):
                 ("counts", C.c_void_p)]
 
 
-_STRUCTS = [KVArgs, ScoreArgs, TopkArgs, AttnArgs, EvalArgs]
+class DecodeArgs(C.Structure):
+    _fields_ = [("B", C.c_int32), ("H", C.c_int32), ("N", C.c_int32), ("k", C.c_int32),
+                ("q_idx", C.c_void_p), ("w", C.c_void_p), ("keys", KVArgs), ("H_attn", C.c_int32),
+                ("q_attn", C.c_void_p), ("kv", KVArgs), ("swa", KVArgs), ("swa_len", C.c_int32),
+                ("scale", C.c_float), ("out", C.c_void_p), ("lse", C.c_void_p), ("scores", C.c_void_p),
+                ("ld_scores", C.c_int64), ("ids", C.c_void_p), ("n_sel", C.c_void_p),
+                ("prefetch", C.c_void_p * 2), ("prefetch_bytes", C.c_uint64 * 2), ("flags", C.c_uint32)]
+
+
+_STRUCTS = [KVArgs, ScoreArgs, TopkArgs, AttnArgs, EvalArgs, DecodeArgs]
 EXPORTS = ("lidx_index_score", "lidx_topk_select", "lidx_sparse_attn_decode", "lidx_selection_eval",
-           "lidx_workspace_size", "lidx_read_device_status", "lidx_status_string", "lidx_abi_version",
-           "lidx_struct_size")
+           "lidx_decode_layer", "lidx_workspace_size", "lidx_read_device_status", "lidx_status_string",
+           "lidx_abi_version", "lidx_struct_size")
 
 _lib = None
 _lock = threading.Lock()
@@ -140,6 +151,7 @@ def lib():
                 ("lidx_topk_select", I, [C.POINTER(TopkArgs), P, SZ, P]),
                 ("lidx_sparse_attn_decode", I, [C.POINTER(AttnArgs), P, SZ, P]),
                 ("lidx_selection_eval", I, [C.POINTER(EvalArgs), P, SZ, P]),
+                ("lidx_decode_layer", I, [C.POINTER(DecodeArgs), P, SZ, P]),
                 ("lidx_workspace_size", I, [I, P, C.POINTER(SZ)]),
                 ("lidx_read_device_status", I, [P, C.POINTER(C.c_uint32), P]),
                 ("lidx_status_string", C.c_char_p, [I]),
@@ -262,20 +274,24 @@ def workspace(nbytes: int, device="cuda") -> torch.Tensor:
 
 
 def topk_args(scores, k, allowed=None, ids=None, n_sel=None, mask=None, mask_bits=None, flags=0,
-              tile_stats=None) -> TopkArgs:
+              tile_stats=None, allowed_bits=None) -> TopkArgs:
     B, Q, N = scores.shape[0], scores.shape[1], scores.shape[2]
+    ldb = 0 if allowed_bits is None else (allowed_bits.stride(0) if allowed_bits.dim() > 1 else (N + 31) // 32)
     return TopkArgs(B, Q, N, k, scores.data_ptr(), scores.stride(1), _ptr(allowed),
                     0 if allowed is None else allowed.stride(0), _ptr(ids), _ptr(n_sel), _ptr(mask),
-                    _ptr(mask_bits), flags, _ptr(tile_stats))
+                    _ptr(mask_bits), flags, _ptr(tile_stats), _ptr(allowed_bits), ldb)
 
 
 def topk_select(scores: torch.Tensor, k: int, allowed: torch.Tensor = None, *, want_mask=False,
-                want_bits=False, ids=None, n_sel=None, ws=None, stream=None, tile_stats=None, bits=None):
+                want_bits=False, ids=None, n_sel=None, ws=None, stream=None, tile_stats=None, bits=None,
+                allowed_bits: torch.Tensor = None):
     """Top-k row ids of scores [B][Q][N] (N = scores.shape[2]).
 
     Returns (ids int32 [B][Q][k] ascending with -1 padding, n_sel int32 [B][Q],
     mask uint8 [B][Q][N] or None, bits uint32 [B][Q][ceil(N/32)] or None).
-    `tile_stats` are the score bounds index_score wrote for these scores."""
+    `tile_stats` are the score bounds index_score wrote for these scores.
+    `allowed` (uint8 [B][N]) and `allowed_bits` (int32 [B][ceil(N/32)], e.g.
+    the gate's fetched set) restrict the eligible entries."""
     B, Q, N = scores.shape
     dev = scores.device
     ids = torch.empty((B, Q, k), dtype=torch.int32, device=dev) if ids is None else ids
@@ -283,7 +299,7 @@ def topk_select(scores: torch.Tensor, k: int, allowed: torch.Tensor = None, *, w
     mask = torch.empty((B, Q, N), dtype=torch.uint8, device=dev) if want_mask else None
     if bits is None and want_bits:
         bits = torch.empty((B, Q, (N + 31) // 32), dtype=torch.int32, device=dev)
-    a = topk_args(scores, k, allowed, ids, n_sel, mask, bits, tile_stats=tile_stats)
+    a = topk_args(scores, k, allowed, ids, n_sel, mask, bits, tile_stats=tile_stats, allowed_bits=allowed_bits)
     if ws is None:
         ws = workspace(workspace_size(OP_TOPK, a), dev)
     _check(lib().lidx_topk_select(C.byref(a), C.c_void_p(ws.data_ptr()), ws.numel(), _stream(stream)),
@@ -292,9 +308,10 @@ def topk_select(scores: torch.Tensor, k: int, allowed: torch.Tensor = None, *, w
 
 
 def attn_args(q, kv: DeviceKV, N, ids, n_sel, swa: Optional[DeviceKV], swa_len, scale, out, lse,
-              flags=0) -> AttnArgs:
+              flags=0, n_dense=0) -> AttnArgs:
+    """ids None with n_dense > 0: the dense rows 0..n_dense-1 (HCA layers)."""
     B, H, D = q.shape
-    n_ids = 0 if ids is None else ids.shape[-1]
+    n_ids = n_dense if ids is None else ids.shape[-1]
     ld_ids = 0 if ids is None else ids.stride(0)
     swa_a = swa.args() if swa is not None else KVArgs(kv.dtype, kv.dim, None, None, None, 0, 0, 0, 0)
     return AttnArgs(B, H, _qdtype(q), q.data_ptr(), kv.args(), N, _ptr(ids), n_ids, ld_ids, _ptr(n_sel),
@@ -303,9 +320,11 @@ def attn_args(q, kv: DeviceKV, N, ids, n_sel, swa: Optional[DeviceKV], swa_len, 
 
 def sparse_attn_decode(q: torch.Tensor, kv: DeviceKV, N: int, ids: torch.Tensor, n_sel: torch.Tensor = None,
                        swa: DeviceKV = None, swa_len: int = 0, scale: float = None, *, out=None, lse=None,
-                       want_lse=True, ws=None, stream=None):
+                       want_lse=True, ws=None, stream=None, n_dense=0):
     """MQA decode attention of q [B][H][512] over rows ids [B][n] (-1 skipped;
-    the first n_sel[b] when given) of kv plus swa rows 0..swa_len-1.
+    the first n_sel[b] when given) of kv plus swa rows 0..swa_len-1.  With
+    ids None the rows are 0..n_dense-1 of every sequence, read whole (the HCA
+    layers: every compressed entry, no top-k).
 
     Returns (out float32 [B][H][512], lse float32 [B][H] or None)."""
     B, H, D = q.shape
@@ -314,11 +333,51 @@ def sparse_attn_decode(q: torch.Tensor, kv: DeviceKV, N: int, ids: torch.Tensor,
     out = torch.empty((B, H, D), dtype=torch.float32, device=q.device) if out is None else out
     if want_lse and lse is None:
         lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
-    a = attn_args(q, kv, N, ids, n_sel, swa, swa_len, scale, out, lse)
+    a = attn_args(q, kv, N, ids, n_sel, swa, swa_len, scale, out, lse, n_dense=n_dense)
     if ws is None:
         ws = workspace(workspace_size(OP_ATTN, a), q.device)
     _check(lib().lidx_sparse_attn_decode(C.byref(a), C.c_void_p(ws.data_ptr()), ws.numel(), _stream(stream)),
            "lidx_sparse_attn_decode")
+    return out, lse
+
+
+def decode_args(q_idx, w, keys: DeviceKV, N: int, k: int, q_attn, kv: DeviceKV, swa: Optional[DeviceKV],
+                swa_len: int, scale: float, out, lse=None, scores=None, ids=None, n_sel=None, prefetch=(),
+                flags=0) -> DecodeArgs:
+    """Argument struct of lidx_decode_layer; q_idx [B][H][128] (or [B][1][H][128]),
+    w [B][H], q_attn [B][64][512]; `prefetch` is up to two (pointer, bytes)
+    pairs pulled into L2 while the layer runs."""
+    B = q_attn.shape[0]
+    H = w.shape[-1]
+    swa_a = swa.args() if swa is not None else KVArgs(kv.dtype, kv.dim, None, None, None, 0, 0, 0, 0)
+    pf = list(prefetch)[:2] + [(None, 0)] * (2 - len(list(prefetch)[:2]))
+    return DecodeArgs(B, H, N, k, q_idx.data_ptr(), w.data_ptr(), keys.args(), q_attn.shape[1], q_attn.data_ptr(),
+                      kv.args(), swa_a, swa_len if swa is not None else 0, float(scale), out.data_ptr(), _ptr(lse),
+                      _ptr(scores), 0 if scores is None else scores.stride(-2) if scores.dim() > 1 else N,
+                      _ptr(ids), _ptr(n_sel), (C.c_void_p * 2)(*[x[0] for x in pf]),
+                      (C.c_uint64 * 2)(*[x[1] for x in pf]), flags)
+
+
+def decode_layer(q_idx: torch.Tensor, w: torch.Tensor, keys: DeviceKV, N: int, k: int, q_attn: torch.Tensor,
+                 kv: DeviceKV, swa: DeviceKV = None, swa_len: int = 0, scale: float = None, *, out=None, lse=None,
+                 want_lse=True, scores=None, ids=None, n_sel=None, prefetch=(), flags=0, ws=None, stream=None):
+    """One CSA decode layer in one launch: index scores -> top-k -> sparse
+    attention over the selected rows plus the window (lidx_decode_layer).
+    Returns (out [B][64][512], lse [B][64] or None); `scores`, `ids` and
+    `n_sel` are filled when given.  `ws` must be zeroed before its first
+    use (workspace() is); the call leaves it ready for the next one."""
+    B = q_attn.shape[0]
+    if scale is None:
+        scale = q_attn.shape[-1] ** -0.5
+    out = torch.empty((B, q_attn.shape[1], 512), dtype=torch.float32, device=q_attn.device) if out is None else out
+    if want_lse and lse is None:
+        lse = torch.empty((B, q_attn.shape[1]), dtype=torch.float32, device=q_attn.device)
+    a = decode_args(q_idx, w, keys, N, k, q_attn, kv, swa, swa_len, scale, out, lse, scores, ids, n_sel, prefetch,
+                    flags)
+    if ws is None:
+        ws = workspace(workspace_size(OP_DECODE, a), q_attn.device)
+    _check(lib().lidx_decode_layer(C.byref(a), C.c_void_p(ws.data_ptr()), ws.numel(), _stream(stream)),
+           "lidx_decode_layer")
     return out, lse
 
 

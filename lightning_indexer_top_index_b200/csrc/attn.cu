@@ -77,7 +77,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int kind = 0;
     int64_t r = 0;
     if (i < n_b) {
-      const int id = a.ids[static_cast<int64_t>(b) * a.ld_ids + i];
+      const int id = a.ids ? a.ids[static_cast<int64_t>(b) * a.ld_ids + i] : i;  // no ids: dense rows
       if (id >= 0 && id < a.N) {
         kind = 1;
         r = static_cast<int64_t>(b) * a.kv.batch_rows + id;

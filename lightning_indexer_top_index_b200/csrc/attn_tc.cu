@@ -200,7 +200,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     auto resolve_row = [&](int r, int &kind, int64_t &src) {
       const int i = i0 + r - swa_len;
       if (i >= 0 && i < n_b) {
-        const int id = a.ids[static_cast<int64_t>(b) * a.ld_ids + i];
+        const int id = a.ids ? a.ids[static_cast<int64_t>(b) * a.ld_ids + i] : i;  // no ids: dense rows
         if (id >= 0 && id < a.N) {
           kind = 1;
           src = static_cast<int64_t>(b) * a.kv.batch_rows + id;

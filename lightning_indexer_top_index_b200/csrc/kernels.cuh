@@ -33,6 +33,11 @@ cudaError_t launch_topk(const lidx_topk_args &a, void *ws, cudaStream_t st);
 size_t attn_workspace(const lidx_attn_args &a);
 cudaError_t launch_attn(const lidx_attn_args &a, void *ws, cudaStream_t st);
 
+// ---- fused decode layer (score -> top-k -> attention in one launch)
+bool decode_fused_supported(const lidx_decode_args &a);
+size_t decode_fused_workspace(const lidx_decode_args &a);
+cudaError_t launch_decode_fused(const lidx_decode_args &a, void *ws, cudaStream_t st);
+
 // ---- selection evaluation
 bool golden_tc_supported(const lidx_eval_args &a);
 size_t golden_tc_workspace(const lidx_eval_args &a);

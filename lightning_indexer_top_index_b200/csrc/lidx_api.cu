@@ -72,6 +72,8 @@ lidx_status check_topk(const lidx_topk_args *a) {
   if (!a || !a->scores || !a->ids) return LIDX_ERR_INVALID_ARG;
   if (a->B < 1 || a->Q < 1 || a->N < 1 || a->k < 1 || a->ld_scores < a->N) return LIDX_ERR_INVALID_ARG;
   if (a->allowed && a->ld_allowed < a->N) return LIDX_ERR_INVALID_ARG;
+  if (a->allowed_bits && (a->ld_allowed_bits < (a->N + 31) / 32 || !aligned(a->allowed_bits, 4)))
+    return LIDX_ERR_INVALID_ARG;
   if (!aligned(a->scores, 4) || !aligned(a->ids, 4) || (a->mask_bits && !aligned(a->mask_bits, 4)))
     return LIDX_ERR_INVALID_ARG;
   if (a->tile_stats && !aligned(a->tile_stats, 8)) return LIDX_ERR_INVALID_ARG;
@@ -82,7 +84,9 @@ lidx_status check_topk(const lidx_topk_args *a) {
 lidx_status check_attn(const lidx_attn_args *a) {
   if (!a || !a->q || !a->out) return LIDX_ERR_INVALID_ARG;
   if (a->B < 1 || a->H < 1 || a->H > 64 || a->n_ids < 0 || a->swa_len < 0) return LIDX_ERR_INVALID_ARG;
-  if (a->n_ids > 0 && (!a->ids || a->ld_ids < a->n_ids || a->N < 1)) return LIDX_ERR_INVALID_ARG;
+  if (a->n_ids > 0 && a->N < 1) return LIDX_ERR_INVALID_ARG;
+  if (a->n_ids > 0 && a->ids && a->ld_ids < a->n_ids) return LIDX_ERR_INVALID_ARG;
+  if (a->n_ids > a->N && !a->ids) return LIDX_ERR_INVALID_ARG;  // dense rows 0..n_ids-1 must exist
   if (!(a->scale == a->scale) || a->scale == INFINITY || a->scale == -INFINITY) return LIDX_ERR_INVALID_ARG;
   if (a->n_ids > 0) {
     lidx_status s = check_kv(a->kv, 512, a->B, a->N);
@@ -125,6 +129,26 @@ lidx_status check_eval(const lidx_eval_args *a) {
   if (a->ops & LIDX_EVAL_OVERLAP) {
     if (!a->set_a || !a->set_b || !a->counts || a->n_pairs < 1 || a->ld_a < 0 || a->ld_b < 0) return LIDX_ERR_INVALID_ARG;
   }
+  return LIDX_OK;
+}
+
+lidx_status check_decode(const lidx_decode_args *a) {
+  if (!a || !a->q_idx || !a->w || !a->q_attn || !a->out) return LIDX_ERR_INVALID_ARG;
+  if (a->B < 1 || a->H < 1 || a->N < 1 || a->k < 1 || a->swa_len < 0 || a->H_attn < 1) return LIDX_ERR_INVALID_ARG;
+  if (!(a->scale == a->scale) || a->scale == INFINITY || a->scale == -INFINITY) return LIDX_ERR_INVALID_ARG;
+  lidx_status s = check_kv(a->keys, 128, a->B, a->N);
+  if (s != LIDX_OK) return s;
+  if ((s = check_kv(a->kv, 512, a->B, a->N)) != LIDX_OK) return s;
+  if (a->swa_len > 0 && (s = check_kv(a->swa, 512, a->B, a->swa_len)) != LIDX_OK) return s;
+  if (a->scores && a->ld_scores < a->N) return LIDX_ERR_INVALID_ARG;
+  if (!aligned(a->q_idx, 16) || !aligned(a->q_attn, 16) || !aligned(a->w, 4) || !aligned(a->out, 16))
+    return LIDX_ERR_INVALID_ARG;
+  if ((a->scores && !aligned(a->scores, 4)) || (a->ids && !aligned(a->ids, 4)) || (a->n_sel && !aligned(a->n_sel, 4)) ||
+      (a->lse && !aligned(a->lse, 4)))
+    return LIDX_ERR_INVALID_ARG;
+  for (int r = 0; r < 2; r++)
+    if (a->prefetch[r] && (!aligned(a->prefetch[r], 16) || a->prefetch_bytes[r] % 16 != 0)) return LIDX_ERR_INVALID_ARG;
+  if (!decode_fused_supported(*a)) return LIDX_ERR_UNSUPPORTED;
   return LIDX_OK;
 }
 
@@ -174,6 +198,14 @@ lidx_status lidx_selection_eval(const lidx_eval_args *args, void *ws, size_t ws_
   return from_cuda(launch_eval(*args, ws, static_cast<cudaStream_t>(stream)));
 }
 
+lidx_status lidx_decode_layer(const lidx_decode_args *args, void *ws, size_t ws_bytes, void *stream) {
+  lidx_status s = check_device();
+  if (s != LIDX_OK) return s;
+  if ((s = check_decode(args)) != LIDX_OK) return s;
+  if ((s = check_ws(ws, ws_bytes, decode_fused_workspace(*args))) != LIDX_OK) return s;
+  return from_cuda(launch_decode_fused(*args, ws, static_cast<cudaStream_t>(stream)));
+}
+
 lidx_status lidx_workspace_size(int op, const void *args, size_t *bytes) {
   if (!args || !bytes) return LIDX_ERR_INVALID_ARG;
   lidx_status s = LIDX_OK;
@@ -193,6 +225,10 @@ lidx_status lidx_workspace_size(int op, const void *args, size_t *bytes) {
     case LIDX_OP_EVAL:
       s = check_eval(static_cast<const lidx_eval_args *>(args));
       if (s == LIDX_OK) *bytes = eval_workspace(*static_cast<const lidx_eval_args *>(args));
+      break;
+    case LIDX_OP_DECODE:
+      s = check_decode(static_cast<const lidx_decode_args *>(args));
+      if (s == LIDX_OK) *bytes = decode_fused_workspace(*static_cast<const lidx_decode_args *>(args));
       break;
     default:
       return LIDX_ERR_INVALID_ARG;
@@ -229,6 +265,7 @@ size_t lidx_struct_size(int which) {
     case 2: return sizeof(lidx_topk_args);
     case 3: return sizeof(lidx_attn_args);
     case 4: return sizeof(lidx_eval_args);
+    case 5: return sizeof(lidx_decode_args);
   }
   return 0;
 }

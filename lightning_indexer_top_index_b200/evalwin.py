@@ -9,8 +9,14 @@ FlashMemory-vs-native post, Acts 1 and 3), on the library's calls:
   window        the >= min_votes layer vote per query and its union G
   gate          the gate's logits at its layers (the index scorer with the
                 gate query and signed head weights) and the fetched set F
+  fetched top-k the native top-k inside F (the tiering of the comparison:
+                the native indexer keeps its top-k among the entries the gate
+                fetched; FlashMemory-vs-native post, "The setup"; write-up,
+                reply #2)
   overlap       |A & B|, |A|, |B| for native vs golden top-k (per layer and
-                query), native top-k vs F (per layer and query), and G vs F
+                query), native top-k vs F (per layer and query), G vs F, and
+                the top-k inside F vs the golden top-k and vs the unrestricted
+                native top-k (per layer and query)
 
 The window owns its buffers and workspaces; `enqueue` only issues the calls.
 """
@@ -60,6 +66,11 @@ class EvalWindow:
         self.counts_nat_gold = torch.zeros((L * T, 3), dtype=torch.int64, device=dev)
         self.counts_nat_f = torch.zeros((L * T, 3), dtype=torch.int64, device=dev)
         self.counts_g_f = torch.zeros((1, 3), dtype=torch.int64, device=dev)
+        self.natf_ids = torch.empty((L, 1, T, k), dtype=torch.int32, device=dev)
+        self.natf_n = torch.empty((L, 1, T), dtype=torch.int32, device=dev)
+        self.natf_bits = torch.zeros((L, 1, T, W), dtype=torch.int32, device=dev)
+        self.counts_natf_gold = torch.zeros((L * T, 3), dtype=torch.int64, device=dev)
+        self.counts_natf_nat = torch.zeros((L * T, 3), dtype=torch.int64, device=dev)
         # workspaces sized once
         ta = topk_args(self.scores[0], k, None, self.nat_ids[0], self.nat_n[0], None, self.nat_bits[0])
         self.ws_topk_nat = workspace(workspace_size(OP_TOPK, ta), dev)
@@ -74,8 +85,8 @@ class EvalWindow:
     def enqueue(self, stream=None, events: Optional[Dict] = None):
         """Issue the window's calls on `stream` (default: current).  With
         `events` (name -> (start, end) CUDA events) the stages "score",
-        "topk", "golden", "topp", "gold_topk", "vote", "gate" and "overlap"
-        are bracketed for timing."""
+        "topk", "golden", "topp", "gold_topk", "vote", "gate", "fetched_topk"
+        and "overlap" are bracketed for timing."""
         L, T, H, N, k = self.L, self.T, self.H, self.N, self.k
         st = stream or torch.cuda.current_stream()
 
@@ -115,6 +126,12 @@ class EvalWindow:
         selection_eval(EVAL_LSA, N=N, gate_logits=self.gate_logits.view(-1, N), fetched_bits=self.fetched_bits,
                        ws=self.ws_small, stream=st)
         mark("gate", 1)
+        mark("fetched_topk", 0)
+        fb = self.fetched_bits.view(1, self.W)
+        for l in range(L):
+            topk_select(self.scores[l], k, want_bits=True, ids=self.natf_ids[l], n_sel=self.natf_n[l],
+                        bits=self.natf_bits[l], ws=self.ws_topk_nat, stream=st, allowed_bits=fb)
+        mark("fetched_topk", 1)
         mark("overlap", 0)
         W = self.W
         selection_eval(EVAL_OVERLAP, N=N, set_a=self.nat_bits.view(L * T, W), set_b=self.gold_bits.view(L * T, W),
@@ -123,16 +140,21 @@ class EvalWindow:
                        n_pairs=L * T, counts=self.counts_nat_f, ws=self.ws_small, stream=st)
         selection_eval(EVAL_OVERLAP, N=N, set_a=self.window_bits, set_b=self.fetched_bits, ld_a=0, ld_b=0,
                        n_pairs=1, counts=self.counts_g_f, ws=self.ws_small, stream=st)
+        selection_eval(EVAL_OVERLAP, N=N, set_a=self.natf_bits.view(L * T, W), set_b=self.gold_bits.view(L * T, W),
+                       n_pairs=L * T, counts=self.counts_natf_gold, ws=self.ws_small, stream=st)
+        selection_eval(EVAL_OVERLAP, N=N, set_a=self.natf_bits.view(L * T, W), set_b=self.nat_bits.view(L * T, W),
+                       n_pairs=L * T, counts=self.counts_natf_nat, ws=self.ws_small, stream=st)
         mark("overlap", 1)
 
     def kernel_launches(self) -> int:
-        """Kernels one window launches: per layer a scorer and a top-k, the
-        golden probabilities (two tensor-core passes around the lse merge on
-        the tcgen05 path, else the lse and probability kernels), top-p, the
-        golden top-k, the vote and its union, a scorer per gate layer and the
-        gate OR, and three overlap counts."""
+        """Kernels one window launches: per layer a scorer, a top-k and a
+        top-k inside the fetched set, the golden probabilities (two
+        tensor-core passes around the lse merge on the tcgen05 path, else the
+        lse and probability kernels), top-p, the golden top-k, the vote and
+        its union, a scorer per gate layer and the gate OR, and five overlap
+        counts."""
         golden = 3 if self.H == 64 and self.qa.dtype == torch.bfloat16 and self.kv_all.dtype == BF16 else 2
-        return 2 * self.L + golden + 1 + 1 + 2 + len(self.gate_layers) + 1 + 3
+        return 3 * self.L + golden + 1 + 1 + 2 + len(self.gate_layers) + 1 + 5
 
     def golden_flops(self) -> float:
         """Tensor FLOPs of the golden passes: two GEMMs of (T*H) x N x 512 per layer."""

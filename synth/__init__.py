@@ -21,8 +21,10 @@ Every tensor draws from its own numpy ``SeedSequence`` keyed by
 """
 from __future__ import annotations
 
+import concurrent.futures
 import dataclasses
 import math
+import os
 from typing import Optional
 
 import numpy as np
@@ -263,12 +265,13 @@ def decode_layer(spec: DecodeSpec, layer: int = 0) -> dict:
     B, N, H = spec.B, spec.N, spec.H
     s, l = spec.seed, layer
     sd_idx = 1.0 / math.sqrt(spec.D_idx)
-    qs, ws, keys, kvs, swas, qas, planted = [], [], [], [], [], [], []
-    for b in range(B):
+
+    def one(b):  # every array of sequence b comes from its own streams
         q = _normal(rng(s, TAG_Q_IDX, l, b), (H, spec.D_idx), sd_idx)
         w = rng(s, TAG_W, l, b).random(H).astype(np.float32)
         k = _normal(rng(s, TAG_KEYS, l, b), (N, spec.D_idx), sd_idx)
         q_st = q.astype(np.float32) if spec.q_dtype == "f32" else bf16_bits(q)
+        rows = None
         if spec.plant:
             # planted rows: shift chosen rows along g = sum_h q_h / |sum_h q_h|
             # so the head-mean of q_h . k rises by 3 sigma (sigma = 1/sqrt(128)).
@@ -279,21 +282,44 @@ def decode_layer(spec: DecodeSpec, layer: int = 0) -> dict:
             c = 3.0 * sd_idx * H / gnorm
             rows = np.sort(rng(s, TAG_PLANT, l, b).choice(N, size=spec.k, replace=False))
             k[rows] += c * ghat
-            planted.append(rows.astype(np.int32))
-        qs.append(q_st)
-        ws.append(w)
-        keys.append(encode_rows(k, spec.key_dtype))
+            rows = rows.astype(np.int32)
+        key = encode_rows(k, spec.key_dtype)
         x = _normal(rng(s, TAG_KV, l, b), (N, spec.D_attn), 1.0)
-        kvs.append(encode_rows(x, spec.kv_dtype))
+        kv = encode_rows(x, spec.kv_dtype)
         sw = _normal(rng(s, TAG_SWA, l, b), (spec.swa, spec.D_attn), 1.0)
-        swas.append(encode_rows(sw, spec.kv_dtype))
+        swa = encode_rows(sw, spec.kv_dtype)
         qa = _normal(rng(s, TAG_Q_ATTN, l, b), (H, spec.D_attn), 1.0)
-        qas.append(qa.astype(np.float32) if spec.q_dtype == "f32" else bf16_bits(qa))
+        qa = qa.astype(np.float32) if spec.q_dtype == "f32" else bf16_bits(qa)
+        return q_st, w, key, kv, swa, qa, rows
+
+    if B > 1 and B * N >= 1 << 16:
+        with concurrent.futures.ThreadPoolExecutor(min(B, os.cpu_count() or 1)) as ex:
+            parts = list(ex.map(one, range(B)))
+    else:
+        parts = [one(b) for b in range(B)]
+    qs, ws, keys, kvs, swas, qas, planted = (list(t) for t in zip(*parts))
     out = dict(q_idx=np.stack(qs), w=np.stack(ws), keys=concat_kv(keys), kv=concat_kv(kvs),
                swa=concat_kv(swas), q_attn=np.stack(qas))
     if spec.plant:
         out["planted"] = np.stack(planted)
     return out
+
+
+def model_layer(spec: DecodeSpec, layer: int) -> dict:
+    """Inputs of model layer `layer` of the hybrid schedule for one decode
+    token (architecture post, section (A): layers 0-1 sliding window only,
+    even layers 2-42 CSA, odd layers 3-41 HCA).  A CSA layer is
+    decode_layer(spec, (layer - 2) // 2); an HCA layer has spec.N // 32
+    compressed rows (128:1 against CSA's 4:1) of width 512 ~ N(0,1), its
+    window and attention queries; an SWA layer has its window and queries.
+    Returns a dict with "kind" and the arrays."""
+    if layer >= 2 and layer % 2 == 0:
+        return dict(kind="csa", **decode_layer(spec, (layer - 2) // 2))
+    sub = dataclasses.replace(spec, N=max(1, spec.N // 32), plant=False)
+    x = decode_layer(sub, 1000 + layer)  # its own streams: layer ids 1000+ are not used by CSA layers
+    if layer < 2:
+        return dict(kind="swa", swa=x["swa"], q_attn=x["q_attn"])
+    return dict(kind="hca", N=sub.N, kv=x["kv"], swa=x["swa"], q_attn=x["q_attn"])
 
 
 # ----------------------------------------------------------------------------

@@ -79,3 +79,20 @@ def test_eval_window_against_oracle(cuda_device):
             assert tuple(c_ng[l * T + t]) == oracle.overlap(nat_bits[l, t], gold_bits[l, t], N)
             assert tuple(c_nf[l * T + t]) == oracle.overlap(nat_bits[l, t], fetched, N)
     assert tuple(win.counts_g_f.cpu().numpy()[0]) == oracle.overlap(window_bits, fetched, N)
+    # the native top-k inside the fetched set, and its overlaps
+    natf_bits = win.natf_bits.cpu().numpy().view(np.uint32).reshape(Lq, T, W)
+    natf_ids = win.natf_ids.cpu().numpy().reshape(Lq, T, spec.k)
+    natf_n = win.natf_n.cpu().numpy().reshape(Lq, T)
+    allowed = synth.unpack_bits(fetched[None], N)[0].astype(np.uint8)
+    assert 0 < allowed.sum() < N  # the gate neither fetched nothing nor everything
+    c_fg = win.counts_natf_gold.cpu().numpy()
+    c_fn = win.counts_natf_nat.cpu().numpy()
+    for l in range(Lq):
+        for t in range(T):
+            ids, n, _ = oracle.topk(scores[l, 0, t], spec.k, allowed)
+            assert natf_n[l, t] == n and np.array_equal(natf_ids[l, t], ids)
+            dense = np.zeros(N, bool)
+            dense[ids[:n]] = True
+            assert np.array_equal(natf_bits[l, t], synth.pack_bits(dense)[0])
+            assert tuple(c_fg[l * T + t]) == oracle.overlap(natf_bits[l, t], gold_bits[l, t], N)
+            assert tuple(c_fn[l * T + t]) == oracle.overlap(natf_bits[l, t], nat_bits[l, t], N)

@@ -142,6 +142,30 @@ def test_topk_allowed_mask_and_nan():
     assert L.read_device_status(ws) == 0
 
 
+@pytest.mark.parametrize("N,k,density", [(5000, 256, 0.3), (16384, 512, 0.05), (16384, 512, 0.5), (777, 64, 0.0)])
+def test_topk_allowed_bits(N, k, density):
+    """A bit-set of eligible entries (the gate's fetched set): the top-k
+    inside it, bit-exact against the oracle with the same set as a mask."""
+    rows = 3
+    s = synth.random_scores(24, rows, N, "ties")
+    bits = synth.random_bits(25, rows, N, density)
+    allowed = synth.unpack_bits(bits, N).astype(np.uint8)
+    st = torch.from_numpy(s).cuda().reshape(rows, 1, N)
+    bt = torch.from_numpy(bits.view(np.int32)).cuda()
+    ids, n_sel, _, _ = L.topk_select(st, k, allowed_bits=bt)
+    ids, n_sel = ids.cpu().numpy(), n_sel.cpu().numpy()
+    for r in range(rows):
+        ref_ids, ref_n, _ = oracle.topk(s[r], k, allowed[r])
+        assert n_sel[r, 0] == ref_n and np.array_equal(ids[r, 0], ref_ids), f"row {r}"
+    # both restrictions at once: the eligible entries are their intersection
+    al2 = (np.random.default_rng(26).random((rows, N)) < 0.5).astype(np.uint8)
+    ids, n_sel, _, _ = L.topk_select(st, k, torch.from_numpy(al2).cuda(), allowed_bits=bt)
+    ids = ids.cpu().numpy()
+    for r in range(rows):
+        ref_ids, _, _ = oracle.topk(s[r], k, allowed[r] & al2[r])
+        assert np.array_equal(ids[r, 0], ref_ids), f"row {r}"
+
+
 # --------------------------------------------------------------- attention
 def _attn_case(spec, n_sel=None, swa_len=None, ids=None, layer=0):
     inp = synth.decode_layer(spec, layer)
@@ -328,3 +352,47 @@ def test_vote_union_lsa_overlap_bit_exact(N):
     c = counts.cpu().numpy()
     for p in range(6):
         assert tuple(c[p]) == oracle.overlap(A[p], B[p], N)
+
+
+# ------------------------------------------------------ dense (HCA) layers
+@pytest.mark.parametrize("spec,swa_len", [
+    (synth.scaled(synth.DECODE_64K, N=512, k=512), 128),
+    (synth.scaled(synth.DECODE_64K, N=512, k=512, B=3), 77),
+    (synth.scaled(synth.DECODE_64K, N=300, k=300, B=2), 0),
+    (synth.scaled(synth.DECODE_500K_FP8, N=3907, k=3907, B=2), 128),
+    (synth.scaled(synth.TINY_1K_F32, N=32, k=32), 128),
+], ids=lambda x: f"{x.name}-N{x.N}-B{x.B}" if hasattr(x, "name") else f"swa{x}")
+def test_attn_dense_rows_hca(spec, swa_len):
+    """The HCA layers of the architecture post (section (A): 128:1
+    compression, about 512 entries at 64K, every entry read, no top-k): the
+    attention with no ids reads rows 0..N-1 of every sequence; the oracle
+    attends over ids = 0..N-1."""
+    inp = synth.decode_layer(spec)
+    B, N = spec.B, spec.N
+    kv, swa = dev_kv(inp["kv"], batch_rows=N), dev_kv(inp["swa"], batch_rows=spec.swa)
+    q = dev_q(inp["q_attn"], spec.q_dtype)
+    out, lse = L.sparse_attn_decode(q, kv, N, None, None, swa, swa_len, spec.scale, n_dense=N)
+    out, lse = out.cpu().numpy(), lse.cpu().numpy()
+    for b in range(B):
+        ro, rl = oracle.attn(inp["q_attn"][b], inp["kv"].slice(b * N, (b + 1) * N), N,
+                             np.arange(N, dtype=np.int32), swa=inp["swa"].slice(b * spec.swa, (b + 1) * spec.swa),
+                             swa_len=swa_len, scale=spec.scale)
+        assert_attn_close(out[b], ro)
+        np.testing.assert_allclose(lse[b], rl, rtol=1e-5, atol=1e-5)
+
+
+def test_attn_dense_rows_with_n_sel():
+    """Dense rows with a per-sequence count: sequence b reads rows 0..n_b-1."""
+    spec = synth.scaled(synth.DECODE_64K, N=512, k=512, B=3)
+    inp = synth.decode_layer(spec)
+    N = spec.N
+    n_b = [512, 100, 0]
+    kv, swa = dev_kv(inp["kv"], batch_rows=N), dev_kv(inp["swa"], batch_rows=spec.swa)
+    ns = torch.tensor(n_b, dtype=torch.int32, device="cuda")
+    out, lse = L.sparse_attn_decode(dev_q(inp["q_attn"], "bf16"), kv, N, None, ns, swa, 64, spec.scale, n_dense=N)
+    out = out.cpu().numpy()
+    for b in range(3):
+        ro, _ = oracle.attn(inp["q_attn"][b], inp["kv"].slice(b * N, (b + 1) * N), N,
+                            np.arange(n_b[b], dtype=np.int32), swa=inp["swa"].slice(b * spec.swa, (b + 1) * spec.swa),
+                            swa_len=64, scale=spec.scale)
+        assert_attn_close(out[b], ro)
