@@ -313,6 +313,42 @@ LIDX_API lidx_status lidx_sparse_attn_decode_noalloc(const lidx_attn_args *args,
                                                      void *stream);
 
 /* ------------------------------------------------------------------------
+ * lidx_cache_append -- the cache write side: quantise new rows into the
+ * storage format and append them (architecture post, "why quantising the KV
+ * does not save memory", point 1: non-RoPE dims as E4M3 with one
+ * power-of-two scale per 64 elements, RoPE dims as bf16).
+ *
+ *   x      [B][R][dim] fp32, 16-byte aligned: the R new rows of each
+ *          sequence (new compressed entries, or new window rows)
+ *   cache  destination rows (dim 128 or 512; LIDX_F32 | LIDX_BF16 |
+ *          LIDX_E4M3); its planes are WRITTEN.  Sequence b's region is rows
+ *          b*batch_rows .. b*batch_rows + capacity - 1.
+ *   pos    [B] int32 (device): new row r of sequence b goes to row
+ *          pos[b] + r of its region, or to (pos[b] + r) mod ring when ring > 0
+ *          (the sliding window as a ring of `ring` rows)
+ * E4M3: for each 64-element block the scale is 2^e with e the smallest
+ * integer in [-127, 127] such that the block's largest finite magnitude is
+ * <= 448 * 2^e (the finest scale that fits; e = 0 for an all-zero block),
+ * stored as the E8M0 byte e + 127; codes are x / 2^e rounded to the nearest
+ * E4M3FN value, ties to even, magnitudes above 448 saturating; NaN is stored
+ * as 0x7F.  bf16 values (RoPE dims, bf16 caches) round to nearest even.
+ * A destination outside [0, capacity) is skipped and sets LIDX_DEV_BOUNDS;
+ * a non-finite input sets LIDX_DEV_NAN.  Needs
+ * lidx_workspace_size(LIDX_OP_APPEND) bytes (the status word).
+ * ------------------------------------------------------------------------ */
+typedef struct lidx_append_args {
+    int32_t B, R;
+    const float *x;
+    lidx_kv cache;
+    int64_t capacity;
+    const int32_t *pos;
+    int32_t ring;
+    uint32_t flags; /* LIDX_LAUNCH_* */
+} lidx_append_args;
+
+LIDX_API lidx_status lidx_cache_append(const lidx_append_args *args, void *ws, size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------------------
  * lidx_selection_eval -- selection evaluation over a tau-window.
  * `ops` is a bit mask; the requested steps run in this order:
  *
@@ -388,6 +424,7 @@ LIDX_API lidx_status lidx_selection_eval(const lidx_eval_args *args, void *ws, s
 #define LIDX_OP_ATTN 2
 #define LIDX_OP_EVAL 3
 #define LIDX_OP_DECODE 4
+#define LIDX_OP_APPEND 5
 
 /* Bytes of workspace call `op` needs for `args` (a pointer to the matching
  * *_args struct, host memory).  Score needs none (0). */
@@ -404,7 +441,8 @@ LIDX_API const char *lidx_status_string(lidx_status s);
 LIDX_API int lidx_abi_version(void);
 
 /* sizeof() of the argument structs as compiled into the library, for binding
- * checks: which = 0 lidx_kv, 1 score, 2 topk, 3 attn, 4 eval, 5 decode. */
+ * checks: which = 0 lidx_kv, 1 score, 2 topk, 3 attn, 4 eval, 5 decode,
+ * 6 append. */
 LIDX_API size_t lidx_struct_size(int which);
 
 #ifdef __cplusplus

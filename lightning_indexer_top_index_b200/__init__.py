@@ -34,7 +34,7 @@ LAUNCH_TEST_LOST_ARRIVAL = 0x80000000
 STATS_SPAN = 32  # entries per score-bounds record (optional scorer output, top-k input)
 
 EVAL_GOLDEN, EVAL_TOPP, EVAL_VOTE, EVAL_LSA, EVAL_OVERLAP = 0x1, 0x2, 0x4, 0x8, 0x10
-OP_SCORE, OP_TOPK, OP_ATTN, OP_EVAL, OP_DECODE = 0, 1, 2, 3, 4
+OP_SCORE, OP_TOPK, OP_ATTN, OP_EVAL, OP_DECODE, OP_APPEND = 0, 1, 2, 3, 4, 5
 
 # Layer schedule of DeepSeek-V4-Flash (architecture post, section (A) table):
 # layers 0-1 sliding window only, even layers 2..42 CSA (4:1 + top-k), odd
@@ -127,10 +127,15 @@ class DecodeArgs(C.Structure):
                 ("prefetch", C.c_void_p * 2), ("prefetch_bytes", C.c_uint64 * 2), ("flags", C.c_uint32)]
 
 
-_STRUCTS = [KVArgs, ScoreArgs, TopkArgs, AttnArgs, EvalArgs, DecodeArgs]
+class AppendArgs(C.Structure):
+    _fields_ = [("B", C.c_int32), ("R", C.c_int32), ("x", C.c_void_p), ("cache", KVArgs),
+                ("capacity", C.c_int64), ("pos", C.c_void_p), ("ring", C.c_int32), ("flags", C.c_uint32)]
+
+
+_STRUCTS = [KVArgs, ScoreArgs, TopkArgs, AttnArgs, EvalArgs, DecodeArgs, AppendArgs]
 EXPORTS = ("lidx_index_score", "lidx_topk_select", "lidx_sparse_attn_decode", "lidx_selection_eval",
-           "lidx_decode_layer", "lidx_workspace_size", "lidx_read_device_status", "lidx_status_string",
-           "lidx_abi_version", "lidx_struct_size")
+           "lidx_decode_layer", "lidx_cache_append", "lidx_workspace_size", "lidx_read_device_status",
+           "lidx_status_string", "lidx_abi_version", "lidx_struct_size")
 
 _lib = None
 _lock = threading.Lock()
@@ -152,6 +157,7 @@ def lib():
                 ("lidx_sparse_attn_decode", I, [C.POINTER(AttnArgs), P, SZ, P]),
                 ("lidx_selection_eval", I, [C.POINTER(EvalArgs), P, SZ, P]),
                 ("lidx_decode_layer", I, [C.POINTER(DecodeArgs), P, SZ, P]),
+                ("lidx_cache_append", I, [C.POINTER(AppendArgs), P, SZ, P]),
                 ("lidx_workspace_size", I, [I, P, C.POINTER(SZ)]),
                 ("lidx_read_device_status", I, [P, C.POINTER(C.c_uint32), P]),
                 ("lidx_status_string", C.c_char_p, [I]),
@@ -379,6 +385,21 @@ def decode_layer(q_idx: torch.Tensor, w: torch.Tensor, keys: DeviceKV, N: int, k
     _check(lib().lidx_decode_layer(C.byref(a), C.c_void_p(ws.data_ptr()), ws.numel(), _stream(stream)),
            "lidx_decode_layer")
     return out, lse
+
+
+def cache_append(x: torch.Tensor, cache: DeviceKV, pos: torch.Tensor, capacity: int, ring: int = 0, *,
+                 ws=None, stream=None, flags=0):
+    """Quantise the new rows x [B][R][dim] (float32) into `cache`'s format
+    and write row r of sequence b at row pos[b] + r of its region (mod
+    `ring` when ring > 0: the sliding window); see lidx_cache_append."""
+    B, R, dim = x.shape
+    assert x.dtype == torch.float32 and x.is_contiguous() and pos.dtype == torch.int32 and dim == cache.dim
+    a = AppendArgs(B, R, x.data_ptr(), cache.args(), capacity, pos.data_ptr(), ring, flags)
+    if ws is None:
+        ws = workspace(workspace_size(OP_APPEND, a), x.device)
+    _check(lib().lidx_cache_append(C.byref(a), C.c_void_p(ws.data_ptr()), ws.numel(), _stream(stream)),
+           "lidx_cache_append")
+    return ws
 
 
 def selection_eval(ops: int, *, L=1, T=1, H=1, N, qa=None, kv: DeviceKV = None, scale=None, probs=None,

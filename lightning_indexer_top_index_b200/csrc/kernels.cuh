@@ -38,6 +38,9 @@ bool decode_fused_supported(const lidx_decode_args &a);
 size_t decode_fused_workspace(const lidx_decode_args &a);
 cudaError_t launch_decode_fused(const lidx_decode_args &a, void *ws, cudaStream_t st);
 
+// ---- cache write side
+cudaError_t launch_append(const lidx_append_args &a, void *ws, cudaStream_t st);
+
 // ---- selection evaluation
 bool golden_tc_supported(const lidx_eval_args &a);
 size_t golden_tc_workspace(const lidx_eval_args &a);

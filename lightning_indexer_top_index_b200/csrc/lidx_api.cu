@@ -152,6 +152,17 @@ lidx_status check_decode(const lidx_decode_args *a) {
   return LIDX_OK;
 }
 
+lidx_status check_append(const lidx_append_args *a) {
+  if (!a || !a->x || !a->pos) return LIDX_ERR_INVALID_ARG;
+  if (a->B < 1 || a->R < 1 || a->capacity < 1 || a->ring < 0 || a->ring > a->capacity) return LIDX_ERR_INVALID_ARG;
+  if (a->cache.dim != 128 && a->cache.dim != 512) return LIDX_ERR_UNSUPPORTED;
+  lidx_status s = check_kv(a->cache, a->cache.dim, a->B, a->capacity);
+  if (s != LIDX_OK) return s;
+  if (!aligned(a->x, 16) || !aligned(a->pos, 4)) return LIDX_ERR_INVALID_ARG;
+  if (a->cache.dtype == LIDX_E4M3 && (a->cache.ld % 8 != 0)) return LIDX_ERR_INVALID_ARG;
+  return LIDX_OK;
+}
+
 lidx_status check_ws(void *ws, size_t have, size_t need) {
   if (!ws || !aligned(ws, 256)) return need ? LIDX_ERR_WORKSPACE : LIDX_OK;
   return have >= need ? LIDX_OK : LIDX_ERR_WORKSPACE;
@@ -206,6 +217,14 @@ lidx_status lidx_decode_layer(const lidx_decode_args *args, void *ws, size_t ws_
   return from_cuda(launch_decode_fused(*args, ws, static_cast<cudaStream_t>(stream)));
 }
 
+lidx_status lidx_cache_append(const lidx_append_args *args, void *ws, size_t ws_bytes, void *stream) {
+  lidx_status s = check_append(args);
+  if (s != LIDX_OK) return s;
+  if ((s = check_ws(ws, ws_bytes, LIDX_WS_HEADER)) != LIDX_OK) return s;
+  if ((s = check_device()) != LIDX_OK) return s;
+  return from_cuda(launch_append(*args, ws, static_cast<cudaStream_t>(stream)));
+}
+
 lidx_status lidx_workspace_size(int op, const void *args, size_t *bytes) {
   if (!args || !bytes) return LIDX_ERR_INVALID_ARG;
   lidx_status s = LIDX_OK;
@@ -225,6 +244,10 @@ lidx_status lidx_workspace_size(int op, const void *args, size_t *bytes) {
     case LIDX_OP_EVAL:
       s = check_eval(static_cast<const lidx_eval_args *>(args));
       if (s == LIDX_OK) *bytes = eval_workspace(*static_cast<const lidx_eval_args *>(args));
+      break;
+    case LIDX_OP_APPEND:
+      s = check_append(static_cast<const lidx_append_args *>(args));
+      if (s == LIDX_OK) *bytes = LIDX_WS_HEADER;
       break;
     case LIDX_OP_DECODE:
       s = check_decode(static_cast<const lidx_decode_args *>(args));
@@ -266,6 +289,7 @@ size_t lidx_struct_size(int which) {
     case 3: return sizeof(lidx_attn_args);
     case 4: return sizeof(lidx_eval_args);
     case 5: return sizeof(lidx_decode_args);
+    case 6: return sizeof(lidx_append_args);
   }
   return 0;
 }

@@ -58,6 +58,10 @@ def _load():
                 "orc_decode_e4m3": (C.c_double, [C.c_uint8]),
                 "orc_decode_e8m0": (C.c_double, [C.c_uint8]),
                 "orc_decode_rows": (I, [RP, I64, P]),
+                "orc_encode_e4m3": (C.c_uint8, [C.c_double]),
+                "orc_encode_bf16": (C.c_uint16, [C.c_float]),
+                "orc_e8m0_for": (C.c_uint8, [C.c_double]),
+                "orc_encode_rows": (I, [P, I64, I, I, P, P, P, P]),
                 "orc_index_score": (I, [I, I, I, I, RP, P, RP, I64, P, I64, P, P]),
                 "orc_topk": (I, [I, I, P, P, P, P, P]),
                 "orc_attn": (I, [I, RP, RP, I, P, I, RP, I, D, P, P]),
@@ -128,6 +132,46 @@ def decode_rows(kv) -> np.ndarray:
     n = keep[0].shape[0]
     out = np.empty((n, r.dim), dtype=np.float64)
     _check(_load().orc_decode_rows(C.byref(r), n, _ptr(out)))
+    return out
+
+
+# ------------------------------------------------------------- the write side
+def encode_e4m3(v: float) -> int:
+    return int(_load().orc_encode_e4m3(float(v)))
+
+
+def encode_bf16(x: float) -> int:
+    return int(_load().orc_encode_bf16(float(x)))
+
+
+def e8m0_for(amax: float) -> int:
+    return int(_load().orc_e8m0_for(float(amax)))
+
+
+def encode_rows(x, dtype: str) -> dict:
+    """Encode fp32 rows x [rows][dim] for storage (see orc_encode_rows).
+    Returns the packed planes: {"data": codes / bf16 bits / fp32,
+    "scale": E8M0 codes (e4m3), "rope": bf16 bits (e4m3), "finite": bool}."""
+    x = np.ascontiguousarray(np.asarray(x, dtype=np.float32))
+    rows, dim = x.shape
+    dt = _DT[dtype]
+    out = {"scale": None, "rope": None}
+    f32 = bits = codes = scales = None
+    if dt == F32:
+        f32 = np.empty((rows, dim), np.float32)
+        out["data"] = f32
+    elif dt == BF16:
+        bits = np.empty((rows, dim), np.uint16)
+        out["data"] = bits
+    else:
+        codes = np.empty((rows, dim - 64), np.uint8)
+        scales = np.empty((rows, (dim - 64) // 64), np.uint8)
+        bits = np.empty((rows, 64), np.uint16)
+        out.update(data=codes, scale=scales, rope=bits)
+    rc = _load().orc_encode_rows(_ptr(x), rows, dim, dt, _ptr(f32), _ptr(bits), _ptr(codes), _ptr(scales))
+    if rc not in (0, 2):
+        _check(rc)
+    out["finite"] = rc == 0
     return out
 
 

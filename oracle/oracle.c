@@ -29,6 +29,9 @@
  *  - orc_lsa_gate      sigmoid(logit) >= 0.5 <=> logit >= 0, OR over the
  *        gate layers (write-up sections 2.2 and 4.1)
  *  - orc_overlap       |A & B|, |A|, |B| (FlashMemory vs native post, Act 1/3)
+ *  - orc_encode_rows   the cache write side: rows stored as E4M3 + per-64
+ *        power-of-two scales + bf16 RoPE dims, or bf16 / fp32 (architecture
+ *        post, "why quantising the KV does not save memory")
  *
  * Storage decoding (architecture post, "why you cannot quantise the KV"):
  * non-RoPE dims are OCP E4M3FN bytes, one E8M0 power-of-two scale per 64
@@ -129,6 +132,121 @@ int orc_decode_rows(const orc_rows *r, int64_t n, double *out)
 {
     for (int64_t i = 0; i < n; i++) decode_row(r, i, out + i * r->dim);
     return ORC_OK;
+}
+
+/* ---------------------------------------------------------------- encoding
+ *
+ * The cache write side (architecture post, "why quantising the KV does not
+ * save memory", point 1): the non-RoPE dims of a row are stored as OCP
+ * E4M3FN codes with one power-of-two (E8M0) scale per 64 elements, the 64
+ * RoPE dims as bf16.  The page fixes the format, not how the scale is chosen;
+ * the reading taken here is the finest scale that still fits the block: the
+ * smallest integer e with amax <= 448 * 2^e (448 is the largest E4M3FN
+ * value), clamped to [-127, 127], stored as the byte e + 127; a block whose
+ * finite values are all zero takes e = 0.  Values are divided by 2^e and
+ * rounded to the nearest E4M3 value, ties to the even code; magnitudes
+ * above 448 saturate to 448 (infinities included); NaN is stored as the
+ * code 0x7F.  RoPE dims and bf16 rows round to nearest even from the fp32
+ * input.
+ */
+
+/* nearest E4M3FN code of v (ties to even); |v| > 448 saturates */
+static uint8_t e4m3_encode(double v)
+{
+    if (isnan(v)) return 0x7F;
+    uint8_t sign = signbit(v) ? 0x80 : 0x00;
+    double a = fabs(v);
+    if (a >= 448.0) return sign | 0x7E;
+    int ex;
+    (void)frexp(a, &ex); /* a = f * 2^ex, f in [0.5, 1): floor(log2 a) = ex - 1 */
+    int e = ex - 1;
+    double q; /* the value on the integer grid of its binade */
+    int E;
+    if (a == 0.0 || e < -6) { /* subnormal: m * 2^-9, m = 0..7 (8 rounds up to the smallest normal) */
+        q = ldexp(a, 9);
+        E = 0;
+    } else {                  /* normal: 2^e * (1 + m/8): q = 8 + m in [8, 16) */
+        q = ldexp(a, 3 - e);
+        E = e + 7;
+    }
+    double fl = floor(q);
+    double rem = q - fl;
+    long n = (long)fl;
+    if (rem > 0.5 || (rem == 0.5 && (n & 1))) n++;
+    int code;
+    if (E == 0) {
+        code = (int)n;                  /* n = 8 is exponent field 1, mantissa 0 */
+    } else {
+        if (n == 16) { n = 8; E++; }    /* carry into the next binade */
+        code = (E << 3) | (int)(n - 8);
+    }
+    if (code > 0x7E) code = 0x7E;       /* 0x7F is NaN: the rounding saturates */
+    return (uint8_t)(sign | code);
+}
+
+/* nearest bf16 of a float (ties to even); NaN stays a quiet NaN */
+static uint16_t bf16_encode(float x)
+{
+    uint32_t u;
+    memcpy(&u, &x, 4);
+    if ((u & 0x7F800000u) == 0x7F800000u && (u & 0x007FFFFFu)) return (uint16_t)((u >> 16) | 0x0040u);
+    uint32_t lower = u & 0xFFFFu, upper = u >> 16;
+    if (lower > 0x8000u || (lower == 0x8000u && (upper & 1u))) upper++;
+    return (uint16_t)upper;
+}
+
+/* E8M0 code of the block scale for largest finite magnitude amax */
+static uint8_t e8m0_for(double amax)
+{
+    if (amax == 0.0) return 127;
+    int e = -127;
+    while (e < 127 && amax > ldexp(448.0, e)) e++;
+    return (uint8_t)(e + 127);
+}
+
+uint8_t orc_encode_e4m3(double v) { return e4m3_encode(v); }
+uint16_t orc_encode_bf16(float x) { return bf16_encode(x); }
+uint8_t orc_e8m0_for(double amax) { return e8m0_for(amax); }
+
+/*
+ * Encode `rows` rows of `dim` fp32 values x[rows][dim] in format `dtype`
+ * into packed planes:
+ *   F32:  f32[rows][dim] (copied)
+ *   BF16: bits[rows][dim]
+ *   E4M3: codes[rows][dim-64], scales[rows][(dim-64)/64], bits[rows][64] (RoPE)
+ * Returns ORC_ENAN (after encoding every row) when an input was not finite.
+ */
+int orc_encode_rows(const float *x, int64_t rows, int dim, int dtype, float *f32, uint16_t *bits,
+                    uint8_t *codes, uint8_t *scales)
+{
+    if (rows < 0 || dim < 64 || dim % 64) return ORC_EINVAL;
+    int nonfinite = 0;
+    for (int64_t r = 0; r < rows; r++) {
+        const float *xr = x + r * dim;
+        for (int d = 0; d < dim; d++) nonfinite |= !isfinite(xr[d]);
+        if (dtype == ORC_F32) {
+            memcpy(f32 + r * dim, xr, sizeof(float) * (size_t)dim);
+        } else if (dtype == ORC_BF16) {
+            for (int d = 0; d < dim; d++) bits[r * dim + d] = bf16_encode(xr[d]);
+        } else if (dtype == ORC_E4M3) {
+            int nope = dim - 64, nb = nope / 64;
+            for (int blk = 0; blk < nb; blk++) {
+                double amax = 0.0;
+                for (int d = 64 * blk; d < 64 * blk + 64; d++) {
+                    double a = fabs((double)xr[d]);
+                    if (isfinite(a) && a > amax) amax = a;
+                }
+                uint8_t sc = e8m0_for(amax);
+                scales[r * nb + blk] = sc;
+                for (int d = 64 * blk; d < 64 * blk + 64; d++)
+                    codes[r * nope + d] = e4m3_encode(ldexp((double)xr[d], 127 - (int)sc));
+            }
+            for (int d = 0; d < 64; d++) bits[r * 64 + d] = bf16_encode(xr[nope + d]);
+        } else {
+            return ORC_EINVAL;
+        }
+    }
+    return nonfinite ? ORC_ENAN : ORC_OK;
 }
 
 /* ------------------------------------------------------------- index score */

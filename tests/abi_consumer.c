@@ -8,8 +8,9 @@
 #include "lidx.h"
 
 int main(void) {
-  const size_t sizes[6] = {sizeof(lidx_kv), sizeof(lidx_score_args), sizeof(lidx_topk_args),
-                           sizeof(lidx_attn_args), sizeof(lidx_eval_args), sizeof(lidx_decode_args)};
+  const size_t sizes[7] = {sizeof(lidx_kv), sizeof(lidx_score_args), sizeof(lidx_topk_args),
+                           sizeof(lidx_attn_args), sizeof(lidx_eval_args), sizeof(lidx_decode_args),
+                           sizeof(lidx_append_args)};
   int bad = 0;
   int i;
   lidx_topk_args t;
@@ -21,7 +22,7 @@ int main(void) {
     printf("abi version %d, header %d\n", lidx_abi_version(), LIDX_ABI_VERSION);
     bad = 1;
   }
-  for (i = 0; i < 6; i++) {
+  for (i = 0; i < 7; i++) {
     if (lidx_struct_size(i) != sizes[i]) {
       printf("struct %d: library %zu, header %zu\n", i, lidx_struct_size(i), sizes[i]);
       bad = 1;

@@ -435,3 +435,93 @@ def test_overlap_random_baseline_matches_page():
     # the Act 1 random baseline 57.6% corresponds to N = 512 / 0.576 ~ 889 chunks
     n_act1 = 512 / _load("page_facts.json")["random_overlap_act1"]["value"]
     assert 880 < n_act1 < 900
+
+
+# ------------------------------------------------------------ the write side
+# The storage format is the architecture post's ("why quantising the KV does
+# not save memory", point 1); E4M3 is the OCP E4M3FN format it names: bias 7,
+# 3 mantissa bits, no infinities, S.1111.111 NaN, largest value 448.
+def test_e4m3_encode_round_trips_every_code():
+    for c in range(256):
+        if c & 0x7F == 0x7F:
+            continue  # the two NaN codes
+        assert oracle.encode_e4m3(oracle.decode_e4m3(c)) == c, hex(c)
+
+
+def test_e4m3_encode_ties_to_even_and_rounds_to_nearest():
+    """Between two adjacent codes the midpoint goes to the even code (mantissa
+    LSB 0, which is the code's LSB), anything off the midpoint to the nearer."""
+    for c in range(0x7E):
+        lo, hi = oracle.decode_e4m3(c), oracle.decode_e4m3(c + 1)
+        mid = (lo + hi) / 2
+        assert oracle.encode_e4m3(mid) == (c if c % 2 == 0 else c + 1), hex(c)
+        assert oracle.encode_e4m3(mid - (hi - lo) * 1e-3) == c
+        assert oracle.encode_e4m3(mid + (hi - lo) * 1e-3) == c + 1
+        assert oracle.encode_e4m3(-mid) == 0x80 | (c if c % 2 == 0 else c + 1)
+
+
+@pytest.mark.parametrize("v,code", [(448.0, 0x7E), (464.0, 0x7E), (1e9, 0x7E), (float("inf"), 0x7E),
+                                    (-float("inf"), 0xFE), (float("nan"), 0x7F), (2.0 ** -6, 0x08),
+                                    (7 * 2.0 ** -9, 0x07), (2.0 ** -9, 0x01), (2.0 ** -10, 0x00),
+                                    (-0.0, 0x80), (1.0, 0x38), (-1.75, 0xBE)])
+def test_e4m3_encode_code_points(v, code):
+    """OCP E4M3FN code points: 448 = 0x7E is the largest value and larger
+    magnitudes saturate to it; 2^-6 = 0x08 is the smallest normal, 2^-9 = 0x01
+    the smallest subnormal."""
+    assert oracle.encode_e4m3(v) == code
+
+
+def test_e4m3_encode_matches_torch_float8():
+    """A library routine for in-range values: torch's float8_e4m3fn cast
+    (round to nearest even)."""
+    g = np.random.default_rng(40)
+    v = np.concatenate([g.standard_normal(4000) * 100, g.standard_normal(2000) * 2.0 ** -7,
+                        g.uniform(-448, 448, 2000)]).astype(np.float32)
+    ref = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([oracle.encode_e4m3(float(x)) for x in v], dtype=np.uint8)
+    inr = np.abs(v) <= 448
+    assert np.array_equal(got[inr], ref[inr])
+
+
+def test_block_scale_is_the_finest_that_fits():
+    """The stored scale 2^e is the smallest power of two with amax <= 448 * 2^e
+    (an all-zero block takes e = 0)."""
+    for amax, code in [(448.0, 127), (449.0, 128), (224.0, 126), (224.0001, 127), (0.0, 127), (1.0, 119)]:
+        assert oracle.e8m0_for(amax) == code, amax
+    g = np.random.default_rng(41)
+    for a in np.exp(g.uniform(-80, 80, 500)):
+        e = oracle.e8m0_for(a) - 127
+        assert a <= 448 * 2.0 ** e and a > 448 * 2.0 ** (e - 1)
+
+
+def test_bf16_encode_ties_to_even_and_matches_torch():
+    assert oracle.encode_bf16(1.0 + 2.0 ** -8) == 0x3F80      # midpoint of 1.0 and 1+2^-7: even
+    assert oracle.encode_bf16(1.0 + 3 * 2.0 ** -8) == 0x3F82  # midpoint of 1+2^-7 and 1+2^-6: even
+    assert oracle.encode_bf16(float(np.float32(3.0e38))) == 0x7F62  # 0x7F61B1E6 rounds up
+    assert oracle.encode_bf16(float(np.float32(3.4e38))) == 0x7F80  # past the largest bf16: inf
+    g = np.random.default_rng(42)
+    v = (g.standard_normal(5000) * np.exp(g.uniform(-30, 30, 5000))).astype(np.float32)
+    ref = torch.from_numpy(v).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got = np.array([oracle.encode_bf16(float(x)) for x in v], dtype=np.uint16)
+    assert np.array_equal(got, ref)
+
+
+@pytest.mark.parametrize("dim", [128, 512])
+def test_encode_rows_decodes_within_half_a_step(dim):
+    """Decoding an encoded row returns each value within half an E4M3 step
+    of its binade times the block scale; each block's largest magnitude lands
+    in (224, 448] after scaling; RoPE dims within bf16 rounding."""
+    g = np.random.default_rng(43)
+    x = (g.standard_normal((6, dim)) * np.exp(g.uniform(-20, 20, (6, dim // 64)).repeat(64, axis=1))).astype(
+        np.float32)
+    enc = oracle.encode_rows(x, "e4m3")
+    assert enc["finite"]
+    kv = synth.KV("e4m3", dim, enc["data"], enc["scale"], enc["rope"])
+    dec = oracle.decode_rows(kv)
+    nope = dim - 64
+    sc = np.exp2(enc["scale"].astype(np.float64) - 127).repeat(64, axis=1)
+    xs = np.abs(x[:, :nope]).astype(np.float64)
+    assert np.all(np.abs(dec[:, :nope] - x[:, :nope]) <= 2.0 ** -4 * xs + 2.0 ** -10 * sc)
+    amax = xs.reshape(6, -1, 64).max(axis=2) / sc[:, ::64]
+    assert np.all((amax > 224) & (amax <= 448))
+    assert np.all(np.abs(dec[:, nope:] - x[:, nope:]) <= 2.0 ** -8 * np.abs(x[:, nope:]))
