@@ -120,6 +120,11 @@ typedef struct lidx_kv {
  *   tile_stats  optional [B][Q][ceil(N/LIDX_STATS_SPAN)][2] uint32, 8-byte
  *           aligned: the score bounds lidx_topk_select can start from (see
  *           LIDX_STATS_SPAN)
+ *   n_visible optional [B][Q] int32: causal entry mask for prefill, where the
+ *           queries sit at different positions: entry j is visible to query
+ *           (b,t) only when j < n_visible[b][t] (the compressed entries formed
+ *           before its token); the scores of the others are written as -inf.
+ *           Pass the same counts as n_valid to lidx_topk_select.
  * Returns INVALID_ARG for null pointers / non-positive sizes / misaligned
  * planes, UNSUPPORTED for other format combinations.
  * ------------------------------------------------------------------------ */
@@ -143,6 +148,7 @@ typedef struct lidx_score_args {
     int64_t ld_scores;
     uint32_t flags;       /* LIDX_LAUNCH_* */
     uint32_t *tile_stats; /* optional score bounds, see LIDX_STATS_SPAN */
+    const int32_t *n_visible; /* optional causal entry mask, [B][Q] */
 } lidx_score_args;
 
 LIDX_API lidx_status lidx_index_score(const lidx_score_args *args, void *stream);
@@ -165,6 +171,9 @@ LIDX_API lidx_status lidx_index_score(const lidx_score_args *args, void *stream)
  *   n_sel   [B][Q] int32 (optional): min(k, #eligible)
  *   mask    [B][Q][N] uint8 (optional): 1 for selected entries (comp_allowed)
  *   mask_bits [B][Q][ceil(N/32)] uint32 (optional): bit j%32 of word j/32
+ *   n_valid [B][Q] int32 (optional): only entries j < n_valid[b][t] are
+ *           eligible (the causal prefix of a prefill query; see n_visible of
+ *           lidx_index_score)
  *   tile_stats optional: the score bounds lidx_index_score wrote for exactly
  *           these scores (LIDX_STATS_SPAN).  Bounds that do not hold give
  *           wrong ids but never a write outside ids[b][t][0..k).
@@ -184,6 +193,7 @@ typedef struct lidx_topk_args {
     const uint32_t *tile_stats; /* optional score bounds, see LIDX_STATS_SPAN */
     const uint32_t *allowed_bits; /* optional [B][ld_allowed_bits] bit set, shared by the Q queries */
     int64_t ld_allowed_bits;      /* words between sequences, >= ceil(N/32) */
+    const int32_t *n_valid;       /* optional per-row eligible prefix, [B][Q] */
 } lidx_topk_args;
 
 LIDX_API lidx_status lidx_topk_select(const lidx_topk_args *args, void *ws, size_t ws_bytes, void *stream);
@@ -205,6 +215,12 @@ LIDX_API lidx_status lidx_topk_select(const lidx_topk_args *args, void *ws, size
  *   kv    comp_kv rows, dim 512, N entries per sequence
  *   ids   [B][ld_ids] int32 (ascending not required; duplicates count twice),
  *         or NULL for the dense rows 0..n_b-1
+ * The rows of the B queries may overlap: kv.batch_rows and swa.batch_rows
+ * may be smaller than the rows one query reads (0: every query reads the
+ * same rows).  So the T queries of a prefill attend through one call: B = T,
+ * kv.batch_rows = 0 (one shared compressed cache, each query with its own
+ * ids), swa rows of query t starting at row t of the raw-token window buffer
+ * (swa.batch_rows = 1).
  *   swa   sliding-window rows, dim 512, same dtype as kv (swa_len may be 0)
  *   out   [B][H][512] fp32
  * Ids outside [-1, N) are skipped and set LIDX_DEV_BOUNDS.  Empty R gives

@@ -89,7 +89,8 @@ class KVArgs(C.Structure):
 class ScoreArgs(C.Structure):
     _fields_ = [("B", C.c_int32), ("Q", C.c_int32), ("H", C.c_int32), ("N", C.c_int32),
                 ("q_dtype", C.c_int32), ("q", C.c_void_p), ("w", C.c_void_p), ("keys", KVArgs),
-                ("scores", C.c_void_p), ("ld_scores", C.c_int64), ("flags", C.c_uint32), ("tile_stats", C.c_void_p)]
+                ("scores", C.c_void_p), ("ld_scores", C.c_int64), ("flags", C.c_uint32), ("tile_stats", C.c_void_p),
+                ("n_visible", C.c_void_p)]
 
 
 class TopkArgs(C.Structure):
@@ -97,7 +98,7 @@ class TopkArgs(C.Structure):
                 ("scores", C.c_void_p), ("ld_scores", C.c_int64), ("allowed", C.c_void_p),
                 ("ld_allowed", C.c_int64), ("ids", C.c_void_p), ("n_sel", C.c_void_p), ("mask", C.c_void_p),
                 ("mask_bits", C.c_void_p), ("flags", C.c_uint32), ("tile_stats", C.c_void_p),
-                ("allowed_bits", C.c_void_p), ("ld_allowed_bits", C.c_int64)]
+                ("allowed_bits", C.c_void_p), ("ld_allowed_bits", C.c_int64), ("n_valid", C.c_void_p)]
 
 
 class AttnArgs(C.Structure):
@@ -251,19 +252,21 @@ def _qdtype(t: torch.Tensor) -> int:
 
 # ---------------------------------------------------------------- the calls
 def index_score(q: torch.Tensor, w: torch.Tensor, keys: DeviceKV, N: int, scores: torch.Tensor = None,
-                stream=None, tile_stats: torch.Tensor = None) -> torch.Tensor:
+                stream=None, tile_stats: torch.Tensor = None, n_visible: torch.Tensor = None) -> torch.Tensor:
     """scores[b,t,j] = sum_h w[b,t,h] * max(q[b,t,h] . keys[b,j], 0).
 
     q [B][Q][H][128] (float32 or bfloat16), w [B][Q][H] float32 -> scores
     float32 [B][Q][N] (or the given tensor with a row stride >= N).  With
     `tile_stats` (int32 [B][Q][ceil(N/STATS_SPAN)][2]) the call also writes
-    the score bounds topk_select can start from."""
+    the score bounds topk_select can start from.  `n_visible` (int32 [B][Q])
+    is the causal entry mask of prefill queries: entries j >= n_visible[b][t]
+    score -inf."""
     B, Q, H, D = q.shape
     assert q.is_contiguous() and w.is_contiguous() and w.dtype == torch.float32
     if scores is None:
         scores = torch.empty((B, Q, N), dtype=torch.float32, device=q.device)
     a = ScoreArgs(B, Q, H, N, _qdtype(q), q.data_ptr(), w.data_ptr(), keys.args(), scores.data_ptr(),
-                  scores.stride(1), 0, _ptr(tile_stats))
+                  scores.stride(1), 0, _ptr(tile_stats), _ptr(n_visible))
     _check(lib().lidx_index_score(C.byref(a), _stream(stream)), "lidx_index_score")
     return scores
 
@@ -280,24 +283,26 @@ def workspace(nbytes: int, device="cuda") -> torch.Tensor:
 
 
 def topk_args(scores, k, allowed=None, ids=None, n_sel=None, mask=None, mask_bits=None, flags=0,
-              tile_stats=None, allowed_bits=None) -> TopkArgs:
+              tile_stats=None, allowed_bits=None, n_valid=None) -> TopkArgs:
     B, Q, N = scores.shape[0], scores.shape[1], scores.shape[2]
     ldb = 0 if allowed_bits is None else (allowed_bits.stride(0) if allowed_bits.dim() > 1 else (N + 31) // 32)
     return TopkArgs(B, Q, N, k, scores.data_ptr(), scores.stride(1), _ptr(allowed),
                     0 if allowed is None else allowed.stride(0), _ptr(ids), _ptr(n_sel), _ptr(mask),
-                    _ptr(mask_bits), flags, _ptr(tile_stats), _ptr(allowed_bits), ldb)
+                    _ptr(mask_bits), flags, _ptr(tile_stats), _ptr(allowed_bits), ldb, _ptr(n_valid))
 
 
 def topk_select(scores: torch.Tensor, k: int, allowed: torch.Tensor = None, *, want_mask=False,
                 want_bits=False, ids=None, n_sel=None, ws=None, stream=None, tile_stats=None, bits=None,
-                allowed_bits: torch.Tensor = None):
+                allowed_bits: torch.Tensor = None, n_valid: torch.Tensor = None):
     """Top-k row ids of scores [B][Q][N] (N = scores.shape[2]).
 
     Returns (ids int32 [B][Q][k] ascending with -1 padding, n_sel int32 [B][Q],
     mask uint8 [B][Q][N] or None, bits uint32 [B][Q][ceil(N/32)] or None).
     `tile_stats` are the score bounds index_score wrote for these scores.
     `allowed` (uint8 [B][N]) and `allowed_bits` (int32 [B][ceil(N/32)], e.g.
-    the gate's fetched set) restrict the eligible entries."""
+    the gate's fetched set) restrict the eligible entries, and so does
+    `n_valid` (int32 [B][Q]: only entries j < n_valid[b][t], the causal
+    prefix of a prefill query)."""
     B, Q, N = scores.shape
     dev = scores.device
     ids = torch.empty((B, Q, k), dtype=torch.int32, device=dev) if ids is None else ids
@@ -305,7 +310,8 @@ def topk_select(scores: torch.Tensor, k: int, allowed: torch.Tensor = None, *, w
     mask = torch.empty((B, Q, N), dtype=torch.uint8, device=dev) if want_mask else None
     if bits is None and want_bits:
         bits = torch.empty((B, Q, (N + 31) // 32), dtype=torch.int32, device=dev)
-    a = topk_args(scores, k, allowed, ids, n_sel, mask, bits, tile_stats=tile_stats, allowed_bits=allowed_bits)
+    a = topk_args(scores, k, allowed, ids, n_sel, mask, bits, tile_stats=tile_stats, allowed_bits=allowed_bits,
+                  n_valid=n_valid)
     if ws is None:
         ws = workspace(workspace_size(OP_TOPK, a), dev)
     _check(lib().lidx_topk_select(C.byref(a), C.c_void_p(ws.data_ptr()), ws.numel(), _stream(stream)),

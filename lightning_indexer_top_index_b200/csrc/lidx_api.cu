@@ -37,7 +37,7 @@ size_t elem_size(int dt) { return dt == LIDX_F32 ? 4 : dt == LIDX_BF16 ? 2 : 1; 
 
 // Layout checks of a row set; `rows_per_batch` is the largest row index used + 1
 // within one batch entry.
-lidx_status check_kv(const lidx_kv &k, int dim, int B, int64_t rows_per_batch) {
+lidx_status check_kv(const lidx_kv &k, int dim, int B, int64_t rows_per_batch, bool overlap_ok = false) {
   if (k.dtype == LIDX_F16) return LIDX_ERR_UNSUPPORTED;
   if (k.dtype != LIDX_F32 && k.dtype != LIDX_BF16 && k.dtype != LIDX_E4M3) return LIDX_ERR_INVALID_ARG;
   if (k.dim != dim) return LIDX_ERR_UNSUPPORTED;
@@ -50,7 +50,7 @@ lidx_status check_kv(const lidx_kv &k, int dim, int B, int64_t rows_per_batch) {
     if (k.ld_scale < (dim - 64) / 64 || k.ld_rope < 64) return LIDX_ERR_INVALID_ARG;
     if (!aligned(k.rope, 16) || (k.ld_rope * 2) % 16 != 0) return LIDX_ERR_INVALID_ARG;
   }
-  if (B > 1 && k.batch_rows < rows_per_batch) return LIDX_ERR_INVALID_ARG;
+  if (B > 1 && (overlap_ok ? k.batch_rows < 0 : k.batch_rows < rows_per_batch)) return LIDX_ERR_INVALID_ARG;
   return LIDX_OK;
 }
 
@@ -65,6 +65,7 @@ lidx_status check_score(const lidx_score_args *a) {
   if (a->keys.dtype != LIDX_F32 && a->q_dtype != LIDX_BF16) return LIDX_ERR_UNSUPPORTED;
   if (!aligned(a->q, 4) || !aligned(a->w, 4) || !aligned(a->scores, 4)) return LIDX_ERR_INVALID_ARG;
   if (a->tile_stats && !aligned(a->tile_stats, 8)) return LIDX_ERR_INVALID_ARG;
+  if (a->n_visible && !aligned(a->n_visible, 4)) return LIDX_ERR_INVALID_ARG;
   return LIDX_OK;
 }
 
@@ -77,6 +78,7 @@ lidx_status check_topk(const lidx_topk_args *a) {
   if (!aligned(a->scores, 4) || !aligned(a->ids, 4) || (a->mask_bits && !aligned(a->mask_bits, 4)))
     return LIDX_ERR_INVALID_ARG;
   if (a->tile_stats && !aligned(a->tile_stats, 8)) return LIDX_ERR_INVALID_ARG;
+  if (a->n_valid && !aligned(a->n_valid, 4)) return LIDX_ERR_INVALID_ARG;
   if (!topk_supported(*a)) return LIDX_ERR_UNSUPPORTED;
   return LIDX_OK;
 }
@@ -89,13 +91,13 @@ lidx_status check_attn(const lidx_attn_args *a) {
   if (a->n_ids > a->N && !a->ids) return LIDX_ERR_INVALID_ARG;  // dense rows 0..n_ids-1 must exist
   if (!(a->scale == a->scale) || a->scale == INFINITY || a->scale == -INFINITY) return LIDX_ERR_INVALID_ARG;
   if (a->n_ids > 0) {
-    lidx_status s = check_kv(a->kv, 512, a->B, a->N);
+    lidx_status s = check_kv(a->kv, 512, a->B, a->N, true);
     if (s != LIDX_OK) return s;
   } else if (a->kv.dtype == LIDX_F16) {
     return LIDX_ERR_UNSUPPORTED;
   }
   if (a->swa_len > 0) {
-    lidx_status s = check_kv(a->swa, 512, a->B, a->swa_len);
+    lidx_status s = check_kv(a->swa, 512, a->B, a->swa_len, true);
     if (s != LIDX_OK) return s;
     if (a->n_ids > 0 && a->swa.dtype != a->kv.dtype) return LIDX_ERR_UNSUPPORTED;
   }

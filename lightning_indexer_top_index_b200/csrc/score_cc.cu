@@ -98,6 +98,7 @@ __global__ void __launch_bounds__(kThreads) score_cc_kernel(lidx_score_args a, i
 #pragma unroll
       for (int hh = 0; hh < HG; hh++) score = fmaf(w_s[h0 + hh], fmaxf(acc[hh], 0.f), score);
     }
+    if (a.n_visible && j >= __ldg(a.n_visible + bt)) score = -INFINITY;  // causal entry mask
     a.scores[static_cast<size_t>(bt) * a.ld_scores + j] = score;
   }
   if (a.tile_stats) {  // score bounds of this warp's span of 32 entries (whole warps)

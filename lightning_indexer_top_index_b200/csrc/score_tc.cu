@@ -57,6 +57,7 @@ struct TcParams {
   int64_t ld_scale;
   uint32_t *stats;    // optional score bounds per span of 32 entries
   int n_spans;
+  const int32_t *n_visible;  // optional causal entry mask [B][Q]
   uint32_t *status;
 };
 
@@ -338,6 +339,7 @@ __global__ void __launch_bounds__(kFp8 ? 32 * kConvWarp0 + 128 : 32 * kConvWarp0
 #pragma unroll
             for (int i = 0; i < 32; i++) s = fmaf(gW[c0 + i], fmaxf(fmaf(sc, v[i], r[i]), 0.f), s);
           }
+          if (p.n_visible && j >= __ldg(p.n_visible + b * p.Q + g)) s = -INFINITY;
           if (j < p.N) p.scores[static_cast<int64_t>(b * p.Q + g) * p.ld_scores + j] = s;
           if (p.stats) span_stats(s, j < p.N, b * p.Q + g, t);
         } else {
@@ -361,6 +363,7 @@ __global__ void __launch_bounds__(kFp8 ? 32 * kConvWarp0 + 128 : 32 * kConvWarp0
             s += (s4[0] + s4[1]) + (s4[2] + s4[3]);
             if (((c + 1) << 5) % p.H == 0) {  // last chunk of query qi
               const int qq = g * p.QG + ((c << 5) / p.H);
+              if (p.n_visible && qq < p.Q && j >= __ldg(p.n_visible + b * p.Q + qq)) s = -INFINITY;
               if (j < p.N && qq < p.Q) p.scores[static_cast<int64_t>(b * p.Q + qq) * p.ld_scores + j] = s;
               if (p.stats && qq < p.Q) span_stats(s, j < p.N, b * p.Q + qq, t);
               s = 0.f;
@@ -481,6 +484,7 @@ cudaError_t launch_score_tc(const lidx_score_args &a, cudaStream_t st) {
   p.ld_scale = a.keys.ld_scale;
   p.stats = a.tile_stats;
   p.n_spans = (a.N + LIDX_STATS_SPAN - 1) / LIDX_STATS_SPAN;
+  p.n_visible = a.n_visible;
   p.status = nullptr;
 
   const uint64_t rows = static_cast<uint64_t>(a.B - 1) * p.key_batch_rows + a.N;

@@ -303,6 +303,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelParams p) 
   const float *s = a.scores + static_cast<size_t>(row) * a.ld_scores + s0;
   const uint8_t *al = a.allowed ? a.allowed + static_cast<size_t>(row / a.Q) * a.ld_allowed + s0 : nullptr;
   const uint32_t *alb = a.allowed_bits ? a.allowed_bits + static_cast<size_t>(row / a.Q) * a.ld_allowed_bits : nullptr;
+  const int n_valid = a.n_valid ? __ldg(a.n_valid + row) : a.N;  // eligible prefix of this row
   float val[C];
   {
     const int head = len > 0 ? static_cast<int>(((16u - (reinterpret_cast<uintptr_t>(s) & 15u)) & 15u) / 4u) : 0;
@@ -360,7 +361,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelParams p) 
     const int pos = p0 + i;
     const bool in = pos < len;
     const int j = s0 + pos;
-    const bool ok = in && !(al && !al[pos]) && !(alb && !((__ldg(alb + (j >> 5)) >> (j & 31)) & 1u));
+    const bool ok = in && j < n_valid && !(al && !al[pos]) && !(alb && !((__ldg(alb + (j >> 5)) >> (j & 31)) & 1u));
     uint32_t kk = in ? order_key(val[i]) : 0u;
     nanf |= (ok && kk == 0u) ? 1u : 0u;
     kk = ok ? kk : 0u;
