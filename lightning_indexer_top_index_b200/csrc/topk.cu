@@ -262,7 +262,9 @@ __device__ __forceinline__ void sum_pushed_hist(SelSmem &sm, uint32_t G, int nbi
 struct SelParams {
   lidx_topk_args a;
   uint32_t *status;
-  int slice;  // positions per CTA (C * kThreads)
+  int slice;    // positions per CTA (C * kThreads)
+  int n_seg;    // segments per row: grid row y is segment y % n_seg of row y / n_seg
+  int seg_len;  // positions per segment (a.N when n_seg == 1)
 };
 
 template <int C>
@@ -275,7 +277,10 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelParams p) 
   const int hg = (tid >> 5) & 7;
   const uint32_t G = gridDim.x;  // the cluster spans the x dimension
   const uint32_t rank = cluster_rank();
-  const int row = blockIdx.y;
+  const int grow = blockIdx.y;                       // this CTA's row of the grid
+  const int row = grow / p.n_seg;                    // the caller's row (b, t)
+  const int seg0 = (grow % p.n_seg) * p.seg_len;     // first position of its segment in that row
+  const int Nr = min(p.seg_len, a.N - seg0);         // positions of the segment
   const int k = a.k;
   const int s0 = static_cast<int>(rank) * p.slice;  // first position of this CTA's slice
   const int p0 = tid * C;                           // first position of this thread, within the slice
@@ -299,9 +304,9 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelParams p) 
 
   // ---- 0. this CTA's slice: one bulk copy into shared memory, then thread t
   // takes positions [t*C, t*C + C) of the slice into registers
-  const int len = max(0, min(p.slice, a.N - s0));
-  const float *s = a.scores + static_cast<size_t>(row) * a.ld_scores + s0;
-  const uint8_t *al = a.allowed ? a.allowed + static_cast<size_t>(row / a.Q) * a.ld_allowed + s0 : nullptr;
+  const int len = max(0, min(p.slice, Nr - s0));
+  const float *s = a.scores + static_cast<size_t>(row) * a.ld_scores + seg0 + s0;
+  const uint8_t *al = a.allowed ? a.allowed + static_cast<size_t>(row / a.Q) * a.ld_allowed + seg0 + s0 : nullptr;
   const uint32_t *alb = a.allowed_bits ? a.allowed_bits + static_cast<size_t>(row / a.Q) * a.ld_allowed_bits : nullptr;
   const int n_valid = a.n_valid ? __ldg(a.n_valid + row) : a.N;  // eligible prefix of this row
   float val[C];
@@ -360,7 +365,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelParams p) 
   for (int i = 0; i < C; i++) {
     const int pos = p0 + i;
     const bool in = pos < len;
-    const int j = s0 + pos;
+    const int j = seg0 + s0 + pos;  // position in the caller's row
     const bool ok = in && j < n_valid && !(al && !al[pos]) && !(alb && !((__ldg(alb + (j >> 5)) >> (j & 31)) & 1u));
     uint32_t kk = in ? order_key(val[i]) : 0u;
     nanf |= (ok && kk == 0u) ? 1u : 0u;
@@ -749,7 +754,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelParams p) 
   uint32_t eq_rank = eq_before;
   // never more than k ids, whatever the counts above say
   const uint32_t n_out = min(gt_total + min(eq_total, need), static_cast<uint32_t>(a.k));
-  int32_t *ids = a.ids + static_cast<size_t>(row) * a.k;
+  int32_t *ids = a.ids + static_cast<size_t>(grow) * a.k;
   uint32_t selbits = 0;
 #pragma unroll
   for (int i = 0; i < C; i++) {
@@ -765,14 +770,14 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelParams p) 
       }
     }
     if (sel) {
-      if (out < static_cast<uint32_t>(a.k)) ids[out] = s0 + p0 + i;
+      if (out < static_cast<uint32_t>(a.k)) ids[out] = seg0 + s0 + p0 + i;
       out++;
       selbits |= 1u << i;
     }
   }
   if (rank == 0) {
     for (int i = static_cast<int>(n_out) + tid; i < a.k; i += kThreads) ids[i] = -1;
-    if (tid == 0 && a.n_sel) a.n_sel[row] = static_cast<int32_t>(n_out);
+    if (tid == 0 && a.n_sel) a.n_sel[grow] = static_cast<int32_t>(n_out);
   }
   const int N = a.N;
   if (a.mask) {
@@ -841,29 +846,163 @@ void plan(int N, int rows, int &G, int &C) {
   while (C * kThreads < per) C <<= 1;
 }
 
+cudaError_t launch_select(const SelParams &p, int grid_rows, int N, cudaStream_t st, bool pdl) {
+  int G, C;
+  plan(N, grid_rows, G, C);
+  SelParams q = p;
+  q.slice = C * kThreads;
+  switch (C) {
+    case 1: return launch_c<1>(G, grid_rows, q, st, pdl);
+    case 2: return launch_c<2>(G, grid_rows, q, st, pdl);
+    case 4: return launch_c<4>(G, grid_rows, q, st, pdl);
+    case 8: return launch_c<8>(G, grid_rows, q, st, pdl);
+    case 16: return launch_c<16>(G, grid_rows, q, st, pdl);
+    default: return launch_c<32>(G, grid_rows, q, st, pdl);
+  }
+}
+
+// ---- rows longer than one cluster holds: each segment's own top-k first
+// (the row's top-k lies in the union of its segments' top-k: an entry with
+// fewer than k entries ranked above it in the row has fewer than k above it
+// in its segment), then the top-k of that union, whose candidates keep the
+// row's index order so ties still go to the lower index.
+constexpr int kSegLen = kMaxCluster * kThreads * 16;  // 131072 positions per segment
+constexpr int kMaxRow = kMaxCluster * kThreads * kMaxItems;
+
+struct BigRowWs {
+  size_t seg_ids, seg_n, cand_s, cand_ok, ids2, total;
+};
+
+BigRowWs big_row_ws(const lidx_topk_args &a) {
+  auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+  const size_t rows = static_cast<size_t>(a.B) * a.Q, n_seg = (a.N + kSegLen - 1) / kSegLen;
+  const size_t nc = n_seg * a.k;
+  BigRowWs w{};
+  size_t o = LIDX_WS_HEADER;
+  w.seg_ids = o;
+  o += up(rows * nc * 4);
+  w.seg_n = o;
+  o += up(rows * n_seg * 4);
+  w.cand_s = o;
+  o += up(rows * nc * 4);
+  w.cand_ok = o;
+  o += up(rows * nc);
+  w.ids2 = o;
+  o += up(rows * a.k * 4);
+  w.total = o;
+  return w;
+}
+
+// candidate c of row r: segment c / k, its i = c % k-th selected id
+__global__ void __launch_bounds__(256) gather_candidates_kernel(const lidx_topk_args a, int n_seg,
+                                                                const int32_t *seg_ids, const int32_t *seg_n,
+                                                                float *cand_s, uint8_t *cand_ok) {
+  pdl_trigger();
+  pdl_wait();
+  const int r = blockIdx.y, nc = n_seg * a.k;
+  for (int c = blockIdx.x * 256 + threadIdx.x; c < nc; c += gridDim.x * 256) {
+    const int sg = c / a.k, i = c % a.k;
+    const size_t sr = static_cast<size_t>(r) * n_seg + sg;
+    const int id = seg_ids[sr * a.k + i];
+    const bool ok = i < seg_n[sr] && id >= 0 && id < a.N;
+    cand_s[static_cast<size_t>(r) * nc + c] = ok ? a.scores[static_cast<size_t>(r) * a.ld_scores + id] : 0.f;
+    cand_ok[static_cast<size_t>(r) * nc + c] = ok ? 1 : 0;
+  }
+}
+
+// final ids: candidate positions back to row positions (still ascending);
+// the optional mask and bit set of the row (cleared before this kernel)
+__global__ void __launch_bounds__(256) map_candidates_kernel(const lidx_topk_args a, int n_seg,
+                                                             const int32_t *seg_ids, const int32_t *ids2) {
+  pdl_trigger();
+  pdl_wait();
+  const int r = blockIdx.y, nc = n_seg * a.k;
+  for (int i = blockIdx.x * 256 + threadIdx.x; i < a.k; i += gridDim.x * 256) {
+    const int c = ids2[static_cast<size_t>(r) * a.k + i];
+    int id = -1;
+    if (c >= 0 && c < nc) id = seg_ids[(static_cast<size_t>(r) * n_seg + c / a.k) * a.k + c % a.k];
+    a.ids[static_cast<size_t>(r) * a.k + i] = id;
+    if (id >= 0) {
+      if (a.mask) a.mask[static_cast<size_t>(r) * a.N + id] = 1;
+      if (a.mask_bits) atomicOr(a.mask_bits + static_cast<size_t>(r) * ((a.N + 31) / 32) + id / 32, 1u << (id % 32));
+    }
+  }
+}
+
+cudaError_t launch_big_row(const lidx_topk_args &a, void *ws, cudaStream_t st, bool pdl) {
+  const BigRowWs w = big_row_ws(a);
+  uint8_t *w8 = static_cast<uint8_t *>(ws);
+  int32_t *seg_ids = reinterpret_cast<int32_t *>(w8 + w.seg_ids), *seg_n = reinterpret_cast<int32_t *>(w8 + w.seg_n);
+  float *cand_s = reinterpret_cast<float *>(w8 + w.cand_s);
+  uint8_t *cand_ok = w8 + w.cand_ok;
+  int32_t *ids2 = reinterpret_cast<int32_t *>(w8 + w.ids2);
+  const int rows = a.B * a.Q, n_seg = (a.N + kSegLen - 1) / kSegLen, nc = n_seg * a.k;
+  // 1. every segment's top-k, ids in row positions
+  SelParams p1{};
+  p1.a = a;
+  p1.a.ids = seg_ids;
+  p1.a.n_sel = seg_n;
+  p1.a.mask = nullptr;
+  p1.a.mask_bits = nullptr;
+  p1.a.tile_stats = nullptr;
+  p1.status = static_cast<uint32_t *>(ws);
+  p1.n_seg = n_seg;
+  p1.seg_len = kSegLen;
+  cudaError_t e = launch_select(p1, rows * n_seg, kSegLen, st, pdl);
+  if (e != cudaSuccess) return e;
+  // 2. their scores in row order, with an eligibility flag
+  const dim3 g2((nc + 255) / 256 < 64 ? (nc + 255) / 256 : 64, rows);
+  e = launch_kernel(gather_candidates_kernel, g2, dim3(256), 0, st, true, a, n_seg, seg_ids, seg_n, cand_s, cand_ok);
+  if (e != cudaSuccess) return e;
+  // 3. the top-k of the union
+  SelParams p2{};
+  p2.a = a;
+  p2.a.B = rows;
+  p2.a.Q = 1;
+  p2.a.N = nc;
+  p2.a.scores = cand_s;
+  p2.a.ld_scores = nc;
+  p2.a.allowed = cand_ok;
+  p2.a.ld_allowed = nc;
+  p2.a.allowed_bits = nullptr;
+  p2.a.n_valid = nullptr;
+  p2.a.ids = ids2;
+  p2.a.mask = nullptr;
+  p2.a.mask_bits = nullptr;
+  p2.a.tile_stats = nullptr;
+  p2.status = static_cast<uint32_t *>(ws);
+  p2.n_seg = 1;
+  p2.seg_len = nc;
+  e = launch_select(p2, rows, nc, st, true);
+  if (e != cudaSuccess) return e;
+  // 4. back to row positions
+  if (a.mask && (e = cudaMemsetAsync(a.mask, 0, static_cast<size_t>(rows) * a.N, st)) != cudaSuccess) return e;
+  if (a.mask_bits &&
+      (e = cudaMemsetAsync(a.mask_bits, 0, static_cast<size_t>(rows) * ((a.N + 31) / 32) * 4, st)) != cudaSuccess)
+    return e;
+  return launch_kernel(map_candidates_kernel, dim3((a.k + 255) / 256, rows), dim3(256), 0, st, true, a, n_seg,
+                       seg_ids, ids2);
+}
+
 }  // namespace
 
-bool topk_supported(const lidx_topk_args &a) { return a.N <= kMaxCluster * kThreads * kMaxItems; }
+bool topk_supported(const lidx_topk_args &a) {
+  if (a.N <= kMaxRow) return true;
+  const int64_t n_seg = (static_cast<int64_t>(a.N) + kSegLen - 1) / kSegLen;
+  return n_seg * a.k <= kMaxRow;
+}
 
-size_t topk_workspace(const lidx_topk_args &) { return LIDX_WS_HEADER; }
+size_t topk_workspace(const lidx_topk_args &a) { return a.N <= kMaxRow ? LIDX_WS_HEADER : big_row_ws(a).total; }
 
 cudaError_t launch_topk(const lidx_topk_args &a, void *ws, cudaStream_t st) {
+  const bool pdl = (a.flags & LIDX_LAUNCH_PDL) != 0;
+  if (a.N > kMaxRow) return launch_big_row(a, ws, st, pdl);
   SelParams p{};
   p.a = a;
   p.status = static_cast<uint32_t *>(ws);
-  const int rows = a.B * a.Q;
-  int G, C;
-  plan(a.N, rows, G, C);
-  p.slice = C * kThreads;
-  const bool pdl = (a.flags & LIDX_LAUNCH_PDL) != 0;
-  switch (C) {
-    case 1: return launch_c<1>(G, rows, p, st, pdl);
-    case 2: return launch_c<2>(G, rows, p, st, pdl);
-    case 4: return launch_c<4>(G, rows, p, st, pdl);
-    case 8: return launch_c<8>(G, rows, p, st, pdl);
-    case 16: return launch_c<16>(G, rows, p, st, pdl);
-    default: return launch_c<32>(G, rows, p, st, pdl);
-  }
+  p.n_seg = 1;
+  p.seg_len = a.N;
+  return launch_select(p, a.B * a.Q, a.N, st, pdl);
 }
 
 }  // namespace lidx

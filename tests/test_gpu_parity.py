@@ -126,6 +126,23 @@ def test_topk_large_row():
     _topk_check(s, 1024)
 
 
+@pytest.mark.parametrize("N,k,rows,kind", [(300000, 1024, 1, "normal"), (300000, 1024, 2, "ties"),
+                                           (1000003, 512, 1, "signed"), (262145, 64, 3, "const")])
+def test_topk_rows_beyond_one_cluster(N, k, rows, kind):
+    """Rows longer than one thread-block cluster holds (262,144 entries) take
+    the segmented path: bit-exact ids, n_sel, mask and bits all the same."""
+    s = synth.random_scores(27, rows, N, kind)
+    _topk_check(s, k)
+
+
+def test_topk_rows_beyond_one_cluster_masked_and_nan():
+    N, k = 400000, 1024
+    s = synth.random_scores(28, 2, N, "ties")
+    s[0, ::1001] = np.nan
+    allowed = (np.random.default_rng(29).random((2, N)) < 0.2).astype(np.uint8)
+    _topk_check(s, k, allowed)
+
+
 def test_topk_allowed_mask_and_nan():
     N = 5000
     s = synth.random_scores(23, 3, N, "ties")
