@@ -244,14 +244,16 @@ __device__ void score_units(const FusedParams &p, const CUtensorMap *tm_keys, co
       if (ready) {
         tc::tc_fence_after();
         const uint32_t base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-        float s4[4] = {0.f, 0.f, 0.f, 0.f};
+        // per 32 heads four partial sums, folded into s chunk by chunk: the
+        // same order as lidx_index_score, so both give identical scores
         for (int c0 = 0; c0 < H; c0 += 32) {
           float v[32];
           tc::tmem_ld32(base + c0, v);
+          float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
           for (int h = 0; h < 32; h++) s4[h & 3] = fmaf(c->w[c0 + h], fmaxf(v[h], 0.f), s4[h & 3]);
+          s += (s4[0] + s4[1]) + (s4[2] + s4[3]);
         }
-        s = (s4[0] + s4[1]) + (s4[2] + s4[3]);
       }
       const bool in = j < p.N;
       if (in) {

@@ -201,6 +201,9 @@ class ModelStep:
                  N_csa: int, N_hca: int, k: int, swa_len: int, scale: float, device="cuda", pdl: bool = True):
         self.kinds = model_schedule(len(csa) + len(hca) + len(swa_only))
         assert self.kinds.count(CSA) == len(csa) and self.kinds.count(HCA) == len(hca)
+        # the argument structs hold raw device pointers: keep every cache they
+        # point into alive for as long as the step (and its graph) exists
+        self.hca_caches, self.swa_caches = list(hca), list(swa_only)
         dev = torch.device(device)
         self.B, self.H = B, H
         self.csa = DecodeStep(csa, B, H, N_csa, k, swa_len, scale, device=device, pdl=pdl, fused=True)

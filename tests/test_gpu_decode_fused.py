@@ -19,8 +19,13 @@ pytestmark = pytest.mark.gpu
 
 
 def _inputs(spec, layer=0):
+    """Inputs of one layer; the attention always has 64 query heads (the
+    generator ties them to the index heads, so other index head counts get
+    their own 64-head attention queries)."""
     x = synth.decode_layer(spec, layer)
     B, H, N = spec.B, spec.H, spec.N
+    if H != 64:
+        x["q_attn"] = synth.decode_layer(synth.scaled(spec, H=64, N=1), 500 + layer)["q_attn"]
     d = dict(q_idx=dev_q(x["q_idx"].reshape(B, H, 128), "bf16"), w=torch.from_numpy(x["w"].reshape(B, H)).cuda(),
              keys=dev_kv(x["keys"], batch_rows=N), q_attn=dev_q(x["q_attn"], "bf16"),
              kv=dev_kv(x["kv"], batch_rows=N), swa=dev_kv(x["swa"], batch_rows=spec.swa))
@@ -195,7 +200,7 @@ def test_fused_lost_arrival_times_out_and_recovers(cuda_device):
 
 
 def test_fused_rejects_what_it_does_not_cover(cuda_device):
-    spec = synth.scaled(synth.DECODE_500K_FP8, N=2000, k=128)
+    spec = synth.scaled(synth.DECODE_500K_FP8, N=2000, k=128, B=1)
     x = synth.decode_layer(spec)
     d = dict(q_idx=dev_q(x["q_idx"].reshape(1, 64, 128), "bf16"), w=torch.from_numpy(x["w"].reshape(1, 64)).cuda(),
              keys=dev_kv(x["keys"], batch_rows=spec.N), q_attn=dev_q(x["q_attn"], "bf16"),
