@@ -65,15 +65,17 @@ constexpr uint32_t kTmemCols = 256;
 constexpr float kLog2e = 1.4426950408889634f;
 // control words of sequence b: ctl[b * kCtlStride + ...]
 constexpr int kCtlStride = 16;
-constexpr int kCtlKmax = 0, kCtlNKmin = 1, kCtlTiles = 2, kCtlReady = 3, kCtlAttn = 4;  // kCtlAttn + hg
+constexpr int kCtlTiles = 2, kCtlReady = 3, kCtlAttn = 4;  // kCtlAttn + hg
 // smem map (offsets from the 1024-aligned base)
 constexpr int kSmKeys = 0;                     // score: two key stages
 constexpr int kSmQidx = 2 * kKeyStage;         // score: query tile, up to 128 heads
-constexpr int kSmData = kSmQidx + 128 * 256;   // end of the data region
+constexpr int kSmRowMax = 64 * kThreads * 4;  // the largest staged score row (N <= 32768)
 constexpr int kSmX = 0, kSmQa = kXBytes, kSmP = kXBytes + kQBytes;  // attention
-constexpr int kSmHist = 0, kSmCand = kNB * 4;  // select
+constexpr int kSmHist = 0, kSmCand = kNB * 4, kSmRow = kSmCand + kCandMax * 8;  // select: the row at kSmRow
+constexpr int kSmData = (kSmQidx + 128 * 256) > (kSmRow + kSmRowMax) ? (kSmQidx + 128 * 256) : (kSmRow + kSmRowMax);
 
 struct __align__(8) Ctl {
+  uint64_t row_full;
   uint64_t key_full[2];
   uint64_t q_full;
   uint64_t mma_done;
@@ -84,6 +86,7 @@ struct __align__(8) Ctl {
   uint32_t abort;
   uint32_t bc[8];         // values broadcast through shared memory
   uint32_t wsum[kWarps];  // per-warp partial sums of the block scans
+  uint32_t wlo[kWarps], whi[kWarps];  // per-warp key bounds
   float w[128];           // head weights of the query tile
   int64_t row_src[kRows];
   int32_t row_kind[kRows];
@@ -92,7 +95,7 @@ struct __align__(8) Ctl {
 
 constexpr size_t smem_bytes() { return 1024 + kSmData + sizeof(Ctl); }
 static_assert(kSmP + 2 * kPBytes <= kSmData, "attention operands fit the data region");
-static_assert(kSmCand + kCandMax * 8 <= kSmData, "selector buffers fit the data region");
+static_assert(kSmRow + kSmRowMax <= kSmData, "selector buffers and the staged row fit the data region");
 
 struct FusedParams {
   int B, H, N, k, swa_len;
@@ -260,13 +263,6 @@ __device__ void score_units(const FusedParams &p, const CUtensorMap *tm_keys, co
         p.scores[static_cast<int64_t>(b) * p.ld_ws + j] = s;
         if (p.scores_user) p.scores_user[static_cast<int64_t>(b) * p.ld_user + j] = s;
       }
-      const uint32_t kk = in ? order_key(s) : 0u;
-      const uint32_t mx = __reduce_max_sync(0xFFFFFFFFu, kk);
-      const uint32_t mn = __reduce_min_sync(0xFFFFFFFFu, kk ? kk : 0xFFFFFFFFu);
-      if (lane == 0 && mx) {
-        atomicMax(p.ctl + b * kCtlStride + kCtlKmax, mx);
-        atomicMax(p.ctl + b * kCtlStride + kCtlNKmin, ~mn);
-      }
     }
     tc::tc_fence_before();
     __syncthreads();
@@ -289,56 +285,64 @@ __device__ void score_units(const FusedParams &p, const CUtensorMap *tm_keys, co
 }
 
 // ----------------------------------------------------------------- select
+// value of an order-preserving key (the inverse of order_key for keys != 0)
+__device__ __forceinline__ float key_value(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+// Exact threshold of the keys one block holds: after it, entry j (key kk) is
+// selected iff kk > T_key or (kk == T_key and j <= T_idx).  Every thread calls
+// it.  The level-0 histogram bins the scores linearly in value over the row's
+// [min, max] (keys of score-like data spread over its bins); a bin too full
+// for rank counting is refined in key space, and a bin of equal keys takes
+// its first entries by index.
 template <int ITEMS>
-__device__ void select_unit(const FusedParams &p, int b, uint8_t *sm, Ctl *c, bool &abort) {
-  const int tid = threadIdx.x;
-  uint32_t *hist = reinterpret_cast<uint32_t *>(sm + kSmHist);
-  uint2 *cand = reinterpret_cast<uint2 *>(sm + kSmCand);
-  uint32_t *ctl = p.ctl + b * kCtlStride;
-  for (int i = tid; i < kNB; i += kThreads) hist[i] = 0u;
-  if (tid == 0) {
-    c->bc[0] = wait_geq(ctl + kCtlTiles, p.n_tiles, p.wait_ns) ? 1u : 0u;
-    c->bc[1] = 0u;  // candidate count
+__device__ void find_threshold(const uint32_t (&key)[ITEMS], int p0, int k, uint32_t *hist, uint2 *cand, Ctl *c,
+                               uint32_t &T_key, uint32_t &T_idx) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  T_key = 1u;  // default: every eligible key
+  T_idx = 0x7FFFFFFFu;
+  // row bounds
+  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+#pragma unroll
+  for (int i = 0; i < ITEMS; i++) {
+    const uint32_t kk = key[i];
+    hi = max(hi, kk);
+    lo = kk ? min(lo, kk) : lo;
+  }
+  lo = __reduce_min_sync(0xFFFFFFFFu, lo);
+  hi = __reduce_max_sync(0xFFFFFFFFu, hi);
+  if (lane == 0) {
+    c->wlo[warp] = lo;
+    c->whi[warp] = hi;
   }
   __syncthreads();
-  if (!c->bc[0]) {
-    abort = true;
-    if (tid == 0) raise_status(p.status, LIDX_DEV_TIMEOUT);
+  lo = 0xFFFFFFFFu;
+  hi = 0u;
+#pragma unroll
+  for (int w = 0; w < kWarps; w++) {
+    lo = min(lo, c->wlo[w]);
+    hi = max(hi, c->whi[w]);
   }
-  const uint32_t kmax = __ldcg(ctl + kCtlKmax), kmin = ~__ldcg(ctl + kCtlNKmin);
-  // keys of positions [tid*ITEMS, tid*ITEMS + ITEMS)
-  uint32_t key[ITEMS];
-  const int p0 = tid * ITEMS;
-  const float *row = p.scores + static_cast<int64_t>(b) * p.ld_ws;
-  bool nan = false;
+  if (hi == 0u) return;  // no eligible key
+  const float vlo = key_value(lo), vhi = key_value(hi);
+  const float range = vhi - vlo;
+  const float scale = static_cast<float>(kNB) / range;
+  const bool linear = hi > lo && isfinite(vlo) && isfinite(vhi) && isfinite(range) && range > 0.f && isfinite(scale);
+  // level-0 bin of a key: linear in value, else the top bits of (key - lo)
+  const uint32_t krange = hi - lo;
+  const uint32_t s0 = krange < kNB ? 0u : static_cast<uint32_t>(32 - __clz(krange) - 11);
+  auto bin0 = [&](uint32_t kk) -> uint32_t {
+    if (linear) return min(static_cast<uint32_t>(kNB - 1), static_cast<uint32_t>((key_value(kk) - vlo) * scale));
+    return (kk - lo) >> s0;
+  };
 #pragma unroll
-  for (int i = 0; i < ITEMS; i += 4) {
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (p0 + i < p.N) v = __ldcg(reinterpret_cast<const float4 *>(row + p0 + i));
-    const float f[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int q = 0; q < 4; q++) {
-      const bool in = p0 + i + q < p.N;
-      const uint32_t kk = in ? order_key(f[q]) : 0u;
-      nan |= in && kk == 0u;
-      key[i + q] = kk;
-    }
-  }
-  if (nan) raise_status(p.status, LIDX_DEV_NAN);
-  // level 1: bins of width 2^s over [kmin, kmax] in key space
-  const uint32_t range = kmax >= kmin ? kmax - kmin : 0u;
-  uint32_t lo = kmin, s = range < kNB ? 0u : static_cast<uint32_t>(32 - __clz(range) - 11);
-  uint32_t above = 0, T_key = 1u, T_idx = 0x7FFFFFFFu;  // default: take every eligible key
-  for (int level = 0; level < 4; level++) {
-    // histogram of the keys in [lo, lo + (kNB << s)) (all eligible keys at level 0)
-    const uint64_t span = static_cast<uint64_t>(kNB) << s;
-#pragma unroll
-    for (int i = 0; i < ITEMS; i++) {
-      const uint32_t kk = key[i];
-      if (kk && kk >= lo && static_cast<uint64_t>(kk - lo) < span) atomicAdd(&hist[(kk - lo) >> s], 1u);
-    }
-    __syncthreads();
-    // suffix scan: thread t holds bins kNB-1-4t .. kNB-4-4t (descending)
+  for (int i = 0; i < ITEMS; i++)
+    if (key[i]) atomicAdd(&hist[bin0(key[i])], 1u);
+  __syncthreads();
+  uint32_t above = 0, in_bin = 0, bin = 0;
+  // suffix scan: thread t holds bins kNB-1-4t .. kNB-4-4t (descending)
+  auto scan_bins = [&](uint32_t need, uint32_t &tot_out) {
     uint32_t cnt[4], ct = 0;
 #pragma unroll
     for (int j = 0; j < 4; j++) {
@@ -346,81 +350,194 @@ __device__ void select_unit(const FusedParams &p, int b, uint8_t *sm, Ctl *c, bo
       ct += cnt[j];
     }
     uint32_t tot;
-    uint32_t e = block_excl_scan(ct, tot, c);  // keys in the bins above this thread's
-    const uint32_t need = static_cast<uint32_t>(p.k) - above;
-    if (level == 0 && tot <= static_cast<uint32_t>(p.k)) break;  // every eligible key is taken
+    uint32_t e = block_excl_scan(ct, tot, c);
+    tot_out = tot;
     if (e < need && need <= e + ct) {
 #pragma unroll
       for (int j = 0; j < 4; j++) {
         if (e < need && need <= e + cnt[j]) {
           c->bc[2] = kNB - 1 - (4 * tid + j);
-          c->bc[3] = above + e;
+          c->bc[3] = e;
           c->bc[4] = cnt[j];
         }
         e += cnt[j];
       }
     }
     __syncthreads();
-    const uint32_t bin = c->bc[2], in_bin = c->bc[4];
-    above = c->bc[3];
-    lo = lo + (bin << s);  // the threshold bin covers keys [lo, lo + 2^s)
-    const uint32_t need2 = static_cast<uint32_t>(p.k) - above;
-    if (in_bin <= static_cast<uint32_t>(kCandMax) || s == 0) {
-      if (in_bin <= static_cast<uint32_t>(kCandMax)) {
-        // gather the bin's keys, rank them (key desc, index asc); the one of
-        // rank need2-1 is the last selected
+  };
+  uint32_t tot;
+  scan_bins(static_cast<uint32_t>(k), tot);
+  if (tot <= static_cast<uint32_t>(k)) return;  // every eligible key is taken
+  bin = c->bc[2];
+  above = c->bc[3];
+  in_bin = c->bc[4];
+  uint32_t need = static_cast<uint32_t>(k) - above;
+  // the keys of that bin form one interval [a, b] (the binning is monotone)
+  uint32_t a = 0xFFFFFFFFu, b = 0u;
 #pragma unroll
-        for (int i = 0; i < ITEMS; i++) {
-          const uint32_t kk = key[i];
-          if (kk && kk >= lo && kk - lo < (1u << s)) {
-            const uint32_t slot = atomicAdd(&c->bc[1], 1u);
-            if (slot < kCandMax) cand[slot] = make_uint2(kk, static_cast<uint32_t>(p0 + i));
-          }
-        }
-        __syncthreads();
-        const uint32_t nc = min(c->bc[1], static_cast<uint32_t>(kCandMax));
-        for (uint32_t ci = tid; ci < nc; ci += kThreads) {
-          const uint2 me = cand[ci];
-          uint32_t rank = 0;
-          for (uint32_t cj = 0; cj < nc; cj++) {
-            const uint2 o = cand[cj];
-            rank += (o.x > me.x || (o.x == me.x && o.y < me.y)) ? 1u : 0u;
-          }
-          if (rank == need2 - 1) {
-            c->bc[5] = me.x;
-            c->bc[6] = me.y;
-          }
-        }
-        __syncthreads();
-        T_key = c->bc[5];
-        T_idx = c->bc[6];
-      } else {
-        // s == 0 with more than kCandMax keys in the bin: they are all equal
-        // (a bin of width 1); take the first need2 of them by index
-        uint32_t tie = 0;
-#pragma unroll
-        for (int i = 0; i < ITEMS; i++) tie += key[i] == lo ? 1u : 0u;
-        uint32_t tt;
-        uint32_t te = block_excl_scan(tie, tt, c);
-#pragma unroll
-        for (int i = 0; i < ITEMS; i++) {
-          if (key[i] == lo) {
-            if (te == need2 - 1) c->bc[6] = static_cast<uint32_t>(p0 + i);
-            te++;
-          }
-        }
-        __syncthreads();
-        T_key = lo;
-        T_idx = c->bc[6];
-      }
-      break;
+  for (int i = 0; i < ITEMS; i++)
+    if (key[i] && bin0(key[i]) == bin) {
+      a = min(a, key[i]);
+      b = max(b, key[i]);
     }
-    // refine: the next level bins the threshold bin's 2^s keys
-    const uint32_t s2 = s > 11 ? s - 11 : 0u;
-    for (int i = tid; i < kNB; i += kThreads) hist[i] = 0u;
+  if (in_bin > static_cast<uint32_t>(kCandMax)) {
+    a = __reduce_min_sync(0xFFFFFFFFu, a);
+    b = __reduce_max_sync(0xFFFFFFFFu, b);
+    if (lane == 0) {
+      c->wlo[warp] = a;
+      c->whi[warp] = b;
+    }
     __syncthreads();
-    s = s2;
+    a = 0xFFFFFFFFu;
+    b = 0u;
+#pragma unroll
+    for (int w = 0; w < kWarps; w++) {
+      a = min(a, c->wlo[w]);
+      b = max(b, c->whi[w]);
+    }
+    // refine in key space over [a, b], 11 bits per level, until the bin is
+    // small enough to rank or holds one key value
+    uint32_t base = a;
+    uint32_t s = (b - a) < kNB ? 0u : static_cast<uint32_t>(32 - __clz(b - a) - 11);
+    for (int level = 0; level < 3 && in_bin > static_cast<uint32_t>(kCandMax) && b > a; level++) {
+      for (int i = tid; i < kNB; i += kThreads) hist[i] = 0u;
+      __syncthreads();
+      const uint64_t span = static_cast<uint64_t>(kNB) << s;
+#pragma unroll
+      for (int i = 0; i < ITEMS; i++) {
+        const uint32_t kk = key[i];
+        if (kk >= a && kk <= b && static_cast<uint64_t>(kk - base) < span) atomicAdd(&hist[(kk - base) >> s], 1u);
+      }
+      __syncthreads();
+      uint32_t t2;
+      scan_bins(need, t2);
+      above += c->bc[3];
+      need -= c->bc[3];
+      in_bin = c->bc[4];
+      const uint32_t nb_lo = base + (c->bc[2] << s);
+      const uint32_t nb_hi = s >= 32 ? 0xFFFFFFFFu : nb_lo + ((1u << s) - 1u);
+      a = max(a, nb_lo);
+      b = min(b, nb_hi);
+      base = a;
+      s = s > 11 ? s - 11 : 0u;
+    }
+    if (in_bin > static_cast<uint32_t>(kCandMax)) {
+      // a bin of one key value: take its first `need` entries by index
+      uint32_t tie = 0;
+#pragma unroll
+      for (int i = 0; i < ITEMS; i++) tie += key[i] == a ? 1u : 0u;
+      uint32_t tt;
+      uint32_t te = block_excl_scan(tie, tt, c);
+#pragma unroll
+      for (int i = 0; i < ITEMS; i++) {
+        if (key[i] == a) {
+          if (te == need - 1) c->bc[6] = static_cast<uint32_t>(p0 + i);
+          te++;
+        }
+      }
+      __syncthreads();
+      T_key = a;
+      T_idx = c->bc[6];
+      return;
+    }
   }
+  // rank the candidates (key desc, index asc); the one of rank need-1 is the
+  // last selected
+  if (tid == 0) c->bc[1] = 0u;
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < ITEMS; i++) {
+    const uint32_t kk = key[i];
+    if (kk && kk >= a && kk <= b && (in_bin <= static_cast<uint32_t>(kCandMax) ? bin0(kk) == bin : true)) {
+      const uint32_t slot = atomicAdd(&c->bc[1], 1u);
+      if (slot < kCandMax) cand[slot] = make_uint2(kk, static_cast<uint32_t>(p0 + i));
+    }
+  }
+  __syncthreads();
+  const uint32_t nc = min(c->bc[1], static_cast<uint32_t>(kCandMax));
+  for (uint32_t ci = tid; ci < nc; ci += kThreads) {
+    const uint2 me = cand[ci];
+    uint32_t rank = 0;
+    for (uint32_t cj = 0; cj < nc; cj++) {
+      const uint2 o = cand[cj];
+      rank += (o.x > me.x || (o.x == me.x && o.y < me.y)) ? 1u : 0u;
+    }
+    if (rank == need - 1) {
+      c->bc[5] = me.x;
+      c->bc[6] = me.y;
+    }
+  }
+  __syncthreads();
+  T_key = c->bc[5];
+  T_idx = c->bc[6];
+}
+
+template <int ITEMS>
+__device__ void select_unit(const FusedParams &p, int b, uint8_t *sm, Ctl *c, bool &abort) {
+  const int tid = threadIdx.x;
+  uint32_t *hist = reinterpret_cast<uint32_t *>(sm + kSmHist);
+  uint2 *cand = reinterpret_cast<uint2 *>(sm + kSmCand);
+  float *srow = reinterpret_cast<float *>(sm + kSmRow);
+  uint32_t *ctl = p.ctl + b * kCtlStride;
+  for (int i = tid; i < kNB; i += kThreads) hist[i] = 0u;
+  // the row of scores: one bulk copy into shared memory once every tile of
+  // the row is scored (the copy reads through the async proxy: fence first)
+  const uint32_t bytes = static_cast<uint32_t>(((p.N + 3) & ~3) * 4);
+  if (tid == 0) {
+    const bool ok = wait_geq(ctl + kCtlTiles, p.n_tiles, p.wait_ns);
+    c->bc[0] = ok ? 1u : 0u;
+    asm volatile("fence.proxy.async;" ::: "memory");
+    tc::mbar_arrive_expect_tx(&c->row_full, bytes);
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            tc::smem_u32(srow)),
+        "l"(p.scores + static_cast<int64_t>(b) * p.ld_ws), "r"(bytes), "r"(tc::smem_u32(&c->row_full))
+        : "memory");
+  }
+  __syncthreads();
+  if (!c->bc[0]) {
+    abort = true;
+    if (tid == 0) raise_status(p.status, LIDX_DEV_TIMEOUT);
+  }
+  {
+    bool landed = false;
+    if ((tid & 31) == 0) {
+      volatile uint32_t no_abort = 0;
+      landed = tc::mbar_wait(&c->row_full, c->bc[7] & 1u, &no_abort);
+    }
+    landed = __shfl_sync(0xFFFFFFFFu, landed, 0);
+    if (!landed && tid == 0) raise_status(p.status, LIDX_DEV_TIMEOUT);
+  }
+  // keys of positions [tid*ITEMS, tid*ITEMS + ITEMS): float4 reads rotated so
+  // the eight lanes of a phase hit eight different 16-byte bank groups
+  uint32_t key[ITEMS];
+  const int p0 = tid * ITEMS;
+  bool nan = false;
+  {
+    constexpr int n4 = ITEMS / 4;
+    const int rot = (tid * n4 / 8) % n4;
+    const float4 *src = reinterpret_cast<const float4 *>(srow + p0);
+#pragma unroll
+    for (int j = 0; j < n4; j++) {
+      const int jj = (j + rot) % n4;
+      const float4 v = p0 + 4 * jj < p.N ? src[jj] : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float f[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int q = 0; q < n4; q++)
+        if (q == jj) {
+#pragma unroll
+          for (int e = 0; e < 4; e++) {
+            const bool in = p0 + 4 * q + e < p.N;
+            const uint32_t kk = in ? order_key(f[e]) : 0u;
+            nan |= in && kk == 0u;
+            key[4 * q + e] = kk;
+          }
+        }
+    }
+  }
+  if (nan) raise_status(p.status, LIDX_DEV_NAN);
+  uint32_t T_key, T_idx;
+  find_threshold<ITEMS>(key, p0, p.k, hist, cand, c, T_key, T_idx);
   // emit ids ascending: entry j is taken when key > T or (key == T and j <= T_idx)
   uint32_t mine = 0;
 #pragma unroll
@@ -450,6 +567,7 @@ __device__ void select_unit(const FusedParams &p, int b, uint8_t *sm, Ctl *c, bo
   if (tid == 0) {
     p.sel_n[b] = n_sel;
     if (p.n_sel_user) p.n_sel_user[b] = n_sel;
+    c->bc[7]++;  // row_full phases used by this CTA
   }
   __syncthreads();
   if (tid == 0) arrive_release(ctl + kCtlReady);
@@ -736,6 +854,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   bool abort = false;
 
   if (tid == 0) {
+    tc::mbar_init(&c->row_full, 1);
+    c->bc[7] = 0u;
     tc::mbar_init(&c->key_full[0], 1);
     tc::mbar_init(&c->key_full[1], 1);
     tc::mbar_init(&c->q_full, 1);
