@@ -15,13 +15,16 @@
 //                       scores, folds the row's largest and smallest
 //                       order-preserving key into two words by atomics, and
 //                       counts the tile done (release)
-//   select (b)          waits for the row's tiles (acquire), then selects
-//                       the k largest exactly in one CTA: a 2048-bin
-//                       histogram over [min, max] in key space, a suffix scan
-//                       to the bin holding the k-th key, rank counting among
-//                       that bin's keys (or further histogram levels and an
-//                       index scan for ties), and a prefix scan that writes
-//                       the ids in ascending order; then it raises the row's
+//   select (b)          waits for the row's tiles (acquire), copies the
+//                       row into shared memory with one bulk copy, then
+//                       selects the k largest exactly in one CTA: a 2048-bin
+//                       histogram linear in value over the row's [min, max],
+//                       a suffix scan to the bin holding the k-th key, rank
+//                       counting among that bin's keys (or key-space
+//                       histogram levels, and an index scan for ties), and a
+//                       prefix scan that writes
+//                       the ids in ascending order (and starts an L2 prefetch
+//                       of each selected row); then it raises the row's
 //                       ready flag (release)
 //   attn   (b, c, hg)   64 entries of the row list (window rows first, then
 //                       the selected ids) x 16 of the 64 heads: rows by TMA
@@ -75,7 +78,6 @@ constexpr int kSmHist = 0, kSmCand = kNB * 4, kSmRow = kSmCand + kCandMax * 8;  
 constexpr int kSmData = (kSmQidx + 128 * 256) > (kSmRow + kSmRowMax) ? (kSmQidx + 128 * 256) : (kSmRow + kSmRowMax);
 
 struct __align__(8) Ctl {
-  uint64_t row_full;
   uint64_t key_full[2];
   uint64_t q_full;
   uint64_t mma_done;
@@ -141,11 +143,16 @@ __device__ __forceinline__ uint64_t globaltimer() {
   return t;
 }
 // Wait until *p >= target (acquire); false when `limit_ns` passed first.
+// Polls with a short sleep and reads the clock every 16 polls, so that many
+// waiting CTAs put little load on the memory system.
 __device__ __noinline__ bool wait_geq(const uint32_t *p, uint32_t target, uint64_t limit_ns) {
+  if (ld_acquire(p) >= target) return true;
   const uint64_t t0 = globaltimer();
-  while (ld_acquire(p) < target)
-    if (globaltimer() - t0 > limit_ns) return false;
-  return true;
+  for (uint32_t i = 1;; i++) {
+    __nanosleep(32);
+    if (ld_acquire(p) >= target) return true;
+    if ((i & 15u) == 0 && globaltimer() - t0 > limit_ns) return false;
+  }
 }
 __device__ __forceinline__ void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n)); }
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
@@ -480,34 +487,31 @@ __device__ void select_unit(const FusedParams &p, int b, uint8_t *sm, Ctl *c, bo
   float *srow = reinterpret_cast<float *>(sm + kSmRow);
   uint32_t *ctl = p.ctl + b * kCtlStride;
   for (int i = tid; i < kNB; i += kThreads) hist[i] = 0u;
-  // the row of scores: one bulk copy into shared memory once every tile of
-  // the row is scored (the copy reads through the async proxy: fence first)
-  const uint32_t bytes = static_cast<uint32_t>(((p.N + 3) & ~3) * 4);
-  if (tid == 0) {
-    const bool ok = wait_geq(ctl + kCtlTiles, p.n_tiles, p.wait_ns);
-    c->bc[0] = ok ? 1u : 0u;
-    asm volatile("fence.proxy.async;" ::: "memory");
-    tc::mbar_arrive_expect_tx(&c->row_full, bytes);
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            tc::smem_u32(srow)),
-        "l"(p.scores + static_cast<int64_t>(b) * p.ld_ws), "r"(bytes), "r"(tc::smem_u32(&c->row_full))
-        : "memory");
-  }
+  // the row of scores, once every tile of it is scored: coalesced 16-byte
+  // loads (all in flight at once) staged through shared memory
+  if (tid == 0) c->bc[0] = wait_geq(ctl + kCtlTiles, p.n_tiles, p.wait_ns) ? 1u : 0u;
   __syncthreads();
   if (!c->bc[0]) {
     abort = true;
     if (tid == 0) raise_status(p.status, LIDX_DEV_TIMEOUT);
   }
   {
-    bool landed = false;
-    if ((tid & 31) == 0) {
-      volatile uint32_t no_abort = 0;
-      landed = tc::mbar_wait(&c->row_full, c->bc[7] & 1u, &no_abort);
+    const int n4 = (p.N + 3) >> 2;
+    const float4 *g4 = reinterpret_cast<const float4 *>(p.scores + static_cast<int64_t>(b) * p.ld_ws);
+    float4 *s4 = reinterpret_cast<float4 *>(srow);
+    float4 v[ITEMS / 4];
+#pragma unroll
+    for (int i = 0; i < ITEMS / 4; i++) {
+      const int f = i * kThreads + tid;
+      if (f < n4) v[i] = __ldcg(g4 + f);
     }
-    landed = __shfl_sync(0xFFFFFFFFu, landed, 0);
-    if (!landed && tid == 0) raise_status(p.status, LIDX_DEV_TIMEOUT);
+#pragma unroll
+    for (int i = 0; i < ITEMS / 4; i++) {
+      const int f = i * kThreads + tid;
+      if (f < n4) s4[f] = v[i];
+    }
   }
+  __syncthreads();
   // keys of positions [tid*ITEMS, tid*ITEMS + ITEMS): float4 reads rotated so
   // the eight lanes of a phase hit eight different 16-byte bank groups
   uint32_t key[ITEMS];
@@ -557,6 +561,9 @@ __device__ void select_unit(const FusedParams &p, int b, uint8_t *sm, Ctl *c, bo
       if (pos < static_cast<uint32_t>(k)) {
         sel[pos] = p0 + i;
         if (uid) uid[pos] = p0 + i;
+        // start the row's trip from HBM now: the attention units gather it
+        // from L2 once the ready flag reaches them
+        prefetch_l2(p.kv + (static_cast<int64_t>(b) * p.kv_batch_rows + p0 + i) * p.kv_ld, kD * 2);
       }
       pos++;
     }
@@ -567,7 +574,6 @@ __device__ void select_unit(const FusedParams &p, int b, uint8_t *sm, Ctl *c, bo
   if (tid == 0) {
     p.sel_n[b] = n_sel;
     if (p.n_sel_user) p.n_sel_user[b] = n_sel;
-    c->bc[7]++;  // row_full phases used by this CTA
   }
   __syncthreads();
   if (tid == 0) arrive_release(ctl + kCtlReady);
@@ -854,8 +860,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   bool abort = false;
 
   if (tid == 0) {
-    tc::mbar_init(&c->row_full, 1);
-    c->bc[7] = 0u;
     tc::mbar_init(&c->key_full[0], 1);
     tc::mbar_init(&c->key_full[1], 1);
     tc::mbar_init(&c->q_full, 1);

@@ -39,14 +39,22 @@ constexpr int kTileM = 128;
 constexpr int kTileBytes = kTileM * 128 * 2;  // bf16 [128][128] as two 64-wide swizzled panels
 constexpr int kPanelBytes = kTileBytes / 2;
 constexpr int kF8Bytes = kTileM * 64;         // raw E4M3 half-tile
-constexpr int kEpiGroups = 2;                 // epilogue groups of four warps
-constexpr int kConvWarp0 = 2 + 4 * kEpiGroups;  // first FP8 converter warp
+constexpr int kMaxGroups = 4;                 // epilogue groups of four warps (at most)
+// bf16 keys: four groups, each with its own TMEM accumulator of <= 128
+// columns; E4M3 keys: two groups (the converter warps need the registers)
+template <bool kFp8>
+struct Roles {
+  static constexpr int kGroups = kFp8 ? 2 : 4;
+  static constexpr int kConv0 = 2 + 4 * kGroups;  // first FP8 converter warp
+  static constexpr int kThreads = 32 * kConv0 + (kFp8 ? 128 : 0);
+};
 
 struct TcParams {
   int B, Q, H, N;
   int QG, n_groups, n_tiles;
   int NM;             // MMA N = QG*H
   int cols_per_acc;   // TMEM columns per accumulator
+  int n_acc;          // accumulators = epilogue groups in use (2 or 4)
   uint32_t tmem_cols;
   long long units;
   int64_t key_batch_rows;
@@ -65,8 +73,8 @@ struct __align__(8) TcBarriers {
   uint64_t full[kStages];
   uint64_t empty[kStages];
   uint64_t conv[kStages];
-  uint64_t tfull[2];
-  uint64_t tempty[2];
+  uint64_t tfull[kMaxGroups];
+  uint64_t tempty[kMaxGroups];
   uint64_t bfull;
   uint64_t bempty;
   uint32_t tmem_base;
@@ -75,7 +83,7 @@ struct __align__(8) TcBarriers {
 
 __host__ __device__ constexpr size_t tc_smem_bytes(int NM, bool fp8) {
   return 1024 + static_cast<size_t>(kStages) * kTileBytes + 2ull * NM * 128 + (fp8 ? kStages * kF8Bytes : 0) +
-         kEpiGroups * 256 * sizeof(float) + sizeof(TcBarriers);
+         kMaxGroups * 256 * sizeof(float) + sizeof(TcBarriers);
 }
 
 // Coordinates (sequence b, query group g, key tile t; bg = b * n_groups + g)
@@ -105,7 +113,7 @@ struct UnitCursor {
 __device__ __forceinline__ void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n)); }
 
 template <bool kFp8>
-__global__ void __launch_bounds__(kFp8 ? 32 * kConvWarp0 + 128 : 32 * kConvWarp0, 1)
+__global__ void __launch_bounds__(Roles<kFp8>::kThreads, 1)
     score_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_rope,
                     const __grid_constant__ CUtensorMap tm_q, const TcParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -114,8 +122,9 @@ __global__ void __launch_bounds__(kFp8 ? 32 * kConvWarp0 + 128 : 32 * kConvWarp0
   uint8_t *sB = sA + kStages * kTileBytes;
   uint8_t *sF8 = sB + 2 * p.NM * 128;
   float *sW = reinterpret_cast<float *>(sF8 + (kFp8 ? kStages * kF8Bytes : 0));
-  TcBarriers *bar = reinterpret_cast<TcBarriers *>(sW + kEpiGroups * 256);
+  TcBarriers *bar = reinterpret_cast<TcBarriers *>(sW + kMaxGroups * 256);
   volatile uint32_t *abort_flag = &bar->abort;
+  constexpr int kConvWarp0 = Roles<kFp8>::kConv0;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long u0 = blockIdx.x * p.units / gridDim.x, u1 = (blockIdx.x + 1) * p.units / gridDim.x;
@@ -142,7 +151,7 @@ __global__ void __launch_bounds__(kFp8 ? 32 * kConvWarp0 + 128 : 32 * kConvWarp0
       tc::mbar_init(&bar->empty[s], 1);
       tc::mbar_init(&bar->conv[s], 128);
     }
-    for (int a = 0; a < 2; a++) {
+    for (int a = 0; a < kMaxGroups; a++) {
       tc::mbar_init(&bar->tfull[a], 1);
       tc::mbar_init(&bar->tempty[a], 4);
     }
@@ -259,7 +268,7 @@ __global__ void __launch_bounds__(kFp8 ? 32 * kConvWarp0 + 128 : 32 * kConvWarp0
           stage = 0;
           phase ^= 1;
         }
-        if (++acc == 2) {
+        if (++acc == p.n_acc) {
           acc = 0;
           acc_par ^= 1;
         }
@@ -269,8 +278,9 @@ __global__ void __launch_bounds__(kFp8 ? 32 * kConvWarp0 + 128 : 32 * kConvWarp0
     // ------------------------------------------------------------ epilogue
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
-    const int grp = (warp - 2) >> 2;             // takes units u0 + grp, u0 + grp + 2, ...
+    const int grp = (warp - 2) >> 2;             // takes units u0 + grp, u0 + grp + n_acc, ...
     const int etid = threadIdx.x - 64 - 128 * grp;
+    const int G = p.n_acc;
     float *gW = sW + grp * 256;                   // this group's head weights
     pdl_wait();  // head weights may come from the previous kernel
     const int acc = grp;
@@ -283,14 +293,15 @@ __global__ void __launch_bounds__(kFp8 ? 32 * kConvWarp0 + 128 : 32 * kConvWarp0
       const int j = cu.t * kTileM + row;
       return j < p.N ? e8m0_to_f32(p.scale[(cu.b * p.key_batch_rows + j) * p.ld_scale]) : 0.f;
     };
+    auto step = [&](UnitCursor &cu) {
+      for (int i = 0; i < G; i++) cu.next(p);
+    };
     UnitCursor cs;  // runs two of this group's units ahead of the tile being reduced
     cs.init(p, u0 + grp);
     float sc_next0 = load_scale(cs, u0 + grp < u1);
-    cs.next(p);
-    cs.next(p);
-    float sc_next1 = load_scale(cs, u0 + grp + 2 < u1);
-    cs.next(p);
-    cs.next(p);
+    step(cs);
+    float sc_next1 = load_scale(cs, u0 + grp + G < u1);
+    step(cs);
     // Score bounds of this warp's 32 keys of a tile (one span record), for the
     // top-k: the largest and the smallest non-NaN order key.  Called by whole
     // warps.
@@ -304,14 +315,14 @@ __global__ void __launch_bounds__(kFp8 ? 32 * kConvWarp0 + 128 : 32 * kConvWarp0
     };
     UnitCursor c;
     c.init(p, u0 + grp);
-    for (long long u = u0 + grp; u < u1; u += kEpiGroups, c.next(p), c.next(p)) {
+    if (grp >= G) c.init(p, u1);  // an idle group (two accumulators in use)
+    for (long long u = u0 + grp; grp < G && u < u1; u += G, step(c)) {
       const int b = c.b, g = c.g, t = c.t;
       const long long bg = c.bg;
       const float sc = sc_next0;
       sc_next0 = sc_next1;
-      sc_next1 = load_scale(cs, u + 4 < u1);
-      cs.next(p);
-      cs.next(p);
+      sc_next1 = load_scale(cs, u + 2 * G < u1);
+      step(cs);
       if (bg != prev_bg) {
         named_sync(2 + grp, 128);
         const int nq = min(p.QG, p.Q - g * p.QG);
@@ -369,24 +380,35 @@ __global__ void __launch_bounds__(kFp8 ? 32 * kConvWarp0 + 128 : 32 * kConvWarp0
               s = 0.f;
             }
           };
+          // the accumulator is free once its last chunk is in registers:
+          // hand it back to the MMA before that chunk is reduced
+          auto release = [&]() {
+            tc::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&bar->tempty[acc]);
+          };
           tc::tmem_ld32_issue(base, ra);
           for (int c = 0; c < nch; c += 2) {
             tc::tmem_ld_wait();
             tc::tmem_ld32_pin(ra);
             if (c + 1 < nch) tc::tmem_ld32_issue(base + 32 * (c + 1), rb);
+            else release();
             reduce(ra, c);
             if (c + 1 < nch) {
               tc::tmem_ld_wait();
               tc::tmem_ld32_pin(rb);
               if (c + 2 < nch) tc::tmem_ld32_issue(base + 32 * (c + 2), ra);
+              else release();
               reduce(rb, c + 1);
             }
           }
         }
       }
-      tc::tc_fence_before();
-      __syncwarp();
-      if (lane == 0 && ready) tc::mbar_arrive(&bar->tempty[acc]);
+      if (kFp8 || !ready) {  // (the bf16 path released the accumulator above)
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0 && ready) tc::mbar_arrive(&bar->tempty[acc]);
+      }
       acc_par ^= 1;
     }
   } else if (kFp8) {
@@ -445,7 +467,7 @@ int sm_count() {
 
 int choose_qg(const lidx_score_args &a) {
   if (a.keys.dtype == LIDX_E4M3) return 1;
-  return std::max(1, std::min(a.Q, 256 / a.H));
+  return std::max(1, std::min(a.Q, 128 / a.H));  // <= 128 columns: four accumulators fit TMEM
 }
 
 }  // namespace
@@ -472,8 +494,9 @@ cudaError_t launch_score_tc(const lidx_score_args &a, cudaStream_t st) {
   p.n_tiles = (a.N + kTileM - 1) / kTileM;
   p.NM = p.QG * a.H;
   p.cols_per_acc = fp8 ? 2 * a.H : p.NM;
+  p.n_acc = (!fp8 && p.cols_per_acc <= 128) ? 4 : 2;
   uint32_t cols = 32;
-  while (cols < static_cast<uint32_t>(2 * p.cols_per_acc)) cols <<= 1;
+  while (cols < static_cast<uint32_t>(p.n_acc * p.cols_per_acc)) cols <<= 1;
   p.tmem_cols = cols;
   p.units = static_cast<long long>(a.B) * p.n_groups * p.n_tiles;
   p.key_batch_rows = a.B > 1 ? a.keys.batch_rows : a.N;
@@ -510,12 +533,12 @@ cudaError_t launch_score_tc(const lidx_score_args &a, cudaStream_t st) {
   const int grid = static_cast<int>(std::min<long long>(p.units, sm_count()));
   if (fp8) {
     cudaFuncSetAttribute(score_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    return launch_kernel(score_tc_kernel<true>, dim3(grid), dim3(32 * kConvWarp0 + 128), smem, st, pdl, tm_a, tm_rope,
-                         tm_q, p);
+    return launch_kernel(score_tc_kernel<true>, dim3(grid), dim3(Roles<true>::kThreads), smem, st, pdl, tm_a,
+                         tm_rope, tm_q, p);
   } else {
     cudaFuncSetAttribute(score_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    return launch_kernel(score_tc_kernel<false>, dim3(grid), dim3(32 * kConvWarp0), smem, st, pdl, tm_a, tm_rope, tm_q,
-                         p);
+    return launch_kernel(score_tc_kernel<false>, dim3(grid), dim3(Roles<false>::kThreads), smem, st, pdl, tm_a,
+                         tm_rope, tm_q, p);
   }
 }
 
