@@ -292,31 +292,28 @@ __device__ void score_units(const FusedParams &p, const CUtensorMap *tm_keys, co
 }
 
 // ----------------------------------------------------------------- select
+// The selector runs once per launch on one SM, so its instructions come cold
+// from L2 or HBM: it is written as short rolled loops over the row's keys in
+// shared memory (not unrolled register arrays), which keeps the code small.
+// Thread t owns positions [t*items, t*items + items), the i-th of them at
+// key slot i*kThreads + t (consecutive threads, consecutive words: no bank
+// conflicts).
+
 // value of an order-preserving key (the inverse of order_key for keys != 0)
 __device__ __forceinline__ float key_value(uint32_t k) {
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
 
-// Exact threshold of the keys one block holds: after it, entry j (key kk) is
-// selected iff kk > T_key or (kk == T_key and j <= T_idx).  Every thread calls
-// it.  The level-0 histogram bins the scores linearly in value over the row's
-// [min, max] (keys of score-like data spread over its bins); a bin too full
-// for rank counting is refined in key space, and a bin of equal keys takes
-// its first entries by index.
-template <int ITEMS>
-__device__ void find_threshold(const uint32_t (&key)[ITEMS], int p0, int k, uint32_t *hist, uint2 *cand, Ctl *c,
-                               uint32_t &T_key, uint32_t &T_idx) {
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  T_key = 1u;  // default: every eligible key
-  T_idx = 0x7FFFFFFFu;
-  // row bounds
-  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
-#pragma unroll
-  for (int i = 0; i < ITEMS; i++) {
-    const uint32_t kk = key[i];
-    hi = max(hi, kk);
-    lo = kk ? min(lo, kk) : lo;
-  }
+struct SelView {
+  const uint32_t *key;  // [items][kThreads]
+  int items;
+  __device__ __forceinline__ uint32_t at(int i) const { return key[i * kThreads + threadIdx.x]; }
+  __device__ __forceinline__ int pos(int i) const { return static_cast<int>(threadIdx.x) * items + i; }
+};
+
+// block-wide min and max of (lo, hi) through the per-warp slots
+__device__ __forceinline__ void block_minmax(uint32_t &lo, uint32_t &hi, Ctl *c) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   lo = __reduce_min_sync(0xFFFFFFFFu, lo);
   hi = __reduce_max_sync(0xFFFFFFFFu, hi);
   if (lane == 0) {
@@ -324,140 +321,140 @@ __device__ void find_threshold(const uint32_t (&key)[ITEMS], int p0, int k, uint
     c->whi[warp] = hi;
   }
   __syncthreads();
-  lo = 0xFFFFFFFFu;
-  hi = 0u;
+  lo = c->wlo[lane & (kWarps - 1)];
+  hi = c->whi[lane & (kWarps - 1)];
+  lo = __reduce_min_sync(0xFFFFFFFFu, lo);
+  hi = __reduce_max_sync(0xFFFFFFFFu, hi);
+  __syncthreads();  // the slots are reused
+}
+
+// Suffix scan of hist (thread t holds bins kNB-1-4t .. kNB-4-4t) to the bin
+// holding the need-th largest key: bc[2] = that bin, bc[3] = keys above it,
+// bc[4] = keys in it; returns the histogram's total.
+__device__ __noinline__ uint32_t find_bin(const uint32_t *hist, uint32_t need, Ctl *c) {
+  const int tid = threadIdx.x;
+  uint32_t cnt[4], ct = 0;
 #pragma unroll
-  for (int w = 0; w < kWarps; w++) {
-    lo = min(lo, c->wlo[w]);
-    hi = max(hi, c->whi[w]);
+  for (int j = 0; j < 4; j++) {
+    cnt[j] = hist[kNB - 1 - (4 * tid + j)];
+    ct += cnt[j];
   }
+  uint32_t tot;
+  uint32_t e = block_excl_scan(ct, tot, c);
+  if (e < need && need <= e + ct) {
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+      if (e < need && need <= e + cnt[j]) {
+        c->bc[2] = kNB - 1 - (4 * tid + j);
+        c->bc[3] = e;
+        c->bc[4] = cnt[j];
+      }
+      e += cnt[j];
+    }
+  }
+  __syncthreads();
+  return tot;
+}
+
+// Exact threshold: entry j (key kk) is selected iff kk > T_key or
+// (kk == T_key and j <= T_idx).  The level-0 histogram bins the scores
+// linearly in value over the row's [min, max] (keys of score-like data spread
+// over its bins); a bin too full for rank counting is refined in key space,
+// and a bin of one key value takes its first entries by index.
+__device__ __noinline__ void find_threshold(const SelView v, int k, uint32_t *hist, uint2 *cand, Ctl *c,
+                                            uint32_t &T_key, uint32_t &T_idx) {
+  const int tid = threadIdx.x;
+  T_key = 1u;  // default: every eligible key
+  T_idx = 0x7FFFFFFFu;
+  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+#pragma unroll 4
+  for (int i = 0; i < v.items; i++) {
+    const uint32_t kk = v.at(i);
+    hi = max(hi, kk);
+    lo = kk ? min(lo, kk) : lo;
+  }
+  block_minmax(lo, hi, c);
   if (hi == 0u) return;  // no eligible key
   const float vlo = key_value(lo), vhi = key_value(hi);
   const float range = vhi - vlo;
   const float scale = static_cast<float>(kNB) / range;
   const bool linear = hi > lo && isfinite(vlo) && isfinite(vhi) && isfinite(range) && range > 0.f && isfinite(scale);
-  // level-0 bin of a key: linear in value, else the top bits of (key - lo)
   const uint32_t krange = hi - lo;
   const uint32_t s0 = krange < kNB ? 0u : static_cast<uint32_t>(32 - __clz(krange) - 11);
+  // level-0 bin of a key: linear in value, else the top bits of (key - lo)
   auto bin0 = [&](uint32_t kk) -> uint32_t {
     if (linear) return min(static_cast<uint32_t>(kNB - 1), static_cast<uint32_t>((key_value(kk) - vlo) * scale));
     return (kk - lo) >> s0;
   };
-#pragma unroll
-  for (int i = 0; i < ITEMS; i++)
-    if (key[i]) atomicAdd(&hist[bin0(key[i])], 1u);
+#pragma unroll 4
+  for (int i = 0; i < v.items; i++) {
+    const uint32_t kk = v.at(i);
+    if (kk) atomicAdd(&hist[bin0(kk)], 1u);
+  }
   __syncthreads();
-  uint32_t above = 0, in_bin = 0, bin = 0;
-  // suffix scan: thread t holds bins kNB-1-4t .. kNB-4-4t (descending)
-  auto scan_bins = [&](uint32_t need, uint32_t &tot_out) {
-    uint32_t cnt[4], ct = 0;
-#pragma unroll
-    for (int j = 0; j < 4; j++) {
-      cnt[j] = hist[kNB - 1 - (4 * tid + j)];
-      ct += cnt[j];
-    }
-    uint32_t tot;
-    uint32_t e = block_excl_scan(ct, tot, c);
-    tot_out = tot;
-    if (e < need && need <= e + ct) {
-#pragma unroll
-      for (int j = 0; j < 4; j++) {
-        if (e < need && need <= e + cnt[j]) {
-          c->bc[2] = kNB - 1 - (4 * tid + j);
-          c->bc[3] = e;
-          c->bc[4] = cnt[j];
-        }
-        e += cnt[j];
-      }
-    }
-    __syncthreads();
-  };
-  uint32_t tot;
-  scan_bins(static_cast<uint32_t>(k), tot);
-  if (tot <= static_cast<uint32_t>(k)) return;  // every eligible key is taken
-  bin = c->bc[2];
-  above = c->bc[3];
-  in_bin = c->bc[4];
-  uint32_t need = static_cast<uint32_t>(k) - above;
+  if (find_bin(hist, static_cast<uint32_t>(k), c) <= static_cast<uint32_t>(k)) return;  // every eligible key
+  const uint32_t bin = c->bc[2];
+  uint32_t need = static_cast<uint32_t>(k) - c->bc[3];
+  uint32_t in_bin = c->bc[4];
   // the keys of that bin form one interval [a, b] (the binning is monotone)
   uint32_t a = 0xFFFFFFFFu, b = 0u;
-#pragma unroll
-  for (int i = 0; i < ITEMS; i++)
-    if (key[i] && bin0(key[i]) == bin) {
-      a = min(a, key[i]);
-      b = max(b, key[i]);
+#pragma unroll 4
+  for (int i = 0; i < v.items; i++) {
+    const uint32_t kk = v.at(i);
+    if (kk && bin0(kk) == bin) {
+      a = min(a, kk);
+      b = max(b, kk);
     }
-  if (in_bin > static_cast<uint32_t>(kCandMax)) {
-    a = __reduce_min_sync(0xFFFFFFFFu, a);
-    b = __reduce_max_sync(0xFFFFFFFFu, b);
-    if (lane == 0) {
-      c->wlo[warp] = a;
-      c->whi[warp] = b;
+  }
+  block_minmax(a, b, c);
+  // refine in key space over [a, b], 11 bits per level, until the bin is
+  // small enough to rank or holds one key value
+  uint32_t s = (b - a) < kNB ? 0u : static_cast<uint32_t>(32 - __clz(b - a) - 11);
+  for (int level = 0; level < 3 && in_bin > static_cast<uint32_t>(kCandMax) && b > a; level++) {
+    for (int i = tid; i < kNB; i += kThreads) hist[i] = 0u;
+    __syncthreads();
+    const uint32_t base = a;
+#pragma unroll 4
+    for (int i = 0; i < v.items; i++) {
+      const uint32_t kk = v.at(i);
+      if (kk >= a && kk <= b) atomicAdd(&hist[(kk - base) >> s], 1u);
     }
     __syncthreads();
-    a = 0xFFFFFFFFu;
-    b = 0u;
-#pragma unroll
-    for (int w = 0; w < kWarps; w++) {
-      a = min(a, c->wlo[w]);
-      b = max(b, c->whi[w]);
-    }
-    // refine in key space over [a, b], 11 bits per level, until the bin is
-    // small enough to rank or holds one key value
-    uint32_t base = a;
-    uint32_t s = (b - a) < kNB ? 0u : static_cast<uint32_t>(32 - __clz(b - a) - 11);
-    for (int level = 0; level < 3 && in_bin > static_cast<uint32_t>(kCandMax) && b > a; level++) {
-      for (int i = tid; i < kNB; i += kThreads) hist[i] = 0u;
-      __syncthreads();
-      const uint64_t span = static_cast<uint64_t>(kNB) << s;
-#pragma unroll
-      for (int i = 0; i < ITEMS; i++) {
-        const uint32_t kk = key[i];
-        if (kk >= a && kk <= b && static_cast<uint64_t>(kk - base) < span) atomicAdd(&hist[(kk - base) >> s], 1u);
+    find_bin(hist, need, c);
+    need -= c->bc[3];
+    in_bin = c->bc[4];
+    const uint32_t nb_lo = base + (c->bc[2] << s);
+    a = max(a, nb_lo);
+    b = min(b, nb_lo + ((1u << s) - 1u));
+    s = s > 11 ? s - 11 : 0u;
+  }
+  if (in_bin > static_cast<uint32_t>(kCandMax)) {
+    // one key value: take its first `need` entries by index
+    uint32_t tie = 0;
+#pragma unroll 4
+    for (int i = 0; i < v.items; i++) tie += v.at(i) == a ? 1u : 0u;
+    uint32_t tt;
+    uint32_t te = block_excl_scan(tie, tt, c);
+    for (int i = 0; i < v.items; i++) {
+      if (v.at(i) == a) {
+        if (te == need - 1) c->bc[6] = static_cast<uint32_t>(v.pos(i));
+        te++;
       }
-      __syncthreads();
-      uint32_t t2;
-      scan_bins(need, t2);
-      above += c->bc[3];
-      need -= c->bc[3];
-      in_bin = c->bc[4];
-      const uint32_t nb_lo = base + (c->bc[2] << s);
-      const uint32_t nb_hi = s >= 32 ? 0xFFFFFFFFu : nb_lo + ((1u << s) - 1u);
-      a = max(a, nb_lo);
-      b = min(b, nb_hi);
-      base = a;
-      s = s > 11 ? s - 11 : 0u;
     }
-    if (in_bin > static_cast<uint32_t>(kCandMax)) {
-      // a bin of one key value: take its first `need` entries by index
-      uint32_t tie = 0;
-#pragma unroll
-      for (int i = 0; i < ITEMS; i++) tie += key[i] == a ? 1u : 0u;
-      uint32_t tt;
-      uint32_t te = block_excl_scan(tie, tt, c);
-#pragma unroll
-      for (int i = 0; i < ITEMS; i++) {
-        if (key[i] == a) {
-          if (te == need - 1) c->bc[6] = static_cast<uint32_t>(p0 + i);
-          te++;
-        }
-      }
-      __syncthreads();
-      T_key = a;
-      T_idx = c->bc[6];
-      return;
-    }
+    __syncthreads();
+    T_key = a;
+    T_idx = c->bc[6];
+    return;
   }
   // rank the candidates (key desc, index asc); the one of rank need-1 is the
   // last selected
   if (tid == 0) c->bc[1] = 0u;
   __syncthreads();
-#pragma unroll
-  for (int i = 0; i < ITEMS; i++) {
-    const uint32_t kk = key[i];
-    if (kk && kk >= a && kk <= b && (in_bin <= static_cast<uint32_t>(kCandMax) ? bin0(kk) == bin : true)) {
+  for (int i = 0; i < v.items; i++) {
+    const uint32_t kk = v.at(i);
+    if (kk >= a && kk <= b && kk) {
       const uint32_t slot = atomicAdd(&c->bc[1], 1u);
-      if (slot < kCandMax) cand[slot] = make_uint2(kk, static_cast<uint32_t>(p0 + i));
+      if (slot < kCandMax) cand[slot] = make_uint2(kk, static_cast<uint32_t>(v.pos(i)));
     }
   }
   __syncthreads();
@@ -479,94 +476,68 @@ __device__ void find_threshold(const uint32_t (&key)[ITEMS], int p0, int k, uint
   T_idx = c->bc[6];
 }
 
-template <int ITEMS>
-__device__ void select_unit(const FusedParams &p, int b, uint8_t *sm, Ctl *c, bool &abort) {
+__device__ __noinline__ void select_unit(const FusedParams &p, int b, uint8_t *sm, Ctl *c, bool &abort) {
   const int tid = threadIdx.x;
+  const int items = p.items;
   uint32_t *hist = reinterpret_cast<uint32_t *>(sm + kSmHist);
   uint2 *cand = reinterpret_cast<uint2 *>(sm + kSmCand);
-  float *srow = reinterpret_cast<float *>(sm + kSmRow);
+  uint32_t *skey = reinterpret_cast<uint32_t *>(sm + kSmRow);
   uint32_t *ctl = p.ctl + b * kCtlStride;
   for (int i = tid; i < kNB; i += kThreads) hist[i] = 0u;
-  // the row of scores, once every tile of it is scored: coalesced 16-byte
-  // loads (all in flight at once) staged through shared memory
   if (tid == 0) c->bc[0] = wait_geq(ctl + kCtlTiles, p.n_tiles, p.wait_ns) ? 1u : 0u;
   __syncthreads();
   if (!c->bc[0]) {
     abort = true;
     if (tid == 0) raise_status(p.status, LIDX_DEV_TIMEOUT);
   }
-  {
-    const int n4 = (p.N + 3) >> 2;
-    const float4 *g4 = reinterpret_cast<const float4 *>(p.scores + static_cast<int64_t>(b) * p.ld_ws);
-    float4 *s4 = reinterpret_cast<float4 *>(srow);
-    float4 v[ITEMS / 4];
-#pragma unroll
-    for (int i = 0; i < ITEMS / 4; i++) {
-      const int f = i * kThreads + tid;
-      if (f < n4) v[i] = __ldcg(g4 + f);
-    }
-#pragma unroll
-    for (int i = 0; i < ITEMS / 4; i++) {
-      const int f = i * kThreads + tid;
-      if (f < n4) s4[f] = v[i];
-    }
-  }
-  __syncthreads();
-  // keys of positions [tid*ITEMS, tid*ITEMS + ITEMS): float4 reads rotated so
-  // the eight lanes of a phase hit eight different 16-byte bank groups
-  uint32_t key[ITEMS];
-  const int p0 = tid * ITEMS;
+  // this thread's positions [tid*items, +items): float4 loads, then one key
+  // per slot; NaN and positions beyond N get key 0 (never selected)
+  const SelView v{skey, items};
+  const int p0 = tid * items;
+  const float *row = p.scores + static_cast<int64_t>(b) * p.ld_ws;
   bool nan = false;
-  {
-    constexpr int n4 = ITEMS / 4;
-    const int rot = (tid * n4 / 8) % n4;
-    const float4 *src = reinterpret_cast<const float4 *>(srow + p0);
+#pragma unroll 2
+  for (int i = 0; i < items; i += 4) {
+    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (p0 + i < p.N) x = __ldcg(reinterpret_cast<const float4 *>(row + p0 + i));
+    const float f[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
-    for (int j = 0; j < n4; j++) {
-      const int jj = (j + rot) % n4;
-      const float4 v = p0 + 4 * jj < p.N ? src[jj] : make_float4(0.f, 0.f, 0.f, 0.f);
-      const float f[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int q = 0; q < n4; q++)
-        if (q == jj) {
-#pragma unroll
-          for (int e = 0; e < 4; e++) {
-            const bool in = p0 + 4 * q + e < p.N;
-            const uint32_t kk = in ? order_key(f[e]) : 0u;
-            nan |= in && kk == 0u;
-            key[4 * q + e] = kk;
-          }
-        }
+    for (int e = 0; e < 4; e++) {
+      const bool in = p0 + i + e < p.N;
+      const uint32_t kk = in ? order_key(f[e]) : 0u;
+      nan |= in && kk == 0u;
+      skey[(i + e) * kThreads + tid] = kk;
     }
   }
   if (nan) raise_status(p.status, LIDX_DEV_NAN);
+  __syncthreads();
   uint32_t T_key, T_idx;
-  find_threshold<ITEMS>(key, p0, p.k, hist, cand, c, T_key, T_idx);
+  find_threshold(v, p.k, hist, cand, c, T_key, T_idx);
   // emit ids ascending: entry j is taken when key > T or (key == T and j <= T_idx)
+  auto taken = [&](int i) {
+    const uint32_t kk = v.at(i);
+    return kk != 0u && (kk > T_key || (kk == T_key && static_cast<uint32_t>(v.pos(i)) <= T_idx));
+  };
   uint32_t mine = 0;
-#pragma unroll
-  for (int i = 0; i < ITEMS; i++) {
-    const uint32_t kk = key[i];
-    mine += (kk != 0u && (kk > T_key || (kk == T_key && static_cast<uint32_t>(p0 + i) <= T_idx))) ? 1u : 0u;
-  }
+#pragma unroll 4
+  for (int i = 0; i < items; i++) mine += taken(i) ? 1u : 0u;
   uint32_t n_out;
   uint32_t pos = block_excl_scan(mine, n_out, c);
   const int k = p.k;
   int32_t *sel = p.sel_ids + static_cast<int64_t>(b) * k;
   int32_t *uid = p.ids_user ? p.ids_user + static_cast<int64_t>(b) * k : nullptr;
-#pragma unroll
-  for (int i = 0; i < ITEMS; i++) {
-    const uint32_t kk = key[i];
-    if (kk != 0u && (kk > T_key || (kk == T_key && static_cast<uint32_t>(p0 + i) <= T_idx))) {
-      if (pos < static_cast<uint32_t>(k)) {
-        sel[pos] = p0 + i;
-        if (uid) uid[pos] = p0 + i;
-        // start the row's trip from HBM now: the attention units gather it
-        // from L2 once the ready flag reaches them
-        prefetch_l2(p.kv + (static_cast<int64_t>(b) * p.kv_batch_rows + p0 + i) * p.kv_ld, kD * 2);
-      }
-      pos++;
+  for (int i = 0; i < items && mine; i++) {
+    if (!taken(i)) continue;
+    mine--;
+    if (pos < static_cast<uint32_t>(k)) {
+      const int j = v.pos(i);
+      sel[pos] = j;
+      if (uid) uid[pos] = j;
+      // start the row's trip from HBM now: the attention units gather it
+      // from L2 once the ready flag reaches them
+      prefetch_l2(p.kv + (static_cast<int64_t>(b) * p.kv_batch_rows + j) * p.kv_ld, kD * 2);
     }
+    pos++;
   }
   const int n_sel = static_cast<int>(min(n_out, static_cast<uint32_t>(k)));
   if (uid)
@@ -848,7 +819,6 @@ __device__ void attn_unit(const FusedParams &p, int a, const CUtensorMap *tm_qa,
 }
 
 // ------------------------------------------------------------------ kernel
-template <int ITEMS>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_fused_kernel(const __grid_constant__ CUtensorMap tm_keys, const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_qa, const __grid_constant__ CUtensorMap tm_win,
@@ -905,7 +875,7 @@ __global__ void __launch_bounds__(kThreads, 1)
        u < p.n_score + p.B; u += p.G) {
     tc::fence_proxy_async_smem();
     __syncthreads();
-    select_unit<ITEMS>(p, u - p.n_score, sm, c, abort);
+    select_unit(p, u - p.n_score, sm, c, abort);
   }
   // the attention unit (at most one per CTA)
   {
@@ -1060,17 +1030,8 @@ cudaError_t launch_decode_fused(const lidx_decode_args &a, void *ws, cudaStream_
   if (!ok) return cudaErrorInvalidValue;
   const size_t smem = smem_bytes();
   const bool pdl = (a.flags & LIDX_LAUNCH_PDL) != 0;
-  auto go = [&](auto kern) {
-    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    return launch_kernel(kern, dim3(p.G), dim3(kThreads), smem, st, pdl, tm_keys, tm_q, tm_qa, tm_win, p);
-  };
-  switch (p.items) {
-    case 4: return go(decode_fused_kernel<4>);
-    case 8: return go(decode_fused_kernel<8>);
-    case 16: return go(decode_fused_kernel<16>);
-    case 32: return go(decode_fused_kernel<32>);
-    default: return go(decode_fused_kernel<64>);
-  }
+  cudaFuncSetAttribute(decode_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  return launch_kernel(decode_fused_kernel, dim3(p.G), dim3(kThreads), smem, st, pdl, tm_keys, tm_q, tm_qa, tm_win, p);
 }
 
 }  // namespace lidx
