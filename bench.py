@@ -315,8 +315,12 @@ def clone_kv(kv):
                       None if kv.rope is None else kv.rope.clone(), kv.batch_rows)
 
 
-def make_replica_steps(spec, layers_inp, R, device):
-    """R DecodeSteps over copies of the same caches (the bench rotates them)."""
+LAYER_FORMS = {"auto": None, "fused": True, "calls": False}
+
+
+def make_replica_steps(spec, layers_inp, R, device, fused=None):
+    """R DecodeSteps over copies of the same caches (the bench rotates them).
+    fused: None lets DecodeStep choose the layer form, True / False force it."""
     import torch
     from lightning_indexer_top_index_b200.decode import DecodeStep, LayerCache
     base = make_caches(spec, layers_inp, device)
@@ -325,7 +329,7 @@ def make_replica_steps(spec, layers_inp, R, device):
     for r in range(R):
         caches = base if r == 0 else [LayerCache(clone_kv(c.keys), clone_kv(c.kv), clone_kv(c.swa)) for c in base]
         steps.append(DecodeStep(caches, spec.B, spec.H, spec.N, spec.k, spec.swa, spec.scale, q_dtype=qdt,
-                                device=device))
+                                device=device, fused=fused))
     return steps
 
 
@@ -355,7 +359,7 @@ def measure_decode(args, name, spec, world, dist, device, local_rank, rank, want
     ab = algorithmic_bytes(spec)
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
     R = max(2, math.ceil(4 * l2 / ab["step"]))
-    steps = make_replica_steps(spec, layers_inp, R, device)
+    steps = make_replica_steps(spec, layers_inp, R, device, fused=LAYER_FORMS[args.layer_form])
     q_idx_h, w_h, q_attn_h = host_queries(spec, layers_inp)
     for s in steps:
         s.set_inputs(q_idx_h.to(device), w_h.to(device), q_attn_h.to(device))
@@ -765,6 +769,8 @@ def main():
     ap.add_argument("--impl", default="lidx", choices=["lidx", "reference"])
     ap.add_argument("--workload", default="decode-64k", choices=sorted(WORKLOADS) + [EVAL, MODEL])
     ap.add_argument("--only", action="store_true", help="time the named workload alone")
+    ap.add_argument("--layer-form", default="auto", choices=sorted(LAYER_FORMS),
+                    help="CSA decode layers: one launch per layer, three calls, or the library's choice")
     args = ap.parse_args()
     args.repeats = max(5, args.repeats)
     rank = int(os.environ.get("RANK", "0"))

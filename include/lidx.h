@@ -269,7 +269,7 @@ LIDX_API lidx_status lidx_sparse_attn_decode(const lidx_attn_args *args, void *w
  *           depends on it).  16-byte aligned, sizes multiples of 16.
  *
  * Supported: bf16 keys, rows and queries, H a multiple of 32 up to 128,
- * N <= 32768, and B * ceil((swa_len + k) / 64) * 4 <= the device's SM count
+ * N <= 16384, and B * ceil((swa_len + k) / 64) * 4 <= the device's SM count
  * (every attention unit runs concurrently); otherwise LIDX_ERR_UNSUPPORTED
  * (use the three calls).  The workspace (lidx_workspace_size(LIDX_OP_DECODE))
  * must be zeroed before its first use; every call leaves its control words

@@ -69,10 +69,21 @@ constexpr float kLog2e = 1.4426950408889634f;
 // control words of sequence b: ctl[b * kCtlStride + ...]
 constexpr int kCtlStride = 16;
 constexpr int kCtlTiles = 2, kCtlReady = 3, kCtlAttn = 4;  // kCtlAttn + hg
+constexpr int kCtlCand = 9;   // score units that published their candidates
+constexpr int kCtlCandN = 10; // candidates in the row's list
+constexpr int kCtlMode = 11;  // kModeSplit: the score units select; kModeOneCta: the selector unit does
+constexpr int kCtlNeed = 12;  // rank (1-based) of the last taken candidate
+constexpr int kCtlAll = 13;   // at most k keys are eligible: all are taken
+constexpr uint32_t kModeSplit = 1, kModeOneCta = 2;
+constexpr int kMaxOwnTiles = 4;   // score units per CTA
+constexpr int kCandSplit = 512;   // largest fine bin the split selection ranks
+constexpr int kNB1 = 256;         // coarse histogram bins (top 8 key bits)
+constexpr int kNB2 = 65536;       // fine histogram bins (top 16 key bits): 256 under each coarse bin
 // smem map (offsets from the 1024-aligned base)
 constexpr int kSmKeys = 0;                     // score: two key stages
 constexpr int kSmQidx = 2 * kKeyStage;         // score: query tile, up to 128 heads
-constexpr int kSmRowMax = 64 * kThreads * 4;  // the largest staged score row (N <= 32768)
+constexpr int kSelItems = 32;                 // row positions per selector thread
+constexpr int kSmRowMax = kSelItems * kThreads * 4 / 32 * 36;  // the staged row, 4 pad words per 32 scores
 constexpr int kSmX = 0, kSmQa = kXBytes, kSmP = kXBytes + kQBytes;  // attention
 constexpr int kSmHist = 0, kSmCand = kNB * 4, kSmRow = kSmCand + kCandMax * 8;  // select: the row at kSmRow
 constexpr int kSmData = (kSmQidx + 128 * 256) > (kSmRow + kSmRowMax) ? (kSmQidx + 128 * 256) : (kSmRow + kSmRowMax);
@@ -88,7 +99,12 @@ struct __align__(8) Ctl {
   uint32_t abort;
   uint32_t bc[8];         // values broadcast through shared memory
   uint32_t wsum[kWarps];  // per-warp partial sums of the block scans
-  uint32_t wlo[kWarps], whi[kWarps];  // per-warp key bounds
+  uint32_t wlo[kWarps], whi[kWarps];  // per-warp key bounds of the selector
+  float tile_x[kMaxOwnTiles][kTileM];  // this CTA's score units: their scores (NaN: none)
+  uint32_t h1[kNB1];                   // a tile's coarse histogram, added to the row's in one go
+  uint32_t ctile[kTileM];              // split view: per tile, candidates taken
+  uint32_t toff[kTileM + 1];           // split view: per tile, offset in the id list
+  int32_t chunk_id[kRows];             // attention: the ids of the chunk's selected rows
   float w[128];           // head weights of the query tile
   int64_t row_src[kRows];
   int32_t row_kind[kRows];
@@ -97,12 +113,13 @@ struct __align__(8) Ctl {
 
 constexpr size_t smem_bytes() { return 1024 + kSmData + sizeof(Ctl); }
 static_assert(kSmP + 2 * kPBytes <= kSmData, "attention operands fit the data region");
+constexpr int kSmSplit = kSmP + 2 * kPBytes;  // split view: the candidates (beside the attention operands)
+static_assert(kSmSplit + kCandSplit * 8 <= kSmData, "split view scratch fits the data region");
 static_assert(kSmRow + kSmRowMax <= kSmData, "selector buffers and the staged row fit the data region");
 
 struct FusedParams {
   int B, H, N, k, swa_len;
   int n_tiles, n_chunks, n_score, n_attn, G;
-  int items;              // scores per selector thread
   int64_t key_batch_rows;
   const float *w;
   const uint16_t *kv;     // bf16 rows
@@ -116,6 +133,10 @@ struct FusedParams {
   int32_t *ids_user, *n_sel_user;
   uint32_t *status, *ctl;
   float *scores;          // workspace copy, row stride ld_ws
+  uint32_t *hist2;        // per sequence: kNB2-bin fine histogram (cleared by the score units)
+  uint32_t *above;        // per score tile: its scores taken without ranking
+  uint2 *gcand;           // per sequence: kCandSplit (key, position) candidates of the threshold bin
+  uint32_t *hist;         // per sequence: kNB1-bin coarse histogram of the score keys (cleared by the score units)
   int64_t ld_ws;
   int32_t *sel_ids, *sel_n;
   float *part_o;
@@ -134,8 +155,8 @@ __device__ __forceinline__ uint32_t ld_acquire(const uint32_t *p) {
 }
 // Count one arrival after the whole CTA's prior writes (called by one thread
 // after a block barrier: the fence is cumulative over what the barrier ordered).
-__device__ __forceinline__ void arrive_release(uint32_t *p) {
-  asm volatile("fence.acq_rel.gpu;\n\tred.relaxed.gpu.global.add.u32 [%0], 1;" ::"l"(p) : "memory");
+__device__ __forceinline__ void arrive_release(uint32_t *p, uint32_t n = 1u) {
+  asm volatile("fence.acq_rel.gpu;\n\tred.relaxed.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(n) : "memory");
 }
 __device__ __forceinline__ uint64_t globaltimer() {
   uint64_t t;
@@ -270,10 +291,31 @@ __device__ void score_units(const FusedParams &p, const CUtensorMap *tm_keys, co
         p.scores[static_cast<int64_t>(b) * p.ld_ws + j] = s;
         if (p.scores_user) p.scores_user[static_cast<int64_t>(b) * p.ld_user + j] = s;
       }
+      // the row's two key histograms (0 = no score: NaN, or past N)
+      const uint32_t kk = in ? order_key(s) : 0u;
+      if (__any_sync(0xFFFFFFFFu, in && kk == 0u) && lane == 0) raise_status(p.status, LIDX_DEV_NAN);
+      {  // one add per distinct bin of the warp (the scores crowd a few bins)
+        const uint32_t m1 = __match_any_sync(0xFFFFFFFFu, kk ? kk >> 24 : 0xFFFFFFFFu);
+        const uint32_t m2 = __match_any_sync(0xFFFFFFFFu, kk ? kk >> 16 : 0xFFFFFFFFu);
+        if (kk && lane == __ffs(m1) - 1) atomicAdd(&c->h1[kk >> 24], static_cast<uint32_t>(__popc(m1)));
+        if (kk && lane == __ffs(m2) - 1)
+          atomicAdd(p.hist2 + static_cast<int64_t>(b) * kNB2 + (kk >> 16), static_cast<uint32_t>(__popc(m2)));
+      }
+      if (i < kMaxOwnTiles) c->tile_x[i][row] = in ? s : NAN;
     }
     tc::tc_fence_before();
     __syncthreads();
     if (c->abort) abort = true;
+    // the tile's coarse histogram into the row's (every tile crowds the same
+    // few coarse bins: one add per bin and tile)
+    if (tid < kNB1) {
+      const uint32_t n = c->h1[tid];
+      if (n) {
+        atomicAdd(p.hist + b * kNB1 + tid, n);
+        c->h1[tid] = 0u;
+      }
+    }
+    __syncthreads();
     if (tid == 0) {
       const int un = u + 2 * p.G;  // the stage is free: fetch the unit after next
       if (un < p.n_score) {
@@ -292,24 +334,39 @@ __device__ void score_units(const FusedParams &p, const CUtensorMap *tm_keys, co
 }
 
 // ----------------------------------------------------------------- select
-// The selector runs once per launch on one SM, so its instructions come cold
-// from L2 or HBM: it is written as short rolled loops over the row's keys in
-// shared memory (not unrolled register arrays), which keeps the code small.
-// Thread t owns positions [t*items, t*items + items), the i-th of them at
-// key slot i*kThreads + t (consecutive threads, consecutive words: no bank
-// conflicts).
+// The k largest scores of a row are found by the score units together, with
+// one wait between them:
+//  * each score unit adds its tile's scores to two histograms of the row, of
+//    the order-preserving keys' top 11 bits (kNB bins) and top 16 bits
+//    (kNB2 bins; 32 fine bins under each coarse one), as it stores them;
+//  * once every tile is scored, each unit finds the same fine bin f holding
+//    the k-th largest key (coarse bin by a scan of the coarse histogram, then
+//    the fine bin among its 32), publishes how many of its keys lie above f,
+//    and appends its keys in f to the row's candidate list;
+//  * once every unit has published, anyone who needs the selection ranks the
+//    few candidates (key desc, index asc): the one of rank need-1 is the last
+//    taken, (T_key, T_idx).  Entry j with key kk is taken iff kk > T_key or
+//    (kk == T_key and j <= T_idx): keys above f exceed T_key, keys below f
+//    fall short of it.  The per-tile counts give each tile's offset in the
+//    ascending id list, so the attention units build their own chunks of it
+//    and the score units write the caller's ids, with no further wait.
+// When at most k keys are eligible all are taken.  A fine bin of more than
+// kCandSplit keys (long runs of ties) leaves the row to the selector unit,
+// which selects it alone (kModeOneCta).
 
-// value of an order-preserving key (the inverse of order_key for keys != 0)
-__device__ __forceinline__ float key_value(uint32_t k) {
-  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+// Bounded wait of the whole CTA for *w >= target; false (and abort) on expiry.
+__device__ __forceinline__ bool block_wait(const FusedParams &p, const uint32_t *w, uint32_t target, Ctl *c,
+                                           bool &abort) {
+  if (threadIdx.x == 0) c->bc[0] = wait_geq(w, target, p.wait_ns) ? 1u : 0u;
+  __syncthreads();
+  const bool ok = c->bc[0] != 0;
+  __syncthreads();  // bc[0] is reused
+  if (!ok) {
+    abort = true;
+    if (threadIdx.x == 0) raise_status(p.status, LIDX_DEV_TIMEOUT);
+  }
+  return ok;
 }
-
-struct SelView {
-  const uint32_t *key;  // [items][kThreads]
-  int items;
-  __device__ __forceinline__ uint32_t at(int i) const { return key[i * kThreads + threadIdx.x]; }
-  __device__ __forceinline__ int pos(int i) const { return static_cast<int>(threadIdx.x) * items + i; }
-};
 
 // block-wide min and max of (lo, hi) through the per-warp slots
 __device__ __forceinline__ void block_minmax(uint32_t &lo, uint32_t &hi, Ctl *c) {
@@ -321,17 +378,15 @@ __device__ __forceinline__ void block_minmax(uint32_t &lo, uint32_t &hi, Ctl *c)
     c->whi[warp] = hi;
   }
   __syncthreads();
-  lo = c->wlo[lane & (kWarps - 1)];
-  hi = c->whi[lane & (kWarps - 1)];
-  lo = __reduce_min_sync(0xFFFFFFFFu, lo);
-  hi = __reduce_max_sync(0xFFFFFFFFu, hi);
+  lo = __reduce_min_sync(0xFFFFFFFFu, c->wlo[lane & (kWarps - 1)]);
+  hi = __reduce_max_sync(0xFFFFFFFFu, c->whi[lane & (kWarps - 1)]);
   __syncthreads();  // the slots are reused
 }
 
 // Suffix scan of hist (thread t holds bins kNB-1-4t .. kNB-4-4t) to the bin
 // holding the need-th largest key: bc[2] = that bin, bc[3] = keys above it,
 // bc[4] = keys in it; returns the histogram's total.
-__device__ __noinline__ uint32_t find_bin(const uint32_t *hist, uint32_t need, Ctl *c) {
+__device__ __forceinline__ uint32_t find_bin(const uint32_t *hist, uint32_t need, Ctl *c) {
   const int tid = threadIdx.x;
   uint32_t cnt[4], ct = 0;
 #pragma unroll
@@ -356,67 +411,254 @@ __device__ __noinline__ uint32_t find_bin(const uint32_t *hist, uint32_t need, C
   return tot;
 }
 
-// Exact threshold: entry j (key kk) is selected iff kk > T_key or
-// (kk == T_key and j <= T_idx).  The level-0 histogram bins the scores
-// linearly in value over the row's [min, max] (keys of score-like data spread
-// over its bins); a bin too full for rank counting is refined in key space,
-// and a bin of one key value takes its first entries by index.
-__device__ __noinline__ void find_threshold(const SelView v, int k, uint32_t *hist, uint2 *cand, Ctl *c,
-                                            uint32_t &T_key, uint32_t &T_idx) {
+// Rank the nc candidates (key desc, index asc): bc[5], bc[6] = the key and
+// index of rank need-1, the last selected entry.  g threads (a power of two,
+// within a warp) share a candidate, each comparing it with every g-th other.
+__device__ __forceinline__ void rank_pick(const uint2 *cand, uint32_t nc, uint32_t need, Ctl *c) {
   const int tid = threadIdx.x;
-  T_key = 1u;  // default: every eligible key
-  T_idx = 0x7FFFFFFFu;
-  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
-#pragma unroll 4
-  for (int i = 0; i < v.items; i++) {
-    const uint32_t kk = v.at(i);
-    hi = max(hi, kk);
-    lo = kk ? min(lo, kk) : lo;
-  }
-  block_minmax(lo, hi, c);
-  if (hi == 0u) return;  // no eligible key
-  const float vlo = key_value(lo), vhi = key_value(hi);
-  const float range = vhi - vlo;
-  const float scale = static_cast<float>(kNB) / range;
-  const bool linear = hi > lo && isfinite(vlo) && isfinite(vhi) && isfinite(range) && range > 0.f && isfinite(scale);
-  const uint32_t krange = hi - lo;
-  const uint32_t s0 = krange < kNB ? 0u : static_cast<uint32_t>(32 - __clz(krange) - 11);
-  // level-0 bin of a key: linear in value, else the top bits of (key - lo)
-  auto bin0 = [&](uint32_t kk) -> uint32_t {
-    if (linear) return min(static_cast<uint32_t>(kNB - 1), static_cast<uint32_t>((key_value(kk) - vlo) * scale));
-    return (kk - lo) >> s0;
-  };
-#pragma unroll 4
-  for (int i = 0; i < v.items; i++) {
-    const uint32_t kk = v.at(i);
-    if (kk) atomicAdd(&hist[bin0(kk)], 1u);
-  }
-  __syncthreads();
-  if (find_bin(hist, static_cast<uint32_t>(k), c) <= static_cast<uint32_t>(k)) return;  // every eligible key
-  const uint32_t bin = c->bc[2];
-  uint32_t need = static_cast<uint32_t>(k) - c->bc[3];
-  uint32_t in_bin = c->bc[4];
-  // the keys of that bin form one interval [a, b] (the binning is monotone)
-  uint32_t a = 0xFFFFFFFFu, b = 0u;
-#pragma unroll 4
-  for (int i = 0; i < v.items; i++) {
-    const uint32_t kk = v.at(i);
-    if (kk && bin0(kk) == bin) {
-      a = min(a, kk);
-      b = max(b, kk);
+  uint32_t g = 1;
+  while (g < 32 && 2 * g * nc <= static_cast<uint32_t>(kThreads)) g *= 2;
+  const uint32_t per = static_cast<uint32_t>(kThreads) / g, sub = static_cast<uint32_t>(tid) % g;
+  for (uint32_t c0 = 0; c0 < nc; c0 += per) {
+    const uint32_t ci = c0 + static_cast<uint32_t>(tid) / g;
+    uint32_t rank = 0;
+    uint2 me = make_uint2(0u, 0u);
+    if (ci < nc) {
+      me = cand[ci];
+      for (uint32_t cj = sub; cj < nc; cj += g) {
+        const uint2 o = cand[cj];
+        rank += (o.x > me.x || (o.x == me.x && o.y < me.y)) ? 1u : 0u;
+      }
+    }
+    for (uint32_t o = g / 2; o; o >>= 1) rank += __shfl_xor_sync(0xFFFFFFFFu, rank, o);
+    if (ci < nc && sub == 0 && rank == need - 1) {
+      c->bc[5] = me.x;
+      c->bc[6] = me.y;
     }
   }
-  block_minmax(a, b, c);
-  // refine in key space over [a, b], 11 bits per level, until the bin is
-  // small enough to rank or holds one key value
+  __syncthreads();
+}
+
+// One warp: lane l holds the counts of bins [8l, 8l + 8) of a 256-bin
+// histogram (h, ascending).  Finds the bin holding the need-th largest key:
+// returns it, with the keys above it in `above` and in it in `in_bin`; the
+// histogram's total in `total` (the search needs need <= total).
+__device__ __forceinline__ uint32_t warp_find_bin(const uint32_t (&h)[8], uint32_t need, uint32_t &above,
+                                                  uint32_t &in_bin, uint32_t &total) {
+  const int lane = threadIdx.x & 31;
+  uint32_t ls = 0;
+#pragma unroll
+  for (int j = 0; j < 8; j++) ls += h[j];
+  uint32_t sfx = ls;  // keys in lanes >= this one
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_down_sync(0xFFFFFFFFu, sfx, o);
+    if (lane + o < 32) sfx += y;
+  }
+  uint32_t nxt = __shfl_down_sync(0xFFFFFFFFu, sfx, 1);
+  if (lane == 31) nxt = 0u;
+  total = __shfl_sync(0xFFFFFFFFu, sfx, 0);
+  uint32_t bin = 0, ab = nxt, in = 0;
+  bool hit = false;
+#pragma unroll
+  for (int j = 7; j >= 0; j--) {
+    if (!hit && ab + h[j] >= need) {
+      hit = true;
+      bin = 8 * lane + j;
+      in = h[j];
+    } else if (!hit) {
+      ab += h[j];
+    }
+  }
+  const uint32_t src = __ffs(__ballot_sync(0xFFFFFFFFu, sfx >= need && nxt < need)) - 1;
+  above = __shfl_sync(0xFFFFFFFFu, ab, src);
+  in_bin = __shfl_sync(0xFFFFFFFFu, in, src);
+  return __shfl_sync(0xFFFFFFFFu, bin, src);
+}
+
+// The candidate step, for each score unit of this CTA once every tile of its
+// row is scored (run after the CTA's last score unit, so the wait cannot hold
+// back a tile; every CTA takes its units in the same order).  Warp 0 finds
+// the coarse bin, then the fine bin f among the 256 under it.  The unit of
+// tile 0 also publishes the row's mode, need and "all taken" flag.  A unit
+// whose wait gave up still counts itself.
+__device__ void cand_units(const FusedParams &p, uint8_t *sm, Ctl *c, bool &abort) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  (void)sm;
+  for (int i = 0, u = blockIdx.x; u < p.n_score; i++, u += p.G) {
+    const int b = u / p.n_tiles, t = u % p.n_tiles;
+    uint32_t *ctl = p.ctl + b * kCtlStride;
+    const bool ok = block_wait(p, ctl + kCtlTiles, p.n_tiles, c, abort);
+    const uint32_t k = static_cast<uint32_t>(p.k);
+    if (warp == 0) {
+      uint32_t h[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+      if (ok) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(p.hist + b * kNB1 + 8 * lane);
+        const uint4 x0 = __ldcg(src), x1 = __ldcg(src + 1);
+        h[0] = x0.x, h[1] = x0.y, h[2] = x0.z, h[3] = x0.w, h[4] = x1.x, h[5] = x1.y, h[6] = x1.z, h[7] = x1.w;
+      }
+      uint32_t above1, in1, total;
+      uint32_t tot;
+      uint32_t lsum = 0;
+#pragma unroll
+      for (int j = 0; j < 8; j++) lsum += h[j];
+      tot = __reduce_add_sync(0xFFFFFFFFu, lsum);
+      const bool all = tot <= k;
+      uint32_t f = 0, need = 0, in2 = 0;
+      if (!all) {
+        const uint32_t cb = warp_find_bin(h, k, above1, in1, total);
+        const uint4 *src = reinterpret_cast<const uint4 *>(p.hist2 + static_cast<int64_t>(b) * kNB2 + cb * 256 + 8 * lane);
+        const uint4 x0 = __ldcg(src), x1 = __ldcg(src + 1);
+        uint32_t g[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+        uint32_t above2, t2;
+        const uint32_t need1 = k - above1;
+        f = cb * 256 + warp_find_bin(g, need1, above2, in2, t2);
+        need = need1 - above2;
+      }
+      if (lane == 0) {
+        c->bc[1] = all ? 1u : 0u;
+        c->bc[5] = f;
+        c->bc[6] = need;
+        c->bc[7] = in2;
+      }
+    }
+    __syncthreads();
+    const bool all = c->bc[1] != 0u;
+    const uint32_t f = c->bc[5], need = c->bc[6];
+    const bool split = all || c->bc[7] <= static_cast<uint32_t>(kCandSplit);
+    if (split) {
+      const float v = tid < kTileM ? c->tile_x[i][tid] : NAN;
+      const uint32_t kk = tid < kTileM ? order_key(v) : 0u;
+      const uint32_t fb = kk >> 16;
+      const bool up = kk != 0u && (all || fb > f), cd = !all && kk != 0u && fb == f;
+      // candidates: one slot range per warp
+      const uint32_t cm = __ballot_sync(0xFFFFFFFFu, cd);
+      uint32_t base = 0;
+      if (lane == 0 && cm) base = atomicAdd(ctl + kCtlCandN, static_cast<uint32_t>(__popc(cm)));
+      base = __shfl_sync(0xFFFFFFFFu, base, 0);
+      if (cd) {
+        const uint32_t slot = base + __popc(cm & ((1u << lane) - 1u));
+        if (slot < static_cast<uint32_t>(kCandSplit))
+          p.gcand[b * kCandSplit + slot] = make_uint2(kk, static_cast<uint32_t>(t * kTileM + tid));
+      }
+      const uint32_t um = __ballot_sync(0xFFFFFFFFu, up);
+      if (lane == 0) c->wsum[warp] = __popc(um);
+    }
+    __syncthreads();
+    if (tid == 0) {
+      if (split) {
+        uint32_t n = 0;
+        for (int w = 0; w < kTileM / 32; w++) n += c->wsum[w];
+        p.above[u] = n;
+      }
+      if (t == 0) {  // ordered before the count by its fence
+        ctl[kCtlMode] = split ? kModeSplit : kModeOneCta;
+        ctl[kCtlNeed] = need;
+        ctl[kCtlAll] = all ? 1u : 0u;
+      }
+      arrive_release(ctl + kCtlCand);
+    }
+    __syncthreads();
+  }
+}
+
+// After the candidate step of row b (split mode): the threshold (T_key,
+// T_idx), and per tile the offset of its first taken entry in the ascending
+// id list (c->toff[0 .. n_tiles], the last being the number taken).  Every
+// thread of the CTA calls it; the control words, the tiles' counts and the
+// candidate slots are read in one round trip.  It uses the split scratch
+// area of shared memory.
+__device__ void split_view(const FusedParams &p, int b, uint8_t *sm, Ctl *c, uint32_t &T_key, uint32_t &T_idx) {
+  const int tid = threadIdx.x;
+  uint2 *cand = reinterpret_cast<uint2 *>(sm + kSmSplit);
+  const uint32_t *ctl = p.ctl + b * kCtlStride;
+  if (tid == 0) {
+    const uint4 w8 = __ldcg(reinterpret_cast<const uint4 *>(ctl + 8)), w12 = __ldcg(reinterpret_cast<const uint4 *>(ctl + 12));
+    c->bc[1] = min(w8.z, static_cast<uint32_t>(kCandSplit));  // kCtlCandN
+    c->bc[2] = w12.x;                                          // kCtlNeed
+    c->bc[3] = w12.y;                                          // kCtlAll
+  }
+  const uint32_t av = tid < p.n_tiles ? __ldcg(p.above + b * p.n_tiles + tid) : 0u;
+  if (tid < kCandSplit) cand[tid] = __ldcg(p.gcand + b * kCandSplit + tid);  // slots past the count are unused
+  // the row's scores into L1 while the candidates are ranked (chunk_rows reads its tiles)
+  for (int q = 32 * tid; q < p.N; q += 32 * kThreads)
+    asm volatile("prefetch.global.L1 [%0];" ::"l"(p.scores + static_cast<int64_t>(b) * p.ld_ws + q));
+  for (int q = tid; q < p.n_tiles; q += kThreads) c->ctile[q] = 0u;
+  __syncthreads();
+  const bool all = c->bc[3] != 0u;
+  const uint32_t nc = all ? 0u : c->bc[1];
+  T_key = 1u;  // all taken: every eligible key
+  T_idx = 0xFFFFFFFFu;
+  if (!all) {
+    rank_pick(cand, nc, c->bc[2], c);
+    T_key = c->bc[5];
+    T_idx = c->bc[6];
+    if (tid < static_cast<int>(nc)) {
+      const uint2 cd = cand[tid];
+      if (cd.x > T_key || (cd.x == T_key && cd.y <= T_idx)) atomicAdd(&c->ctile[cd.y / kTileM], 1u);
+    }
+    __syncthreads();
+  }
+  const uint32_t cnt = tid < p.n_tiles ? av + c->ctile[tid] : 0u;
+  uint32_t total;
+  const uint32_t off = block_excl_scan(cnt, total, c);
+  if (tid < p.n_tiles) c->toff[tid] = off;
+  if (tid == 0) c->toff[p.n_tiles] = total;
+  __syncthreads();
+}
+
+// Entry j with key kk is taken
+__device__ __forceinline__ bool taken_key(uint32_t kk, uint32_t j, uint32_t T_key, uint32_t T_idx) {
+  return kk != 0u && (kk > T_key || (kk == T_key && j <= T_idx));
+}
+
+// The selector unit clears the row's histogram bins for the next call, once
+// every score unit has read them (the candidate step is complete): it reads
+// the row's scores back and zeroes the bins of their keys.
+__device__ void clear_row(const FusedParams &p, int b) {
+  const float *row = p.scores + static_cast<int64_t>(b) * p.ld_ws;
+  for (int q = 4 * threadIdx.x; q < p.N; q += 4 * kThreads) {
+    const float4 v = __ldcg(reinterpret_cast<const float4 *>(row + q));  // the row is padded to 4 scores
+    const float f[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 4; e++) {
+      const uint32_t kk = q + e < p.N ? order_key(f[e]) : 0u;
+      if (kk) {
+        p.hist[b * kNB1 + (kk >> 24)] = 0u;
+        p.hist2[static_cast<int64_t>(b) * kNB2 + (kk >> 16)] = 0u;
+      }
+    }
+  }
+}
+
+// Key-space threshold search of the selector unit over its register keys x
+// (NaN = not eligible), starting from the row's key range [a, b]: 11 bits a
+// level until the interval is small enough to rank or holds one key value,
+// which then takes its first entries by index.  Every branch is uniform over
+// the block.
+__device__ __forceinline__ void find_threshold(const float (&x)[kSelItems], uint32_t a, uint32_t b, int k,
+                                               uint32_t *hist, uint2 *cand, Ctl *c, uint32_t &T_key,
+                                               uint32_t &T_idx) {
+  const int tid = threadIdx.x;
+  const int pos0 = tid * kSelItems;
+  uint32_t need = static_cast<uint32_t>(k), in_bin = 0;
+  T_key = 1u;  // every eligible key (when at most k are)
+  T_idx = 0xFFFFFFFFu;
+  {
+    uint32_t n = 0;
+#pragma unroll
+    for (int i = 0; i < kSelItems; i++) n += order_key(x[i]) ? 1u : 0u;
+    block_excl_scan(n, in_bin, c);
+    if (in_bin <= need) return;
+  }
   uint32_t s = (b - a) < kNB ? 0u : static_cast<uint32_t>(32 - __clz(b - a) - 11);
   for (int level = 0; level < 3 && in_bin > static_cast<uint32_t>(kCandMax) && b > a; level++) {
     for (int i = tid; i < kNB; i += kThreads) hist[i] = 0u;
     __syncthreads();
     const uint32_t base = a;
-#pragma unroll 4
-    for (int i = 0; i < v.items; i++) {
-      const uint32_t kk = v.at(i);
+#pragma unroll
+    for (int i = 0; i < kSelItems; i++) {
+      const uint32_t kk = order_key(x[i]);
       if (kk >= a && kk <= b) atomicAdd(&hist[(kk - base) >> s], 1u);
     }
     __syncthreads();
@@ -431,13 +673,14 @@ __device__ __noinline__ void find_threshold(const SelView v, int k, uint32_t *hi
   if (in_bin > static_cast<uint32_t>(kCandMax)) {
     // one key value: take its first `need` entries by index
     uint32_t tie = 0;
-#pragma unroll 4
-    for (int i = 0; i < v.items; i++) tie += v.at(i) == a ? 1u : 0u;
+#pragma unroll
+    for (int i = 0; i < kSelItems; i++) tie += order_key(x[i]) == a ? 1u : 0u;
     uint32_t tt;
     uint32_t te = block_excl_scan(tie, tt, c);
-    for (int i = 0; i < v.items; i++) {
-      if (v.at(i) == a) {
-        if (te == need - 1) c->bc[6] = static_cast<uint32_t>(v.pos(i));
+#pragma unroll
+    for (int i = 0; i < kSelItems; i++) {
+      if (order_key(x[i]) == a) {
+        if (te == need - 1) c->bc[6] = static_cast<uint32_t>(pos0 + i);
         te++;
       }
     }
@@ -446,98 +689,91 @@ __device__ __noinline__ void find_threshold(const SelView v, int k, uint32_t *hi
     T_idx = c->bc[6];
     return;
   }
-  // rank the candidates (key desc, index asc); the one of rank need-1 is the
-  // last selected
   if (tid == 0) c->bc[1] = 0u;
   __syncthreads();
-  for (int i = 0; i < v.items; i++) {
-    const uint32_t kk = v.at(i);
+#pragma unroll
+  for (int i = 0; i < kSelItems; i++) {
+    const uint32_t kk = order_key(x[i]);
     if (kk >= a && kk <= b && kk) {
       const uint32_t slot = atomicAdd(&c->bc[1], 1u);
-      if (slot < kCandMax) cand[slot] = make_uint2(kk, static_cast<uint32_t>(v.pos(i)));
+      if (slot < kCandMax) cand[slot] = make_uint2(kk, static_cast<uint32_t>(pos0 + i));
     }
   }
   __syncthreads();
-  const uint32_t nc = min(c->bc[1], static_cast<uint32_t>(kCandMax));
-  for (uint32_t ci = tid; ci < nc; ci += kThreads) {
-    const uint2 me = cand[ci];
-    uint32_t rank = 0;
-    for (uint32_t cj = 0; cj < nc; cj++) {
-      const uint2 o = cand[cj];
-      rank += (o.x > me.x || (o.x == me.x && o.y < me.y)) ? 1u : 0u;
-    }
-    if (rank == need - 1) {
-      c->bc[5] = me.x;
-      c->bc[6] = me.y;
-    }
-  }
-  __syncthreads();
+  rank_pick(cand, min(c->bc[1], static_cast<uint32_t>(kCandMax)), need, c);
   T_key = c->bc[5];
   T_idx = c->bc[6];
 }
 
+// padded shared-memory word of row position q
+__device__ __forceinline__ int sel_pad(int q) { return q + (q >> 5) * 4; }
+
+// The selector unit of row b: waits for the candidate step; in split mode
+// the row is the score units' already.  Otherwise it selects the row alone:
+// thread t owns positions [t*kSelItems, +kSelItems) and keeps their scores
+// in registers.  The row is staged through shared memory by coalesced
+// 16-byte loads, stored with 4 pad words after every 32 scores, so each
+// thread then reads its 32 consecutive scores as 8 conflict-free loads.
 __device__ __noinline__ void select_unit(const FusedParams &p, int b, uint8_t *sm, Ctl *c, bool &abort) {
   const int tid = threadIdx.x;
-  const int items = p.items;
   uint32_t *hist = reinterpret_cast<uint32_t *>(sm + kSmHist);
   uint2 *cand = reinterpret_cast<uint2 *>(sm + kSmCand);
-  uint32_t *skey = reinterpret_cast<uint32_t *>(sm + kSmRow);
+  float *srow = reinterpret_cast<float *>(sm + kSmRow);
   uint32_t *ctl = p.ctl + b * kCtlStride;
-  for (int i = tid; i < kNB; i += kThreads) hist[i] = 0u;
-  if (tid == 0) c->bc[0] = wait_geq(ctl + kCtlTiles, p.n_tiles, p.wait_ns) ? 1u : 0u;
-  __syncthreads();
-  if (!c->bc[0]) {
-    abort = true;
-    if (tid == 0) raise_status(p.status, LIDX_DEV_TIMEOUT);
-  }
-  // this thread's positions [tid*items, +items): float4 loads, then one key
-  // per slot; NaN and positions beyond N get key 0 (never selected)
-  const SelView v{skey, items};
-  const int p0 = tid * items;
+  const bool ok = block_wait(p, ctl + kCtlCand, p.n_tiles, c, abort);
+  clear_row(p, b);
+  if (ok && __ldcg(ctl + kCtlMode) == kModeSplit) return;
+  // stage the row: chunk j*kThreads + tid holds positions 4*chunk .. +3 (the
+  // workspace row is padded to a multiple of 4 scores)
   const float *row = p.scores + static_cast<int64_t>(b) * p.ld_ws;
-  bool nan = false;
-#pragma unroll 2
-  for (int i = 0; i < items; i += 4) {
-    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (p0 + i < p.N) x = __ldcg(reinterpret_cast<const float4 *>(row + p0 + i));
-    const float f[4] = {x.x, x.y, x.z, x.w};
+  {
+    float4 v[kSelItems / 4];
 #pragma unroll
-    for (int e = 0; e < 4; e++) {
-      const bool in = p0 + i + e < p.N;
-      const uint32_t kk = in ? order_key(f[e]) : 0u;
-      nan |= in && kk == 0u;
-      skey[(i + e) * kThreads + tid] = kk;
+    for (int j = 0; j < kSelItems / 4; j++) {
+      const int q = 4 * (j * kThreads + tid);
+      v[j] = ok && q < p.N ? __ldcg(reinterpret_cast<const float4 *>(row + q)) : make_float4(NAN, NAN, NAN, NAN);
+    }
+#pragma unroll
+    for (int j = 0; j < kSelItems / 4; j++) {
+      const int q = 4 * (j * kThreads + tid);
+      *reinterpret_cast<float4 *>(srow + sel_pad(q)) = v[j];
     }
   }
-  if (nan) raise_status(p.status, LIDX_DEV_NAN);
   __syncthreads();
-  uint32_t T_key, T_idx;
-  find_threshold(v, p.k, hist, cand, c, T_key, T_idx);
-  // emit ids ascending: entry j is taken when key > T or (key == T and j <= T_idx)
-  auto taken = [&](int i) {
-    const uint32_t kk = v.at(i);
-    return kk != 0u && (kk > T_key || (kk == T_key && static_cast<uint32_t>(v.pos(i)) <= T_idx));
-  };
-  uint32_t mine = 0;
-#pragma unroll 4
-  for (int i = 0; i < items; i++) mine += taken(i) ? 1u : 0u;
+  // this thread's scores; positions beyond N become NaN (never selected)
+  const int pos0 = tid * kSelItems;
+  float x[kSelItems];
+  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+#pragma unroll
+  for (int q = 0; q < kSelItems / 4; q++) {
+    const float4 v = *reinterpret_cast<const float4 *>(srow + sel_pad(pos0 + 4 * q));
+    const float f[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 4; e++) {
+      x[4 * q + e] = pos0 + 4 * q + e < p.N ? f[e] : NAN;
+      const uint32_t kk = order_key(x[4 * q + e]);
+      hi = max(hi, kk);
+      lo = kk ? min(lo, kk) : lo;
+    }
+  }
+  block_minmax(lo, hi, c);
+  uint32_t T_key = 0xFFFFFFFFu, T_idx = 0u;  // no eligible key: nothing is taken
+  if (hi) find_threshold(x, lo, hi, p.k, hist, cand, c, T_key, T_idx);
+  // emit ids ascending
+  uint32_t mask = 0;
+#pragma unroll
+  for (int i = 0; i < kSelItems; i++)
+    mask |= (taken_key(order_key(x[i]), static_cast<uint32_t>(pos0 + i), T_key, T_idx) ? 1u : 0u) << i;
   uint32_t n_out;
-  uint32_t pos = block_excl_scan(mine, n_out, c);
+  uint32_t pos = block_excl_scan(__popc(mask), n_out, c);
   const int k = p.k;
   int32_t *sel = p.sel_ids + static_cast<int64_t>(b) * k;
   int32_t *uid = p.ids_user ? p.ids_user + static_cast<int64_t>(b) * k : nullptr;
-  for (int i = 0; i < items && mine; i++) {
-    if (!taken(i)) continue;
-    mine--;
-    if (pos < static_cast<uint32_t>(k)) {
-      const int j = v.pos(i);
-      sel[pos] = j;
-      if (uid) uid[pos] = j;
-      // start the row's trip from HBM now: the attention units gather it
-      // from L2 once the ready flag reaches them
-      prefetch_l2(p.kv + (static_cast<int64_t>(b) * p.kv_batch_rows + j) * p.kv_ld, kD * 2);
-    }
-    pos++;
+  for (; mask && pos < static_cast<uint32_t>(k); pos++) {
+    const int j = pos0 + __ffs(mask) - 1;
+    mask &= mask - 1u;
+    sel[pos] = j;
+    if (uid) uid[pos] = j;
   }
   const int n_sel = static_cast<int>(min(n_out, static_cast<uint32_t>(k)));
   if (uid)
@@ -547,10 +783,57 @@ __device__ __noinline__ void select_unit(const FusedParams &p, int b, uint8_t *s
     if (p.n_sel_user) p.n_sel_user[b] = n_sel;
   }
   __syncthreads();
-  if (tid == 0) arrive_release(ctl + kCtlReady);
+  if (tid == 0) arrive_release(ctl + kCtlReady, static_cast<uint32_t>(p.n_tiles));
 }
 
 // -------------------------------------------------------------- attention
+// The ids at positions [s0, s1) of row b's ascending selected list (split
+// mode, after split_view): the tiles holding them are read back from the
+// workspace scores, one tile per warp, and their taken entries ranked in
+// position order.  c->chunk_id[q - s0] = the id at position q.
+__device__ void chunk_rows(const FusedParams &p, int b, int s0, int s1, uint32_t T_key, uint32_t T_idx, Ctl *c) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (s0 < s1) {
+    // the tiles holding positions s0 and s1 - 1
+    for (int t = tid; t < p.n_tiles; t += kThreads) {
+      const uint32_t a = c->toff[t], e = c->toff[t + 1];
+      if (a <= static_cast<uint32_t>(s0) && static_cast<uint32_t>(s0) < e) c->bc[1] = t;
+      if (a < static_cast<uint32_t>(s1) && static_cast<uint32_t>(s1) <= e) c->bc[2] = t;
+    }
+    __syncthreads();
+    const int t0 = static_cast<int>(c->bc[1]), t1 = static_cast<int>(c->bc[2]);
+    const float *row = p.scores + static_cast<int64_t>(b) * p.ld_ws;
+    for (int t = t0 + warp; t <= t1; t += kWarps) {
+      const int j0 = t * kTileM + 4 * lane;
+      float4 v = make_float4(NAN, NAN, NAN, NAN);
+      if (j0 < p.N) v = *reinterpret_cast<const float4 *>(row + j0);  // the row is padded to 4 scores; in L1
+      const float f[4] = {v.x, v.y, v.z, v.w};
+      uint32_t bits = 0;
+#pragma unroll
+      for (int e = 0; e < 4; e++) {
+        const uint32_t kk = j0 + e < p.N ? order_key(f[e]) : 0u;
+        bits |= (taken_key(kk, static_cast<uint32_t>(j0 + e), T_key, T_idx) ? 1u : 0u) << e;
+      }
+      const uint32_t n = __popc(bits);
+      uint32_t x = n;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+        if (lane >= o) x += y;
+      }
+      uint32_t g = c->toff[t] + x - n;  // this lane's first position
+#pragma unroll
+      for (int e = 0; e < 4; e++) {
+        if (bits >> e & 1u) {
+          if (g >= static_cast<uint32_t>(s0) && g < static_cast<uint32_t>(s1)) c->chunk_id[g - s0] = j0 + e;
+          g++;
+        }
+      }
+    }
+  }
+  __syncthreads();
+}
+
 __device__ void attn_unit(const FusedParams &p, int a, const CUtensorMap *tm_qa, const CUtensorMap *tm_win,
                           uint8_t *sm, Ctl *c, uint32_t tmem, bool &abort) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -581,20 +864,35 @@ __device__ void attn_unit(const FusedParams &p, int a, const CUtensorMap *tm_qa,
   __syncthreads();
   if (!pure_window) {
     // window rows of a mixed chunk, then the selected rows once they are known
-    if (tid == 0) c->bc[0] = wait_geq(p.ctl + b * kCtlStride + kCtlReady, 1u, p.wait_ns) ? 1u : 0u;
     for (int r = warp; r < kRows; r += kWarps) {
       if (c->row_kind[r] != 2) continue;
       const uint16_t *src = p.swa + c->row_src[r] * p.swa_ld;
       cp_async16(xs + x_off(r, lane), src + lane * 8);
       cp_async16(xs + x_off(r, lane + 32), src + (lane + 32) * 8);
     }
-    __syncthreads();
-    const bool ready = c->bc[0] != 0;
-    if (!ready) {
-      abort = true;
-      if (tid == 0) raise_status(p.status, LIDX_DEV_TIMEOUT);
+    const uint32_t *ctl = p.ctl + b * kCtlStride;
+    const bool ok = block_wait(p, ctl + kCtlCand, p.n_tiles, c, abort);
+    const bool split = ok && __ldcg(ctl + kCtlMode) == kModeSplit;  // uniform over the CTA
+    int n_b = 0;
+    const int s0 = max(0, i0 - swa_len);  // the chunk's first position in the selected list
+    if (split) {
+      uint32_t T_key, T_idx;
+      split_view(p, b, sm, c, T_key, T_idx);
+      n_b = static_cast<int>(min(c->toff[p.n_tiles], static_cast<uint32_t>(p.k)));
+      chunk_rows(p, b, s0, min(n_b, i0 + kRows - swa_len), T_key, T_idx, c);
+      if (hg == 0) {  // the caller's ids at this chunk's list positions (-1 past the count)
+        const int q1 = min(p.k, i0 + kRows - swa_len);
+        if (p.ids_user)
+          for (int q = s0 + tid; q < q1; q += kThreads)
+            p.ids_user[static_cast<int64_t>(b) * p.k + q] = q < n_b ? c->chunk_id[q - s0] : -1;
+        if (s0 == 0 && tid == 0) {
+          p.sel_n[b] = n_b;
+          if (p.n_sel_user) p.n_sel_user[b] = n_b;
+        }
+      }
+    } else if (ok && block_wait(p, ctl + kCtlReady, static_cast<uint32_t>(p.n_tiles), c, abort)) {
+      n_b = __ldcg(p.sel_n + b);  // the selector unit's list
     }
-    const int n_b = ready ? __ldcg(p.sel_n + b) : 0;
     // warp w gathers rows w + 16j; lane j resolves row w + 16j
     constexpr int kPerWarp = kRows / kWarps;
     int kind = 0;
@@ -605,7 +903,7 @@ __device__ void attn_unit(const FusedParams &p, int a, const CUtensorMap *tm_qa,
       src = c->row_src[r];
       const int i = i0 + r - swa_len;
       if (kind == 0 && i >= 0 && i < n_b) {
-        const int id = __ldcg(p.sel_ids + static_cast<int64_t>(b) * p.k + i);
+        const int id = split ? c->chunk_id[i - s0] : __ldcg(p.sel_ids + static_cast<int64_t>(b) * p.k + i);
         if (id >= 0 && id < p.N) {
           kind = 1;
           src = static_cast<int64_t>(b) * p.kv_batch_rows + id;
@@ -779,25 +1077,31 @@ __device__ void attn_unit(const FusedParams &p, int a, const CUtensorMap *tm_qa,
   }
   constexpr int kF4 = kHG * kD / 4;  // float4 outputs of the group
   const int f0 = ch * kF4 / p.n_chunks, f1 = (ch + 1) * kF4 / p.n_chunks;
-  for (int f = f0 + tid; f < f1; f += kThreads) {
+  // two threads per output: each folds every other partial (all of its loads
+  // in one round for up to 16 chunks), then the pair combines
+  const int par = tid & 1;
+  for (int fb = f0; fb < f1; fb += kThreads / 2) {
+    const int f = fb + tid / 2;
+    const bool act = f < f1;
     const int h = f / (kD / 4), d4 = f % (kD / 4);
     const int head = hg * kHG + h;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     float M = -INFINITY, L = 0.f;
-    for (int s0 = 0; s0 < p.n_chunks; s0 += 8) {
+    for (int s0 = par; act && s0 < p.n_chunks; s0 += 16) {
       float2 ml[8];
       float4 v[8];
 #pragma unroll
       for (int q = 0; q < 8; q++) {
-        if (s0 + q < p.n_chunks) {
-          const size_t base = (static_cast<size_t>(b) * p.n_chunks + s0 + q) * kHA + head;
+        ml[q] = make_float2(-INFINITY, 0.f);
+        if (s0 + 2 * q < p.n_chunks) {
+          const size_t base = (static_cast<size_t>(b) * p.n_chunks + s0 + 2 * q) * kHA + head;
           ml[q] = __ldcg(p.part_ml + base);
           v[q] = __ldcg(reinterpret_cast<const float4 *>(p.part_o + base * kD) + d4);
         }
       }
 #pragma unroll
       for (int q = 0; q < 8; q++) {
-        if (s0 + q < p.n_chunks && ml[q].x != -INFINITY) {
+        if (ml[q].x != -INFINITY) {
           const float mn = fmaxf(M, ml[q].x);
           const float cf = exp2f(M - mn);
           const float e = exp2f(ml[q].x - mn);
@@ -810,6 +1114,16 @@ __device__ void attn_unit(const FusedParams &p, int a, const CUtensorMap *tm_qa,
         }
       }
     }
+    // the pair's two folds
+    const float Mo = __shfl_xor_sync(0xFFFFFFFFu, M, 1), Lo = __shfl_xor_sync(0xFFFFFFFFu, L, 1);
+    const float ax = __shfl_xor_sync(0xFFFFFFFFu, acc.x, 1), ay = __shfl_xor_sync(0xFFFFFFFFu, acc.y, 1);
+    const float az = __shfl_xor_sync(0xFFFFFFFFu, acc.z, 1), aw = __shfl_xor_sync(0xFFFFFFFFu, acc.w, 1);
+    if (!act || par) continue;
+    const float mn = fmaxf(M, Mo);
+    const float c0 = M == -INFINITY ? 0.f : exp2f(M - mn), c1 = Mo == -INFINITY ? 0.f : exp2f(Mo - mn);
+    L = L * c0 + Lo * c1;
+    acc = make_float4(acc.x * c0 + ax * c1, acc.y * c0 + ay * c1, acc.z * c0 + az * c1, acc.w * c0 + aw * c1);
+    M = mn;
     const float il = L > 0.f ? 1.f / L : 0.f;
     reinterpret_cast<float4 *>(p.out + (static_cast<size_t>(b) * kHA + head) * kD)[d4] =
         make_float4(acc.x * il, acc.y * il, acc.z * il, acc.w * il);
@@ -822,7 +1136,7 @@ __device__ void attn_unit(const FusedParams &p, int a, const CUtensorMap *tm_qa,
 __global__ void __launch_bounds__(kThreads, 1)
     decode_fused_kernel(const __grid_constant__ CUtensorMap tm_keys, const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_qa, const __grid_constant__ CUtensorMap tm_win,
-                        const FusedParams p) {
+                        const __grid_constant__ FusedParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Ctl *c = reinterpret_cast<Ctl *>(sm + kSmData);
@@ -851,6 +1165,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   if (warp == 1) tc::tmem_alloc(&c->tmem_base, kTmemCols);
+  for (int i = tid; i < kNB1; i += kThreads) c->h1[i] = 0u;
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
@@ -870,6 +1185,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         prefetch_l2(p.pf[r] + o, static_cast<uint32_t>(s1 - o < 4096 ? s1 - o : 4096));
     }
   }
+  cand_units(p, sm, c, abort);
   // select units
   for (int u = blockIdx.x + ((p.n_score - static_cast<int>(blockIdx.x) + p.G - 1) / p.G) * p.G;
        u < p.n_score + p.B; u += p.G) {
@@ -893,16 +1209,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem, kTmemCols);
   }
+  // the last CTA to leave zeroes the control words for the next call
   if (tid == 0) {
     if (c->abort) raise_status(p.status, LIDX_DEV_TIMEOUT);
-    // the last CTA to leave zeroes the control words for the next call
-    uint32_t *exit_cnt = p.ctl + p.B * kCtlStride;
     uint32_t prev;
-    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(prev) : "l"(exit_cnt) : "memory");
-    if (prev == static_cast<uint32_t>(p.G - 1)) {
-      for (int i = 0; i < p.B * kCtlStride; i++) p.ctl[i] = 0u;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(prev) : "l"(p.ctl + p.B * kCtlStride) : "memory");
+    c->bc[0] = prev == static_cast<uint32_t>(p.G - 1) ? 1u : 0u;
+  }
+  __syncthreads();
+  if (c->bc[0]) {
+    for (int i = tid; i < p.B * kCtlStride; i += kThreads) p.ctl[i] = 0u;
+    // after a wait gave up, a histogram may hold counts nobody cleared
+    if (ld_acquire(p.status) & LIDX_DEV_TIMEOUT) {
+      for (int i = tid; i < p.B * kNB1; i += kThreads) p.hist[i] = 0u;
+      for (int64_t i = tid; i < static_cast<int64_t>(p.B) * kNB2; i += kThreads) p.hist2[i] = 0u;
+    }
+    __syncthreads();
+    if (tid == 0) {
       __threadfence();
-      *exit_cnt = 0u;
+      p.ctl[p.B * kCtlStride] = 0u;
     }
   }
   (void)abort;
@@ -920,14 +1245,8 @@ int n_chunks(const lidx_decode_args &a) {
   return rows > 0 ? (rows + kRows - 1) / kRows : 1;
 }
 
-int items_for(int N) {
-  int it = 4;
-  while (it * kThreads < N) it <<= 1;
-  return it;
-}
-
 struct WsLayout {
-  size_t ctl, sel_ids, sel_n, part_ml, part_o, scores, total;
+  size_t ctl, sel_ids, sel_n, part_ml, part_o, scores, hist, hist2, above, gcand, total;
   int64_t ld_ws;
 };
 
@@ -949,6 +1268,14 @@ WsLayout ws_layout(const lidx_decode_args &a) {
   o += up(static_cast<size_t>(a.B) * nc * kHA * kD * 4);
   l.scores = o;
   o += up(static_cast<size_t>(a.B) * l.ld_ws * 4);
+  l.hist = o;
+  o += up(static_cast<size_t>(a.B) * kNB1 * 4);
+  l.hist2 = o;
+  o += up(static_cast<size_t>(a.B) * kNB2 * 4);
+  l.above = o;
+  o += up(static_cast<size_t>(a.B) * ((a.N + kTileM - 1) / kTileM) * 4);
+  l.gcand = o;
+  o += up(static_cast<size_t>(a.B) * kCandSplit * 8);
   l.total = o;
   return l;
 }
@@ -959,8 +1286,11 @@ bool decode_fused_supported(const lidx_decode_args &a) {
   if (a.keys.dtype != LIDX_BF16 || a.kv.dtype != LIDX_BF16) return false;
   if (a.swa_len > 0 && a.swa.dtype != LIDX_BF16) return false;
   if (a.H % 32 != 0 || a.H > 128 || a.H_attn != kHA) return false;
-  if (a.N > 64 * kThreads) return false;
+  if (a.N > kSelItems * kThreads) return false;
   if (static_cast<int64_t>(a.B) * n_chunks(a) * 4 > sm_count()) return false;
+  const int64_t n_score = static_cast<int64_t>(a.B) * ((a.N + kTileM - 1) / kTileM);
+  const int64_t G = std::min<int64_t>(sm_count(), n_score + a.B + static_cast<int64_t>(a.B) * n_chunks(a) * 4);
+  if (n_score > kMaxOwnTiles * G) return false;
   const int64_t rows = static_cast<int64_t>(a.B - 1) * (a.B > 1 ? a.keys.batch_rows : a.N) + a.N;
   return rows < (1ll << 31);
 }
@@ -981,7 +1311,6 @@ cudaError_t launch_decode_fused(const lidx_decode_args &a, void *ws, cudaStream_
   p.n_score = a.B * p.n_tiles;
   p.n_attn = a.B * p.n_chunks * 4;
   p.G = std::min(sm_count(), p.n_score + a.B + p.n_attn);
-  p.items = items_for(a.N);
   p.key_batch_rows = a.B > 1 ? a.keys.batch_rows : a.N;
   p.w = a.w;
   p.kv = static_cast<const uint16_t *>(a.kv.data);
@@ -1005,6 +1334,10 @@ cudaError_t launch_decode_fused(const lidx_decode_args &a, void *ws, cudaStream_
   p.part_o = reinterpret_cast<float *>(w8 + l.part_o);
   p.scores = reinterpret_cast<float *>(w8 + l.scores);
   p.ld_ws = l.ld_ws;
+  p.hist2 = reinterpret_cast<uint32_t *>(w8 + l.hist2);
+  p.hist = reinterpret_cast<uint32_t *>(w8 + l.hist);
+  p.above = reinterpret_cast<uint32_t *>(w8 + l.above);
+  p.gcand = reinterpret_cast<uint2 *>(w8 + l.gcand);
   for (int r = 0; r < 2; r++) {
     p.pf[r] = static_cast<const uint8_t *>(a.prefetch[r]);
     p.pf_bytes[r] = a.prefetch[r] ? a.prefetch_bytes[r] : 0;

@@ -69,11 +69,21 @@ def _check_against_oracle(spec, x, res, swa_len):
     (synth.scaled(synth.DECODE_64K, N=1000, k=64, B=3, H=32), 77),
     (synth.scaled(synth.DECODE_64K, N=300, k=512), 128),
     (synth.scaled(synth.DECODE_64K, N=777, k=100, H=128), 0),
-    (synth.scaled(synth.DECODE_64K, N=20000, k=512), 128),
+    (synth.scaled(synth.DECODE_64K, N=16383, k=512), 128),
 ], ids=lambda x: f"{x.name}-N{x.N}-B{x.B}-H{x.H}-k{x.k}" if hasattr(x, "name") else f"swa{x}")
 def test_fused_layer_parity(cuda_device, spec, swa_len):
     x, d = _inputs(spec)
     _check_against_oracle(spec, x, _run(spec, d, swa_len), swa_len)
+
+
+def test_fused_layer_rejects_rows_beyond_one_selector(cuda_device):
+    """One CTA selects a row of at most 16384 entries: a longer row is
+    LIDX_ERR_UNSUPPORTED (the three-call layer takes it), before any launch."""
+    spec = synth.scaled(synth.DECODE_64K, N=16385, k=512)
+    x, d = _inputs(spec)
+    with pytest.raises(L.LidxError) as e:
+        _run(spec, d, 128)
+    assert e.value.status == L.ERR_UNSUPPORTED
 
 
 def test_fused_layer_full_size_64k(cuda_device):
