@@ -195,7 +195,7 @@ class ClockSampler:
             os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                                          "-i", str(self.gpu), "-lms", "100"], stdout=self.f,
+                                          "-i", str(self.gpu), "-lms", "20"], stdout=self.f,
                                          stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
@@ -349,7 +349,7 @@ def host_queries(spec, layers_inp):
     return q_idx, w, q_attn
 
 
-def measure_decode(args, name, spec, world, dist, device, local_rank, rank, want_cpu) -> dict:
+def measure_decode(args, name, spec, world, dist, device, local_rank, rank, want_cpu, form=None) -> dict:
     """The stack of CSA layers: R cache replicas rotated so each step reads
     from HBM (R x step bytes >= 4 x L2), captured as CUDA graphs."""
     import torch
@@ -359,7 +359,7 @@ def measure_decode(args, name, spec, world, dist, device, local_rank, rank, want
     ab = algorithmic_bytes(spec)
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
     R = max(2, math.ceil(4 * l2 / ab["step"]))
-    steps = make_replica_steps(spec, layers_inp, R, device, fused=LAYER_FORMS[args.layer_form])
+    steps = make_replica_steps(spec, layers_inp, R, device, fused=form)
     q_idx_h, w_h, q_attn_h = host_queries(spec, layers_inp)
     for s in steps:
         s.set_inputs(q_idx_h.to(device), w_h.to(device), q_attn_h.to(device))
@@ -451,6 +451,29 @@ def measure_decode(args, name, spec, world, dist, device, local_rank, rank, want
     del steps
     torch.cuda.empty_cache()
     return res
+
+
+def decode_forms(args, name, spec, world, dist, device, local_rank, rank, want_cpu) -> dict:
+    """--layer-form auto: where the one-launch layer covers the shape, time
+    both layer forms and report the faster (both values under layer_forms)."""
+    import lightning_indexer_top_index_b200 as L
+    if args.layer_form != "auto":
+        return measure_decode(args, name, spec, world, dist, device, local_rank, rank, want_cpu,
+                              form=LAYER_FORMS[args.layer_form])
+    try:
+        fused = measure_decode(args, name, spec, world, dist, device, local_rank, rank, False, form=True)
+    except L.LidxError as e:
+        if e.status != L.ERR_UNSUPPORTED:
+            raise
+        return measure_decode(args, name, spec, world, dist, device, local_rank, rank, want_cpu, form=False)
+    calls = measure_decode(args, name, spec, world, dist, device, local_rank, rank, want_cpu, form=False)
+    best = dict(fused if fused["value"] > calls["value"] else calls)
+    if "cpu_baseline" in calls:
+        best["cpu_baseline"] = calls["cpu_baseline"]
+    best["layer_forms"] = {r["config"]["layer_form"]: {"value": r["value"], "ms_per_step": r["ms_per_step"],
+                                                        "e2e": r["e2e"]["value"], "gpu_launches_per_step":
+                                                        r["gpu_launches_per_step"]} for r in (fused, calls)}
+    return best
 
 
 def measure_model(args, world, dist, device, local_rank, rank, want_cpu) -> dict:
@@ -738,7 +761,7 @@ def run_lidx(args, rank, world, local_rank):
             return measure_eval(args, world, dist, device, local_rank, rank, want_cpu)
         if name == MODEL:
             return measure_model(args, world, dist, device, local_rank, rank, want_cpu)
-        return measure_decode(args, name, WORKLOADS[name], world, dist, device, local_rank, rank, want_cpu)
+        return decode_forms(args, name, WORKLOADS[name], world, dist, device, local_rank, rank, want_cpu)
 
     head = one(args.workload)
     side = {}
@@ -770,7 +793,8 @@ def main():
     ap.add_argument("--workload", default="decode-64k", choices=sorted(WORKLOADS) + [EVAL, MODEL])
     ap.add_argument("--only", action="store_true", help="time the named workload alone")
     ap.add_argument("--layer-form", default="auto", choices=sorted(LAYER_FORMS),
-                    help="CSA decode layers: one launch per layer, three calls, or the library's choice")
+                    help="CSA decode layers: one launch per layer, three calls, or (auto) time both and "
+                         "report the faster")
     args = ap.parse_args()
     args.repeats = max(5, args.repeats)
     rank = int(os.environ.get("RANK", "0"))
