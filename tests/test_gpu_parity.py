@@ -151,7 +151,8 @@ def test_topk_allowed_mask_and_nan():
     allowed = (g.random((3, N)) < 0.3).astype(np.uint8)
     allowed[2] = 0  # nothing allowed
     st = torch.from_numpy(s).cuda().reshape(3, 1, N)
-    ws = L.workspace(4096)
+    ids = torch.empty((3, 1, 256), dtype=torch.int32, device="cuda")
+    ws = L.workspace(L.workspace_size(L.OP_TOPK, L.topk_args(st, 256, torch.from_numpy(allowed).cuda(), ids)))
     L.topk_select(st, 256, torch.from_numpy(allowed).cuda(), ws=ws)
     _topk_check(s, 256, allowed)
     # NaN raises the device status flag (row 1 has NaN among allowed entries)

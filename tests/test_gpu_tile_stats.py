@@ -80,8 +80,9 @@ def test_topk_bounds_with_nan_and_allowed_mask():
     allowed = (np.random.default_rng(52).random((3, N)) < 0.3).astype(np.uint8)
     allowed[2, 7] = 1
     b = _dev_bounds(bounds_of(s)).reshape(3, 1, -1, 2)
-    ws = L.workspace(4096)
     st = torch.from_numpy(s).cuda().reshape(3, 1, N)
+    ids = torch.empty((3, 1, 256), dtype=torch.int32, device="cuda")
+    ws = L.workspace(L.workspace_size(L.OP_TOPK, L.topk_args(st, 256, torch.from_numpy(allowed).cuda(), ids)))
     ids, n_sel, _, _ = L.topk_select(st, 256, torch.from_numpy(allowed).cuda(), ws=ws, tile_stats=b)
     _check(s, ids, n_sel, 256, allowed)
     assert L.read_device_status(ws) & L.DEV_NAN
