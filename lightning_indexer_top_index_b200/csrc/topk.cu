@@ -38,7 +38,7 @@ namespace {
 constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / 32;
 constexpr int kMaxItems = 32;
-constexpr int kMaxCluster = 8;
+constexpr int kMaxCluster = 16;  // 16-CTA clusters (a non-portable size) where the device schedules them
 constexpr int kSlot = 512;                       // candidates a CTA pushes to every CTA of its cluster
 constexpr int kGatherMax = kSlot * kMaxCluster;  // candidates every CTA can gather
 constexpr int kRankMax = 96;       // candidates resolved by direct rank counting (quadratic work)
@@ -807,9 +807,15 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelParams p) 
 }
 
 template <int C>
+size_t select_smem() {
+  return ((sizeof(SelSmem) + 15) & ~size_t(15)) + (static_cast<size_t>(C) * kThreads + 4) * sizeof(float);
+}
+
+template <int C>
 cudaError_t launch_c(int G, int rows, const SelParams &p, cudaStream_t st, bool pdl) {
-  const size_t smem = ((sizeof(SelSmem) + 15) & ~size_t(15)) + (static_cast<size_t>(C) * kThreads + 4) * sizeof(float);
+  const size_t smem = select_smem<C>();
   cudaFuncSetAttribute(select_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  cudaFuncSetAttribute(select_kernel<C>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(G, rows);
   cfg.blockDim = dim3(kThreads);
@@ -832,15 +838,46 @@ cudaError_t launch_c(int G, int rows, const SelParams &p, cudaStream_t st, bool 
   return cudaLaunchKernelEx(&cfg, select_kernel<C>, p);
 }
 
+// Whether the device schedules a 16-CTA cluster of the select kernel (a
+// non-portable size), found once per device.
+bool cluster16_ok() {
+  static int cache[64] = {};  // 0 unknown, 1 yes, 2 no
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return false;
+  if (!cache[dev]) {
+    cudaFuncSetAttribute(select_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         static_cast<int>(select_smem<32>()));
+    cudaFuncSetAttribute(select_kernel<32>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(16, 1);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = select_smem<32>();
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 16;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    const cudaError_t e = cudaOccupancyMaxActiveClusters(&n, select_kernel<32>, &cfg);
+    cudaGetLastError();
+    cache[dev] = e == cudaSuccess && n >= 1 ? 1 : 2;
+  }
+  return cache[dev] == 1;
+}
+
 // Cluster size and items per thread for rows of N entries.
 void plan(int N, int rows, int &G, int &C) {
+  const int gmax = cluster16_ok() ? 16 : 8;
   G = 1;
   if (rows < 148) {
     G = 148 / rows;
-    G = G >= 8 ? 8 : G >= 4 ? 4 : G >= 2 ? 2 : 1;
+    G = G >= gmax ? gmax : G >= 8 ? 8 : G >= 4 ? 4 : G >= 2 ? 2 : 1;
     while (G > 1 && (N + G - 1) / G < 2048) G >>= 1;  // keep slices worth a CTA
   }
-  while ((N + G - 1) / G > kThreads * kMaxItems && G < kMaxCluster) G <<= 1;
+  while ((N + G - 1) / G > kThreads * kMaxItems && G < gmax) G <<= 1;
   const int per = (N + G - 1) / G;
   C = 1;
   while (C * kThreads < per) C <<= 1;
@@ -866,8 +903,11 @@ cudaError_t launch_select(const SelParams &p, int grid_rows, int N, cudaStream_t
 // fewer than k entries ranked above it in the row has fewer than k above it
 // in its segment), then the top-k of that union, whose candidates keep the
 // row's index order so ties still go to the lower index.
-constexpr int kSegLen = kMaxCluster * kThreads * 16;  // 131072 positions per segment
-constexpr int kMaxRow = kMaxCluster * kThreads * kMaxItems;
+// Longest row one cluster holds, and the segment length of longer rows (half
+// a cluster's capacity): 524288 and 262144 positions with 16-CTA clusters,
+// 262144 and 131072 with 8.
+int max_row() { return (cluster16_ok() ? 16 : 8) * kThreads * kMaxItems; }
+int seg_len() { return (cluster16_ok() ? 16 : 8) * kThreads * 16; }
 
 struct BigRowWs {
   size_t seg_ids, seg_n, cand_s, cand_ok, ids2, total;
@@ -875,7 +915,7 @@ struct BigRowWs {
 
 BigRowWs big_row_ws(const lidx_topk_args &a) {
   auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
-  const size_t rows = static_cast<size_t>(a.B) * a.Q, n_seg = (a.N + kSegLen - 1) / kSegLen;
+  const size_t rows = static_cast<size_t>(a.B) * a.Q, n_seg = (a.N + seg_len() - 1) / seg_len();
   const size_t nc = n_seg * a.k;
   BigRowWs w{};
   size_t o = LIDX_WS_HEADER;
@@ -936,7 +976,7 @@ cudaError_t launch_big_row(const lidx_topk_args &a, void *ws, cudaStream_t st, b
   float *cand_s = reinterpret_cast<float *>(w8 + w.cand_s);
   uint8_t *cand_ok = w8 + w.cand_ok;
   int32_t *ids2 = reinterpret_cast<int32_t *>(w8 + w.ids2);
-  const int rows = a.B * a.Q, n_seg = (a.N + kSegLen - 1) / kSegLen, nc = n_seg * a.k;
+  const int rows = a.B * a.Q, n_seg = (a.N + seg_len() - 1) / seg_len(), nc = n_seg * a.k;
   // 1. every segment's top-k, ids in row positions
   SelParams p1{};
   p1.a = a;
@@ -947,8 +987,8 @@ cudaError_t launch_big_row(const lidx_topk_args &a, void *ws, cudaStream_t st, b
   p1.a.tile_stats = nullptr;
   p1.status = static_cast<uint32_t *>(ws);
   p1.n_seg = n_seg;
-  p1.seg_len = kSegLen;
-  cudaError_t e = launch_select(p1, rows * n_seg, kSegLen, st, pdl);
+  p1.seg_len = seg_len();
+  cudaError_t e = launch_select(p1, rows * n_seg, seg_len(), st, pdl);
   if (e != cudaSuccess) return e;
   // 2. their scores in row order, with an eligibility flag
   const dim3 g2((nc + 255) / 256 < 64 ? (nc + 255) / 256 : 64, rows);
@@ -987,16 +1027,16 @@ cudaError_t launch_big_row(const lidx_topk_args &a, void *ws, cudaStream_t st, b
 }  // namespace
 
 bool topk_supported(const lidx_topk_args &a) {
-  if (a.N <= kMaxRow) return true;
-  const int64_t n_seg = (static_cast<int64_t>(a.N) + kSegLen - 1) / kSegLen;
-  return n_seg * a.k <= kMaxRow;
+  if (a.N <= max_row()) return true;
+  const int64_t n_seg = (static_cast<int64_t>(a.N) + seg_len() - 1) / seg_len();
+  return n_seg * a.k <= max_row();
 }
 
-size_t topk_workspace(const lidx_topk_args &a) { return a.N <= kMaxRow ? LIDX_WS_HEADER : big_row_ws(a).total; }
+size_t topk_workspace(const lidx_topk_args &a) { return a.N <= max_row() ? LIDX_WS_HEADER : big_row_ws(a).total; }
 
 cudaError_t launch_topk(const lidx_topk_args &a, void *ws, cudaStream_t st) {
   const bool pdl = (a.flags & LIDX_LAUNCH_PDL) != 0;
-  if (a.N > kMaxRow) return launch_big_row(a, ws, st, pdl);
+  if (a.N > max_row()) return launch_big_row(a, ws, st, pdl);
   SelParams p{};
   p.a = a;
   p.status = static_cast<uint32_t *>(ws);
