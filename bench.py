@@ -276,10 +276,12 @@ def cpu_baseline_decode(spec, layers_inp, budget_s=15.0) -> dict:
 
 
 # -------------------------------------------------------------- GPU timing
-def timed_loop(fn, steps: int, repeats: int, dist, device, between=None) -> tuple:
+def timed_loop(fn, steps: int, repeats: int, dist, device, between=None, begin=None, end=None) -> tuple:
     """Median over `repeats` of the device time of `steps` calls of fn()
     (CUDA events, synchronised on both sides, after a barrier); returns
-    (ms per step: the median, max over ranks; every repeat's ms)."""
+    (ms per step: the median, max over ranks; every repeat's ms).  begin()
+    and end() run right after the first and right before the last event (on
+    the current stream), e.g. to order a side stream inside the region."""
     import torch
     per = []
     for _ in range(repeats):
@@ -288,8 +290,12 @@ def timed_loop(fn, steps: int, repeats: int, dist, device, between=None) -> tupl
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
+        if begin:
+            begin()
         for i in range(steps):
             fn(i)
+        if end:
+            end()
         e1.record()
         torch.cuda.synchronize()
         per.append(e0.elapsed_time(e1) / steps)
@@ -297,6 +303,55 @@ def timed_loop(fn, steps: int, repeats: int, dist, device, between=None) -> tupl
             between()
     ms = max_over_ranks(statistics.median(per), dist, device)
     return ms, per
+
+
+def pipelined_e2e(steps, h2d, d2h):
+    """End-to-end steps over the rotating replicas with the copies on a side
+    stream: step i copies its inputs into replica i % R (h2d(step)), replays
+    it, and copies its result back (d2h(step, r)); the copy of step i+1's
+    inputs overlaps step i.  Events keep a replica's inputs and outputs from
+    being overwritten while in use.  Returns (step(i), begin(), end()): begin
+    orders the side stream after the region's start, end makes the current
+    stream wait for the last copies."""
+    import torch
+    R = len(steps)
+    side = torch.cuda.Stream()
+    h2d_done = [torch.cuda.Event() for _ in range(R)]
+    used = [torch.cuda.Event() for _ in range(R)]     # the replica's step has read its inputs
+    d2h_done = [torch.cuda.Event() for _ in range(R)]
+    state = {"next": 0}
+
+    def copy_in(i):
+        r = i % R
+        with torch.cuda.stream(side):
+            side.wait_event(used[r])
+            h2d(steps[r])
+            h2d_done[r].record(side)
+
+    def step(i):
+        main = torch.cuda.current_stream()
+        r = i % R
+        if state["next"] <= i:  # this step's inputs not yet on their way
+            copy_in(i)
+        main.wait_event(h2d_done[r])
+        main.wait_event(d2h_done[r])
+        steps[r].replay()
+        used[r].record(main)
+        copy_in(i + 1)
+        state["next"] = i + 2
+        with torch.cuda.stream(side):
+            side.wait_event(used[r])
+            d2h(steps[r], r)
+            d2h_done[r].record(side)
+
+    def begin():
+        side.wait_stream(torch.cuda.current_stream())
+        state["next"] = 0
+
+    def end():
+        torch.cuda.current_stream().wait_stream(side)
+
+    return step, begin, end
 
 
 def make_caches(spec, layers_inp, device):
@@ -396,19 +451,16 @@ def measure_decode(args, name, spec, world, dist, device, local_rank, rank, want
 
     # end to end: pinned host queries in, attention outputs back, every step
     q_idx_p, w_p, q_attn_p = q_idx_h.pin_memory(), w_h.pin_memory(), q_attn_h.pin_memory()
-    out_p = torch.empty(steps[0].out.shape, dtype=torch.float32).pin_memory()
-
-    def e2e_step(i):
-        s = steps[i % R]
-        s.set_inputs(q_idx_p, w_p, q_attn_p)
-        s.replay()
-        out_p.copy_(s.out, non_blocking=True)
-
+    out_ps = [torch.empty(steps[0].out.shape, dtype=torch.float32).pin_memory() for _ in range(R)]
+    e2e_step, e2e_begin, e2e_end = pipelined_e2e(steps, lambda s: s.set_inputs(q_idx_p, w_p, q_attn_p),
+                                                 lambda s, r: out_ps[r].copy_(s.out, non_blocking=True))
+    e2e_begin()
     for i in range(args.warmup):
         e2e_step(i)
-    e2e_ms, _ = timed_loop(e2e_step, args.steps, args.repeats, dist, device)
+    e2e_end()
+    e2e_ms, _ = timed_loop(e2e_step, args.steps, args.repeats, dist, device, begin=e2e_begin, end=e2e_end)
     h2d = sum(x.numel() * x.element_size() for x in (q_idx_p, w_p, q_attn_p))
-    d2h = out_p.numel() * out_p.element_size()
+    d2h = out_ps[0].numel() * out_ps[0].element_size()
     status = 0
     for s in steps:
         for ws in s.workspaces():
@@ -516,18 +568,20 @@ def measure_model(args, world, dist, device, local_rank, rank, want_cpu) -> dict
     ms, per = timed_loop(lambda i: steps[i % R].replay(), args.steps, args.repeats, dist, device)
     clk = clocks.stop()
     pins = [t.pin_memory() for t in (q_idx_h, w_h, qa_h)]
-    out_p = torch.empty(steps[0].out.shape, dtype=torch.float32).pin_memory()
+    out_ps = [torch.empty(steps[0].out.shape, dtype=torch.float32).pin_memory() for _ in range(R)]
+    csa_ps = [torch.empty(steps[0].csa.out.shape, dtype=torch.float32).pin_memory() for _ in range(R)]
+    out_p = out_ps[0]
 
-    def e2e_step(i):
-        s = steps[i % R]
-        s.set_inputs(*pins)
-        s.replay()
-        out_p.copy_(s.out, non_blocking=True)
-        out_p[s._csa_layer].copy_(s.csa.out, non_blocking=True)
+    def d2h(s, r):  # the window-only and HCA layers' outputs, and the CSA layers'
+        out_ps[r].copy_(s.out, non_blocking=True)
+        csa_ps[r].copy_(s.csa.out, non_blocking=True)
 
+    e2e_step, e2e_begin, e2e_end = pipelined_e2e(steps, lambda s: s.set_inputs(*pins), d2h)
+    e2e_begin()
     for i in range(args.warmup):
         e2e_step(i)
-    e2e_ms, _ = timed_loop(e2e_step, args.steps, args.repeats, dist, device)
+    e2e_end()
+    e2e_ms, _ = timed_loop(e2e_step, args.steps, args.repeats, dist, device, begin=e2e_begin, end=e2e_end)
     status = 0
     for s in steps:
         for ws in s.workspaces():
@@ -550,7 +604,7 @@ def measure_model(args, world, dist, device, local_rank, rank, want_cpu) -> dict
                      "avg_launch_us": ms * 1e3},
         "e2e": {"value": job_rate(1, world, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in pins),
-                "d2h_bytes_per_step": out_p.numel() * out_p.element_size()},
+                "d2h_bytes_per_step": out_p.numel() * out_p.element_size() + steps[0].csa.out.numel() * 4},
         "gpu_launches": args.steps * args.repeats * steps[0].kernel_launches(),
         "gpu_launches_per_step": steps[0].kernel_launches(),
         "device_status": status,
