@@ -66,6 +66,7 @@ def _load():
                 "orc_topk": (I, [I, I, P, P, P, P, P]),
                 "orc_attn": (I, [I, RP, RP, I, P, I, RP, I, D, P, P]),
                 "orc_golden": (I, [I, I, I, RP, RP, D, P]),
+                "orc_golden_index": (I, [I, I, P, I64, P]),
                 "orc_topp": (I, [I, P, C.c_uint32, C.c_uint32, I, P, P]),
                 "orc_vote": (I, [I, I, P, I, P]),
                 "orc_union": (I, [I, I, P, P]),
@@ -237,6 +238,18 @@ def golden(qa, kv, T, H, N, scale=None):
     sc = 1.0 / np.sqrt(kr.dim) if scale is None else scale
     p = np.empty((T, N), dtype=np.float32)
     _check(_load().orc_golden(T, H, N, C.byref(qr), C.byref(kr), float(sc), _ptr(p)))
+    return p
+
+
+def golden_index(scores):
+    """Softmax of each row of scores [..][N] over its N entries (the golden
+    probabilities read as a softmax of the indexer logits); float32, same
+    shape.  NaN and -inf scores take no mass."""
+    s = np.ascontiguousarray(scores, dtype=np.float32)
+    N = s.shape[-1]
+    R = s.size // N
+    p = np.empty(s.shape, dtype=np.float32)
+    _check(_load().orc_golden_index(R, N, _ptr(s), N, _ptr(p)))
     return p
 
 

@@ -22,6 +22,9 @@
  *  - orc_golden        head-mean of per-head dense softmax over all entries
  *        (FlashMemory vs native indexer post, Act 3: unmasked dense attention
  *        as ground truth; write-up section 3.2 step 1)
+ *  - orc_golden_index  the other reading of the golden probabilities: the
+ *        softmax over all entries of the indexer's own logits (write-up
+ *        section 3.2 step 1 softmaxes the indexer logits)
  *  - orc_topp          the minimal prefix of entries (descending probability)
  *        whose mass reaches the fraction p of the total (write-up 3.2 step 2)
  *  - orc_vote          entries chosen by at least m of the layers (write-up
@@ -450,6 +453,31 @@ int orc_golden(int T, int H, int N, const orc_rows *qa, const orc_rows *kv, doub
     free(qv);
     free(lg);
     free(acc);
+    return ORC_OK;
+}
+
+/*
+ * Softmax over the N entries of each of R rows of scores (row r at
+ * s + r * ld): p_j = exp(s_j - m) / sum_i exp(s_i - m), m the row's largest
+ * score.  NaN and -inf scores take no mass (p = 0); a row without any finite
+ * score is all zeros.  Rounded to fp32 at the end.
+ */
+int orc_golden_index(int R, int N, const float *s, int64_t ld, float *p)
+{
+    if (R < 1 || N < 1 || ld < N) return ORC_EINVAL;
+    for (int r = 0; r < R; r++) {
+        const float *x = s + (size_t)r * ld;
+        float *out = p + (size_t)r * N;
+        double m = -INFINITY;
+        for (int j = 0; j < N; j++)
+            if (x[j] == x[j] && (double)x[j] > m) m = x[j];
+        double l = 0.0;
+        if (m > -INFINITY)
+            for (int j = 0; j < N; j++)
+                if (x[j] == x[j]) l += exp((double)x[j] - m);
+        for (int j = 0; j < N; j++)
+            out[j] = (m > -INFINITY && x[j] == x[j]) ? (float)(exp((double)x[j] - m) / l) : 0.0f;
+    }
     return ORC_OK;
 }
 

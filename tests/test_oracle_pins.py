@@ -334,6 +334,41 @@ def test_golden_agrees_with_attention_lse():
     np.testing.assert_allclose(p, np.exp(logit - lse[0]), rtol=1e-5)
 
 
+def test_golden_index_closed_forms():
+    """The softmax-of-the-indexer-logits reading: values fixed in closed form
+    (a uniform row, logits that differ by ln 3 and ln 2), and the same values
+    at logits near 1000, where exp without the row maximum subtracted
+    overflows."""
+    ln2, ln3 = np.log(2.0), np.log(3.0)
+    p = oracle.golden_index(np.array([[2.5] * 8, [0.0, ln3] + [-np.inf] * 6], dtype=np.float32))
+    np.testing.assert_array_equal(p[0], np.full(8, 0.125, dtype=np.float32))
+    np.testing.assert_allclose(p[1, :2], [0.25, 0.75], rtol=1e-6)
+    assert np.all(p[1, 2:] == 0)
+    x = np.array([1000.0 + ln2, 1000.0, 1000.0], dtype=np.float32)
+    d = float(x[0]) - 1000.0  # the stored offset (fp32 spacing at 1000 is 6e-5)
+    p = oracle.golden_index(x)
+    np.testing.assert_allclose(p, np.array([np.exp(d), 1.0, 1.0]) / (np.exp(d) + 2.0), rtol=1e-6)
+    assert abs(p[0] - 0.5) < 1e-4
+
+
+def test_golden_index_nan_and_empty_rows():
+    """NaN and -inf logits carry no mass; a row with no finite logit is all
+    zeros; otherwise a row sums to 1 and matches scipy's softmax over its
+    finite entries."""
+    g = np.random.default_rng(5)
+    s = g.standard_normal((3, 300)).astype(np.float32) * 4
+    s[1, ::7] = np.nan
+    s[1, 3::11] = -np.inf
+    s[2, :] = -np.inf
+    p = oracle.golden_index(s)
+    assert np.all(p[2] == 0)
+    fin = np.isfinite(s[1])
+    assert np.all(p[1, ~fin] == 0)
+    np.testing.assert_allclose(p[1, fin], scipy.special.softmax(s[1, fin].astype(np.float64)), rtol=1e-6)
+    np.testing.assert_allclose(p[0], scipy.special.softmax(s[0].astype(np.float64)), rtol=1e-6)
+    np.testing.assert_allclose(p[:2].sum(axis=1), 1.0, rtol=1e-6)
+
+
 # ----------------------------------------------------------------------- top-p
 @pytest.mark.parametrize("ex", HAND["topp"])
 def test_topp_hand_examples(ex):
