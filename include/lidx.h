@@ -39,7 +39,7 @@
 extern "C" {
 #endif
 
-#define LIDX_ABI_VERSION 4
+#define LIDX_ABI_VERSION 5
 
 #if defined(__GNUC__)
 #define LIDX_API __attribute__((visibility("default")))
@@ -371,6 +371,13 @@ LIDX_API lidx_status lidx_cache_append(const lidx_append_args *args, void *ws, s
  *  LIDX_EVAL_GOLDEN  (FlashMemory-vs-native post, Act 3; write-up 3.2 step 1)
  *     probs[l][t][j] = (1/H) sum_h softmax_j(scale * qa[l][t][h] . kv_l[j])
  *     over the N entries of layer l (kv rows l*kv.batch_rows + j).
+ *  LIDX_EVAL_GOLDEN_INDEX (write-up 3.2 step 1, which applies the softmax
+ *     to the indexer logits: the other reading of the golden step)
+ *     probs[l][t][j] = softmax_j(index_scores[l*T + t][j]) over the N
+ *     entries, row r of index_scores at index_scores + r * ld_index_scores
+ *     (>= N).  NaN and -inf scores carry no mass (a NaN sets LIDX_DEV_NAN);
+ *     a row without a finite score is all zeros.  Excludes LIDX_EVAL_GOLDEN
+ *     (both write probs).
  *  LIDX_EVAL_TOPP    (write-up 3.2 step 2)
  *     per row (l,t): with m_j = floor(probs_j * 2^40) and M = sum m_j, the
  *     shortest prefix of the ranking (probs descending, ties to the lower
@@ -398,6 +405,7 @@ LIDX_API lidx_status lidx_cache_append(const lidx_append_args *args, void *ws, s
 #define LIDX_EVAL_VOTE 0x4u
 #define LIDX_EVAL_LSA 0x8u
 #define LIDX_EVAL_OVERLAP 0x10u
+#define LIDX_EVAL_GOLDEN_INDEX 0x20u
 
 typedef struct lidx_eval_args {
     uint32_t ops;
@@ -427,6 +435,9 @@ typedef struct lidx_eval_args {
     const uint32_t *set_b;
     int64_t ld_b;
     int64_t *counts;          /* [n_pairs][3] */
+    /* GOLDEN_INDEX */
+    const float *index_scores; /* [L*T][ld_index_scores] */
+    int64_t ld_index_scores;
 } lidx_eval_args;
 
 LIDX_API lidx_status lidx_selection_eval(const lidx_eval_args *args, void *ws, size_t ws_bytes,

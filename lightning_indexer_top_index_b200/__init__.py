@@ -34,6 +34,7 @@ LAUNCH_TEST_LOST_ARRIVAL = 0x80000000
 STATS_SPAN = 32  # entries per score-bounds record (optional scorer output, top-k input)
 
 EVAL_GOLDEN, EVAL_TOPP, EVAL_VOTE, EVAL_LSA, EVAL_OVERLAP = 0x1, 0x2, 0x4, 0x8, 0x10
+EVAL_GOLDEN_INDEX = 0x20  # probs as the softmax of the indexer logits (the other golden reading)
 OP_SCORE, OP_TOPK, OP_ATTN, OP_EVAL, OP_DECODE, OP_APPEND = 0, 1, 2, 3, 4, 5
 
 # Layer schedule of DeepSeek-V4-Flash (architecture post, section (A) table):
@@ -116,7 +117,7 @@ class EvalArgs(C.Structure):
                 ("window_bits", C.c_void_p), ("n_gate", C.c_int32), ("gate_logits", C.c_void_p),
                 ("gate_bias", C.c_float), ("fetched_bits", C.c_void_p), ("n_pairs", C.c_int32),
                 ("set_a", C.c_void_p), ("ld_a", C.c_int64), ("set_b", C.c_void_p), ("ld_b", C.c_int64),
-                ("counts", C.c_void_p)]
+                ("counts", C.c_void_p), ("index_scores", C.c_void_p), ("ld_index_scores", C.c_int64)]
 
 
 class DecodeArgs(C.Structure):
@@ -411,12 +412,13 @@ def cache_append(x: torch.Tensor, cache: DeviceKV, pos: torch.Tensor, capacity: 
 def selection_eval(ops: int, *, L=1, T=1, H=1, N, qa=None, kv: DeviceKV = None, scale=None, probs=None,
                    top_p=(3, 5), topp_bits=None, min_votes=3, vote_bits=None, window_bits=None,
                    gate_logits=None, gate_bias=0.0, fetched_bits=None, set_a=None, ld_a=None, set_b=None,
-                   ld_b=None, n_pairs=0, counts=None, ws=None, stream=None):
+                   ld_b=None, n_pairs=0, counts=None, index_scores=None, ws=None, stream=None):
     """Run the requested evaluation steps (EVAL_* bit mask), in the order
-    GOLDEN, TOPP, VOTE, LSA, OVERLAP.  Output tensors must be given by the
+    GOLDEN (or GOLDEN_INDEX: probs as the softmax of index_scores [L*T][>= N]
+    rows), TOPP, VOTE, LSA, OVERLAP.  Output tensors must be given by the
     caller (see lidx_eval_args for shapes); returns them in a dict."""
     dev = None
-    for t in (qa, probs, topp_bits, gate_logits, set_a):
+    for t in (qa, probs, topp_bits, gate_logits, set_a, index_scores):
         if t is not None:
             dev = t.device
             break
@@ -430,7 +432,8 @@ def selection_eval(ops: int, *, L=1, T=1, H=1, N, qa=None, kv: DeviceKV = None, 
                  (set_a.stride(0) if set_a is not None and set_a.dim() > 1 else 0) if ld_a is None else ld_a,
                  _ptr(set_b),
                  (set_b.stride(0) if set_b is not None and set_b.dim() > 1 else 0) if ld_b is None else ld_b,
-                 _ptr(counts))
+                 _ptr(counts), _ptr(index_scores),
+                 0 if index_scores is None else index_scores.stride(-2) if index_scores.dim() > 1 else N)
     if ws is None:
         ws = workspace(workspace_size(OP_EVAL, a), dev)
     _check(lib().lidx_selection_eval(C.byref(a), C.c_void_p(ws.data_ptr()), ws.numel(), _stream(stream)),

@@ -377,6 +377,51 @@ size_t vote_bytes(const lidx_eval_args &a) {
 
 }  // namespace
 
+// Softmax of one score row per CTA over its N entries (the golden step read
+// as a softmax of the indexer logits): the row's largest non-NaN score m,
+// l = sum exp(s - m) over the non-NaN scores, then p = exp(s - m) / l.
+// NaN scores get p = 0 (and LIDX_DEV_NAN); -inf ones get 0 by exp; a row
+// without a finite score (m = -inf) is all zeros.
+__global__ void __launch_bounds__(256) golden_index_kernel(lidx_eval_args a, uint32_t *status) {
+  __shared__ float red[8];
+  const int r = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const float *s = a.index_scores + static_cast<size_t>(r) * a.ld_index_scores;
+  float *p = a.probs + static_cast<size_t>(r) * a.N;
+  float m = -INFINITY;
+  bool nan = false;
+  for (int j = tid; j < a.N; j += 256) {
+    const float v = s[j];
+    nan |= v != v;
+    m = fmaxf(m, v);  // fmaxf skips NaN
+  }
+  if (nan) raise_status(status, LIDX_DEV_NAN);
+  for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  if (lane == 0) red[warp] = m;
+  __syncthreads();
+  m = red[0];
+  for (int w = 1; w < 8; w++) m = fmaxf(m, red[w]);
+  __syncthreads();
+  if (m == -INFINITY) {
+    for (int j = tid; j < a.N; j += 256) p[j] = 0.f;
+    return;
+  }
+  float l = 0.f;
+  for (int j = tid; j < a.N; j += 256) {
+    const float v = s[j];
+    if (v == v) l += expf(v - m);
+  }
+  for (int o = 16; o; o >>= 1) l += __shfl_xor_sync(0xFFFFFFFFu, l, o);
+  if (lane == 0) red[warp] = l;
+  __syncthreads();
+  l = 0.f;
+  for (int w = 0; w < 8; w++) l += red[w];
+  const float il = 1.f / l;
+  for (int j = tid; j < a.N; j += 256) {
+    const float v = s[j];
+    p[j] = v == v ? expf(v - m) * il : 0.f;
+  }
+}
+
 size_t eval_workspace(const lidx_eval_args &a) {
   size_t n = LIDX_WS_HEADER;
   if (a.ops & LIDX_EVAL_GOLDEN) n += golden_tc_supported(a) ? golden_tc_workspace(a) : lse_bytes(a);
@@ -413,6 +458,10 @@ cudaError_t launch_eval(const lidx_eval_args &a, void *ws, cudaStream_t st) {
         golden_prob_kernel<LIDX_E4M3><<<g2, 128, smem, st>>>(a, lse2);
         break;
     }
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  if (a.ops & LIDX_EVAL_GOLDEN_INDEX) {
+    golden_index_kernel<<<a.L * a.T, 256, 0, st>>>(a, status);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   if (a.ops & LIDX_EVAL_TOPP) {

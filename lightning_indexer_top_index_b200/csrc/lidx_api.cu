@@ -109,13 +109,18 @@ lidx_status check_attn(const lidx_attn_args *a) {
 }
 
 lidx_status check_eval(const lidx_eval_args *a) {
-  if (!a || a->ops == 0 || (a->ops & ~0x1Fu)) return LIDX_ERR_INVALID_ARG;
+  if (!a || a->ops == 0 || (a->ops & ~0x3Fu)) return LIDX_ERR_INVALID_ARG;
+  if ((a->ops & LIDX_EVAL_GOLDEN) && (a->ops & LIDX_EVAL_GOLDEN_INDEX)) return LIDX_ERR_INVALID_ARG;
   if (a->N < 1) return LIDX_ERR_INVALID_ARG;
   if (a->ops & LIDX_EVAL_GOLDEN) {
     if (!a->qa || !a->probs || a->L < 1 || a->T < 1 || a->H < 1 || a->H > 64) return LIDX_ERR_INVALID_ARG;
     lidx_status s = check_kv(a->kv, 512, a->L, a->N);
     if (s != LIDX_OK) return s;
     if (a->kv.dtype == LIDX_F32 ? a->qa_dtype != LIDX_F32 : a->qa_dtype != LIDX_BF16) return LIDX_ERR_UNSUPPORTED;
+  }
+  if (a->ops & LIDX_EVAL_GOLDEN_INDEX) {
+    if (!a->index_scores || !a->probs || a->L < 1 || a->T < 1 || a->ld_index_scores < a->N) return LIDX_ERR_INVALID_ARG;
+    if (!aligned(a->index_scores, 4) || !aligned(a->probs, 4)) return LIDX_ERR_INVALID_ARG;
   }
   if (a->ops & LIDX_EVAL_TOPP) {
     if (!a->probs || !a->topp_bits || a->L < 1 || a->T < 1) return LIDX_ERR_INVALID_ARG;

@@ -4,8 +4,10 @@ FlashMemory-vs-native post, Acts 1 and 3), on the library's calls:
 
   per layer     native index scores of the window's T queries and their
                 top-k (the native selection)
-  all layers    golden dense-attention probabilities, their top-p sets and
-                the golden top-k
+  all layers    golden dense-attention probabilities (or, with
+                golden="index", the softmax of the native index scores: the
+                write-up's step 1 read as a softmax of the indexer logits),
+                their top-p sets and the golden top-k
   window        the >= min_votes layer vote per query and its union G
   gate          the gate's logits at its layers (the index scorer with the
                 gate query and signed head weights) and the fetched set F
@@ -26,18 +28,24 @@ from typing import Dict, Optional, Sequence
 
 import torch
 
-from . import (DeviceKV, EVAL_GOLDEN, EVAL_LSA, EVAL_OVERLAP, EVAL_TOPP, EVAL_VOTE, OP_EVAL, OP_TOPK, EvalArgs,
+from . import (DeviceKV, EVAL_GOLDEN, EVAL_GOLDEN_INDEX, EVAL_LSA, EVAL_OVERLAP, EVAL_TOPP, EVAL_VOTE, OP_EVAL, OP_TOPK, EvalArgs,
                index_score, selection_eval, topk_args, topk_select, workspace, workspace_size, KVArgs, BF16)
 
 
 class EvalWindow:
     def __init__(self, keys: Sequence[DeviceKV], kv_all: DeviceKV, q_idx: torch.Tensor, w: torch.Tensor,
                  qa: torch.Tensor, gate_q: torch.Tensor, gate_u: torch.Tensor, gate_layers: Sequence[int], N: int,
-                 k: int = 512, top_p=(3, 5), min_votes: int = 3, scale: Optional[float] = None):
+                 k: int = 512, top_p=(3, 5), min_votes: int = 3, scale: Optional[float] = None,
+                 golden: str = "attention"):
         """keys: per layer the index keys (dim 128); kv_all: every layer's
         attention rows, layer l at rows [l*batch_rows, l*batch_rows + N);
         q_idx [L][T][H][128], w [L][T][H], qa [L][T][H][512] (bf16);
-        gate_q [G][H][128], gate_u [G][H] for the gate layers."""
+        gate_q [G][H][128], gate_u [G][H] for the gate layers.  golden:
+        "attention" (dense attention probabilities) or "index" (the softmax
+        of the native index scores)."""
+        if golden not in ("attention", "index"):
+            raise ValueError(golden)
+        self.golden = golden
         self.keys, self.kv_all = list(keys), kv_all
         self.L, self.T, self.H = q_idx.shape[0], q_idx.shape[1], q_idx.shape[2]
         self.N, self.k, self.top_p, self.min_votes = N, k, top_p, min_votes
@@ -105,8 +113,12 @@ class EvalWindow:
                         bits=self.nat_bits[l], ws=self.ws_topk_nat, stream=st)
         mark("topk", 1)
         mark("golden", 0)
-        selection_eval(EVAL_GOLDEN, L=L, T=T, H=H, N=N, qa=self.qa, kv=self.kv_all, scale=self.scale,
-                       probs=self.probs, ws=self.ws_golden, stream=st)
+        if self.golden == "index":
+            selection_eval(EVAL_GOLDEN_INDEX, L=L, T=T, N=N, index_scores=self.scores.view(L * T, N),
+                           probs=self.probs, ws=self.ws_small, stream=st)
+        else:
+            selection_eval(EVAL_GOLDEN, L=L, T=T, H=H, N=N, qa=self.qa, kv=self.kv_all, scale=self.scale,
+                           probs=self.probs, ws=self.ws_golden, stream=st)
         mark("golden", 1)
         mark("topp", 0)
         selection_eval(EVAL_TOPP, L=L, T=T, N=N, probs=self.probs, top_p=self.top_p, topp_bits=self.topp_bits,

@@ -15,7 +15,7 @@ from lightning_indexer_top_index_b200.evalwin import EvalWindow
 pytestmark = pytest.mark.gpu
 
 
-def _window(spec):
+def _window(spec, golden="attention"):
     layers = [synth.eval_layer(spec, l) for l in range(spec.L)]
     gate = synth.eval_gate(spec)
     keys = [dev_kv(x["keys"], batch_rows=spec.N) for x in layers]
@@ -24,7 +24,8 @@ def _window(spec):
     w = torch.stack([torch.from_numpy(x["w"]).cuda() for x in layers])
     qa = torch.stack([dev_q(x["qa"], "bf16") for x in layers])
     win = EvalWindow(keys, kv_all, q_idx, w, qa, dev_q(gate["g"], "bf16"), torch.from_numpy(gate["u"]).cuda(),
-                     spec.gate_layers, spec.N, spec.k, (spec.top_p_num, spec.top_p_den), spec.min_votes, spec.scale)
+                     spec.gate_layers, spec.N, spec.k, (spec.top_p_num, spec.top_p_den), spec.min_votes, spec.scale,
+                     golden=golden)
     return layers, gate, win
 
 
@@ -96,3 +97,25 @@ def test_eval_window_against_oracle(cuda_device):
             assert np.array_equal(natf_bits[l, t], synth.pack_bits(dense)[0])
             assert tuple(c_fg[l * T + t]) == oracle.overlap(natf_bits[l, t], gold_bits[l, t], N)
             assert tuple(c_fn[l * T + t]) == oracle.overlap(natf_bits[l, t], nat_bits[l, t], N)
+
+
+def test_eval_window_golden_from_index_logits(cuda_device):
+    """golden="index": the golden probabilities are the softmax of the
+    window's native index scores (the write-up's step 1 read as a softmax of
+    the indexer logits).  Against the oracle on the GPU's own scores, and the
+    top-p sets and vote bit-exact on the GPU's own probabilities."""
+    spec = synth.scaled(synth.EVAL_WINDOW, L=3, T=2, N=1500, k=64, gate_layers=(0, 1, 2))
+    _, _, win = _window(spec, golden="index")
+    win.enqueue()
+    torch.cuda.synchronize()
+    N, T, Lq, W = spec.N, spec.T, spec.L, (spec.N + 31) // 32
+    scores = win.scores.cpu().numpy().reshape(Lq, T, N)
+    probs = win.probs.cpu().numpy()
+    np.testing.assert_allclose(probs, oracle.golden_index(scores), rtol=2e-5, atol=1e-30)
+    topp_bits = win.topp_bits.cpu().numpy().view(np.uint32)
+    for l in range(Lq):
+        for t in range(T):
+            bits, _ = oracle.topp(probs[l, t], spec.top_p_num, spec.top_p_den)
+            assert np.array_equal(topp_bits[l, t], bits)
+    assert np.array_equal(win.window_bits.cpu().numpy().view(np.uint32),
+                          oracle.union(np.stack([oracle.vote(topp_bits[:, t], N, spec.min_votes) for t in range(T)]), N))

@@ -267,6 +267,37 @@ def test_chain_tiny_config():
 
 
 # ------------------------------------------------------------------- eval
+@pytest.mark.parametrize("Lq,T,N", [(2, 3, 1100), (1, 4, 32768), (1, 1, 1)])
+def test_golden_index_parity(Lq, T, N):
+    """probs = the softmax of each score row (LIDX_EVAL_GOLDEN_INDEX), on
+    rows with NaN and -inf entries, a row of -inf only, and a padded row
+    stride: within 2e-5 relative of the oracle (fp32 exp and a sum over the
+    row against double), zeros where the oracle has zeros, NaN flagged."""
+    g = np.random.default_rng(40 + N)
+    s = (g.standard_normal((Lq * T, N + 5)) * 3).astype(np.float32)
+    if Lq * T > 1:
+        s[0, ::13] = np.nan
+        s[0, 1::17] = -np.inf
+        s[1, :] = -np.inf
+    st = torch.from_numpy(s).cuda()[:, :N]
+    probs = torch.full((Lq, T, N), 7.0, device="cuda")
+    ws = L.workspace(4096)
+    L.selection_eval(L.EVAL_GOLDEN_INDEX, L=Lq, T=T, N=N, index_scores=st, probs=probs, ws=ws)
+    got = probs.cpu().numpy().reshape(Lq * T, N)
+    ref = oracle.golden_index(s[:, :N])
+    np.testing.assert_allclose(got, ref, rtol=2e-5, atol=1e-30)
+    assert np.array_equal(got == 0, ref == 0)
+    assert bool(L.read_device_status(ws) & L.DEV_NAN) == bool(np.isnan(s[:, :N]).any())
+
+
+def test_golden_index_excludes_golden():
+    st = torch.zeros((1, 8), device="cuda")
+    probs = torch.empty((1, 1, 8), device="cuda")
+    with pytest.raises(L.LidxError) as e:
+        L.selection_eval(L.EVAL_GOLDEN | L.EVAL_GOLDEN_INDEX, L=1, T=1, H=1, N=8, index_scores=st, probs=probs)
+    assert e.value.status == L.ERR_INVALID_ARG
+
+
 def test_golden_probs_parity():
     spec = synth.scaled(synth.EVAL_WINDOW, L=2, T=3, H=8, N=1100)
     qa = np.stack([synth.eval_layer(spec, l)["qa"][:, :spec.H] for l in range(spec.L)])
