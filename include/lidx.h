@@ -39,7 +39,7 @@
 extern "C" {
 #endif
 
-#define LIDX_ABI_VERSION 5
+#define LIDX_ABI_VERSION 6
 
 #if defined(__GNUC__)
 #define LIDX_API __attribute__((visibility("default")))
@@ -456,6 +456,16 @@ LIDX_API lidx_status lidx_selection_eval(const lidx_eval_args *args, void *ws, s
 /* Bytes of workspace call `op` needs for `args` (a pointer to the matching
  * *_args struct, host memory).  Score needs none (0). */
 LIDX_API lidx_status lidx_workspace_size(int op, const void *args, size_t *bytes);
+
+/* Number of kernels call `op` launches for `args` (host memory), after the
+ * same argument checks as the call (their status on failure): 1 for the
+ * scorer, the decode layer and the append; 1 for lidx_topk_select on rows
+ * one cluster holds, 4 beyond (segment selects, candidate gather, candidate
+ * select, map back); 2 for lidx_sparse_attn_decode (split kernel, merge);
+ * for lidx_selection_eval the sum over the requested ops.  Memsets and
+ * copies a call enqueues are not counted.  For launch accounting and for
+ * checking a captured graph. */
+LIDX_API lidx_status lidx_launch_count(int op, const void *args, int *count);
 
 /* Synchronises `stream`, copies the status word at the start of `ws` into
  * *status (host) and clears it on the device. */

@@ -136,7 +136,8 @@ class AppendArgs(C.Structure):
 
 _STRUCTS = [KVArgs, ScoreArgs, TopkArgs, AttnArgs, EvalArgs, DecodeArgs, AppendArgs]
 EXPORTS = ("lidx_index_score", "lidx_topk_select", "lidx_sparse_attn_decode", "lidx_selection_eval",
-           "lidx_decode_layer", "lidx_cache_append", "lidx_workspace_size", "lidx_read_device_status",
+           "lidx_decode_layer", "lidx_cache_append", "lidx_workspace_size", "lidx_launch_count",
+           "lidx_read_device_status",
            "lidx_status_string", "lidx_abi_version", "lidx_struct_size")
 
 _lib = None
@@ -161,6 +162,7 @@ def lib():
                 ("lidx_decode_layer", I, [C.POINTER(DecodeArgs), P, SZ, P]),
                 ("lidx_cache_append", I, [C.POINTER(AppendArgs), P, SZ, P]),
                 ("lidx_workspace_size", I, [I, P, C.POINTER(SZ)]),
+                ("lidx_launch_count", I, [I, P, C.POINTER(I)]),
                 ("lidx_read_device_status", I, [P, C.POINTER(C.c_uint32), P]),
                 ("lidx_status_string", C.c_char_p, [I]),
                 ("lidx_abi_version", I, []),
@@ -275,6 +277,13 @@ def index_score(q: torch.Tensor, w: torch.Tensor, keys: DeviceKV, N: int, scores
 def workspace_size(op: int, args) -> int:
     n = C.c_size_t(0)
     _check(lib().lidx_workspace_size(op, C.byref(args), C.byref(n)), "lidx_workspace_size")
+    return n.value
+
+
+def launch_count(op: int, args) -> int:
+    """Kernels the call `op` launches for `args` on the current device."""
+    n = C.c_int(0)
+    _check(lib().lidx_launch_count(op, C.byref(args), C.byref(n)), "lidx_launch_count")
     return n.value
 
 

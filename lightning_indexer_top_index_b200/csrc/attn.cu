@@ -258,6 +258,8 @@ size_t attn_workspace(const lidx_attn_args &a) {
   return LIDX_WS_HEADER + part_o_bytes(a, ns) + static_cast<size_t>(ns) * a.B * a.H * sizeof(float2);
 }
 
+int attn_launches(const lidx_attn_args &) { return 2; }  // split kernel + merge kernel
+
 cudaError_t launch_attn(const lidx_attn_args &a, void *ws, cudaStream_t st) {
   uint32_t *status = static_cast<uint32_t *>(ws);
   const int ns = splits_for(a);

@@ -429,6 +429,20 @@ size_t eval_workspace(const lidx_eval_args &a) {
   return n;
 }
 
+// Kernels launch_eval launches for a.ops, in its order: golden (two tensor-core
+// passes around the lse merge, or the lse and probability kernels), golden
+// from the index logits, top-p, vote + union, gate, overlap.
+int eval_launches(const lidx_eval_args &a) {
+  int n = 0;
+  if (a.ops & LIDX_EVAL_GOLDEN) n += golden_tc_supported(a) ? 3 : 2;
+  if (a.ops & LIDX_EVAL_GOLDEN_INDEX) n += 1;
+  if (a.ops & LIDX_EVAL_TOPP) n += 1;
+  if (a.ops & LIDX_EVAL_VOTE) n += 2;
+  if (a.ops & LIDX_EVAL_LSA) n += 1;
+  if (a.ops & LIDX_EVAL_OVERLAP) n += 1;
+  return n;
+}
+
 cudaError_t launch_eval(const lidx_eval_args &a, void *ws, cudaStream_t st) {
   uint32_t *status = static_cast<uint32_t *>(ws);
   char *cur = static_cast<char *>(ws) + LIDX_WS_HEADER;

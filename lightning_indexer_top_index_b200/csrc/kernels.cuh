@@ -27,10 +27,12 @@ bool score_tc_supported(const lidx_score_args &a);
 // ---- top-k
 bool topk_supported(const lidx_topk_args &a);
 size_t topk_workspace(const lidx_topk_args &a);
+int topk_launches(const lidx_topk_args &a);  // kernels one call launches
 cudaError_t launch_topk(const lidx_topk_args &a, void *ws, cudaStream_t st);
 
 // ---- sparse attention decode
 size_t attn_workspace(const lidx_attn_args &a);
+int attn_launches(const lidx_attn_args &a);  // kernels one call launches
 cudaError_t launch_attn(const lidx_attn_args &a, void *ws, cudaStream_t st);
 
 // ---- fused decode layer (score -> top-k -> attention in one launch)
@@ -46,6 +48,7 @@ bool golden_tc_supported(const lidx_eval_args &a);
 size_t golden_tc_workspace(const lidx_eval_args &a);
 cudaError_t launch_golden_tc(const lidx_eval_args &a, void *scratch, uint32_t *status, cudaStream_t st);
 size_t eval_workspace(const lidx_eval_args &a);
+int eval_launches(const lidx_eval_args &a);
 cudaError_t launch_eval(const lidx_eval_args &a, void *ws, cudaStream_t st);
 
 }  // namespace lidx

@@ -266,6 +266,40 @@ lidx_status lidx_workspace_size(int op, const void *args, size_t *bytes) {
   return s;
 }
 
+lidx_status lidx_launch_count(int op, const void *args, int *count) {
+  if (!args || !count) return LIDX_ERR_INVALID_ARG;
+  lidx_status s = LIDX_OK;
+  switch (op) {
+    case LIDX_OP_SCORE:
+      s = check_score(static_cast<const lidx_score_args *>(args));
+      if (s == LIDX_OK) *count = 1;
+      break;
+    case LIDX_OP_TOPK:
+      s = check_topk(static_cast<const lidx_topk_args *>(args));
+      if (s == LIDX_OK) *count = topk_launches(*static_cast<const lidx_topk_args *>(args));
+      break;
+    case LIDX_OP_ATTN:
+      s = check_attn(static_cast<const lidx_attn_args *>(args));
+      if (s == LIDX_OK) *count = attn_launches(*static_cast<const lidx_attn_args *>(args));
+      break;
+    case LIDX_OP_EVAL:
+      s = check_eval(static_cast<const lidx_eval_args *>(args));
+      if (s == LIDX_OK) *count = eval_launches(*static_cast<const lidx_eval_args *>(args));
+      break;
+    case LIDX_OP_APPEND:
+      s = check_append(static_cast<const lidx_append_args *>(args));
+      if (s == LIDX_OK) *count = 1;
+      break;
+    case LIDX_OP_DECODE:
+      s = check_decode(static_cast<const lidx_decode_args *>(args));
+      if (s == LIDX_OK) *count = 1;
+      break;
+    default:
+      return LIDX_ERR_INVALID_ARG;
+  }
+  return s;
+}
+
 lidx_status lidx_read_device_status(void *ws, uint32_t *status, void *stream) {
   if (!ws || !status) return LIDX_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

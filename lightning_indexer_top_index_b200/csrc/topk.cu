@@ -1034,6 +1034,10 @@ bool topk_supported(const lidx_topk_args &a) {
 
 size_t topk_workspace(const lidx_topk_args &a) { return a.N <= max_row() ? LIDX_WS_HEADER : big_row_ws(a).total; }
 
+// one cluster select, or: segment selects, candidate gather, candidate select,
+// map back (the mask clears are memsets, not kernels)
+int topk_launches(const lidx_topk_args &a) { return a.N <= max_row() ? 1 : 4; }
+
 cudaError_t launch_topk(const lidx_topk_args &a, void *ws, cudaStream_t st) {
   const bool pdl = (a.flags & LIDX_LAUNCH_PDL) != 0;
   if (a.N > max_row()) return launch_big_row(a, ws, st, pdl);

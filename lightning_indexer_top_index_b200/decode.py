@@ -22,8 +22,9 @@ from typing import List, Optional, Sequence
 
 import torch
 
-from . import (AttnArgs, DeviceKV, ScoreArgs, TopkArgs, BF16, LAUNCH_PDL, OP_ATTN, OP_DECODE, OP_TOPK, STATS_SPAN,
-               ERR_UNSUPPORTED, LidxError, attn_args, decode_args, lib, topk_args, workspace, workspace_size)
+from . import (AttnArgs, DeviceKV, ScoreArgs, TopkArgs, BF16, LAUNCH_PDL, OP_ATTN, OP_DECODE, OP_SCORE, OP_TOPK,
+               STATS_SPAN, ERR_UNSUPPORTED, LidxError, attn_args, decode_args, launch_count, lib, topk_args,
+               workspace, workspace_size)
 
 
 class LayerCache:
@@ -162,9 +163,13 @@ class DecodeStep:
         self.q_attn.copy_(q_attn, non_blocking=non_blocking)
 
     def kernel_launches(self) -> int:
-        """Kernels one step launches: per layer one fused kernel, or 1 scorer,
-        1 top-k, attention + merge."""
-        return self.L * (1 if self.fused else 4)
+        """Kernels one step launches, as the library reports them: per layer
+        one fused kernel, or the scorer, the top-k and the attention's split
+        and merge kernels."""
+        if self.fused:
+            return self.L
+        return sum(launch_count(OP_SCORE, self._score[l]) + launch_count(OP_TOPK, self._topk[l]) +
+                   launch_count(OP_ATTN, self._attn[l]) for l in range(self.L))
 
     def workspaces(self):
         """The workspaces whose status words the step's calls report into."""
@@ -288,8 +293,10 @@ class ModelStep:
         return o
 
     def kernel_launches(self) -> int:
-        """One launch per CSA layer; attention + merge per HCA and SWA layer."""
-        return sum(1 if k == CSA else 2 for k in self.kinds)
+        """The CSA step's kernels plus the attention kernels of every HCA and
+        SWA layer (as the library reports them)."""
+        return self.csa.kernel_launches() + sum(launch_count(OP_ATTN, a) for _, _, a, _ in self._calls
+                                                 if a is not None)
 
     def workspaces(self):
         return self.csa.workspaces() + [ws for _, _, _, ws in self._calls if ws is not None]

@@ -119,12 +119,30 @@ def test_attn_argument_errors_and_workspace(lib):
     a = L.AttnArgs(1, 64, L.BF16, 0x1000, kv, 16384, 0x2000, 512, 512, None, sw, 128, 0.044, 0x3000, None)
     n = C.c_size_t(0)
     assert lib.lidx_workspace_size(L.OP_ATTN, C.byref(a), C.byref(n)) == L.OK and n.value > 256
+    cnt = C.c_int(0)
+    assert lib.lidx_launch_count(L.OP_ATTN, C.byref(a), C.byref(cnt)) == L.OK and cnt.value == 2
     assert lib.lidx_sparse_attn_decode(C.byref(a), None, 0, None) == L.ERR_WORKSPACE
     kv16 = _kv(dtype=L.F16, dim=512, ld=512)
     f16 = L.AttnArgs(1, 64, L.BF16, 0x1000, kv16, 16384, 0x2000, 512, 512, None, sw, 128, 0.044, 0x3000, None)
     assert lib.lidx_sparse_attn_decode(C.byref(f16), C.c_void_p(0x10000), 1 << 30, None) == L.ERR_UNSUPPORTED
     nan = L.AttnArgs(1, 64, L.BF16, 0x1000, kv, 16384, 0x2000, 512, 512, None, sw, 128, float("nan"), 0x3000, None)
     assert lib.lidx_sparse_attn_decode(C.byref(nan), C.c_void_p(0x10000), 1 << 30, None) == L.ERR_INVALID_ARG
+
+
+def test_launch_count_arguments(lib):
+    """lidx_launch_count runs the call's own argument checks; the score call
+    is one kernel."""
+    kv = _kv()
+    a = L.ScoreArgs(1, 1, 64, 1000, L.BF16, 0x1000, 0x2000, kv, 0x3000, 1000, 0, None, None)
+    n = C.c_int(-1)
+    assert lib.lidx_launch_count(L.OP_SCORE, C.byref(a), C.byref(n)) == L.OK and n.value == 1
+    bad = L.ScoreArgs(1, 1, 64, 0, L.BF16, 0x1000, 0x2000, kv, 0x3000, 1000, 0, None, None)
+    assert lib.lidx_launch_count(L.OP_SCORE, C.byref(bad), C.byref(n)) == L.ERR_INVALID_ARG
+    assert lib.lidx_launch_count(L.OP_SCORE, C.byref(a), None) == L.ERR_INVALID_ARG
+    assert lib.lidx_launch_count(L.OP_SCORE, None, C.byref(n)) == L.ERR_INVALID_ARG
+    assert lib.lidx_launch_count(99, C.byref(a), C.byref(n)) == L.ERR_INVALID_ARG
+    t = L.TopkArgs(2, 1, 1000, 64, 0x1000, 1000, None, 0, 0x2000, None, None, None)
+    assert lib.lidx_launch_count(L.OP_TOPK, C.byref(t), C.byref(n)) == L.OK and n.value == 1
 
 
 def test_eval_argument_errors(lib):

@@ -8,7 +8,7 @@ import torch
 import lightning_indexer_top_index_b200 as L
 import oracle
 import synth
-from _helpers import (assert_attn_close, assert_scores_close, dev_kv, dev_q, score_bound,
+from _helpers import (assert_attn_close, assert_scores_close, dev_kv, dev_q, graph_kernel_count, score_bound,
                       topk_sets_equivalent)
 
 pytestmark = pytest.mark.gpu
@@ -40,6 +40,11 @@ def _score_case(spec, layer=0):
     synth.scaled(synth.DECODE_64K, N=16384),
     synth.scaled(synth.DECODE_64K, N=4099, B=3, H=32),
     synth.scaled(synth.DECODE_500K_FP8, N=3001, B=2),
+    # E4M3 keys over more tiles per CTA than the ring has stages (7 at 64
+    # heads, 6 at 128), so every stage and conversion buffer is reused
+    synth.scaled(synth.DECODE_500K_FP8, N=80000, B=2),
+    synth.scaled(synth.DECODE_500K_FP8, N=70001, B=2, H=128),
+    synth.scaled(synth.DECODE_500K_FP8, N=5000, B=3, H=32),
     synth.scaled(synth.DECODE_128K_B32, N=2500, B=2, k=64),
 ], ids=lambda s: f"{s.name}-N{s.N}-B{s.B}-H{s.H}")
 def test_score_parity(spec):
@@ -126,13 +131,27 @@ def test_topk_large_row():
     _topk_check(s, 1024)
 
 
-@pytest.mark.parametrize("N,k,rows,kind", [(300000, 1024, 1, "normal"), (300000, 1024, 2, "ties"),
-                                           (1000003, 512, 1, "signed"), (262145, 64, 3, "const")])
+@pytest.mark.parametrize("N,k,rows,kind", [(600000, 1024, 1, "normal"), (600000, 1024, 2, "ties"),
+                                           (1000003, 512, 1, "signed"), (524289, 64, 3, "const")])
 def test_topk_rows_beyond_one_cluster(N, k, rows, kind):
-    """Rows longer than one thread-block cluster holds (262,144 entries) take
-    the segmented path: bit-exact ids, n_sel, mask and bits all the same."""
+    """Rows longer than one thread-block cluster holds (524,288 entries on
+    16-CTA clusters) take the segmented path: bit-exact ids, n_sel, mask and
+    bits all the same."""
     s = synth.random_scores(27, rows, N, kind)
     _topk_check(s, k)
+
+
+@pytest.mark.parametrize("N,n_expected", [(16384, 1), (524288, 1), (524289, 4)])
+def test_topk_launch_count_matches_graph(N, n_expected):
+    """One cluster select up to 524,288 entries a row (16-CTA clusters); four
+    kernels beyond."""
+    st = torch.from_numpy(synth.random_scores(28, 2, N, "normal")).cuda().reshape(2, 1, N)
+    ids = torch.empty((2, 1, 512), dtype=torch.int32, device="cuda")
+    n_sel = torch.empty((2, 1), dtype=torch.int32, device="cuda")
+    a = L.topk_args(st, 512, None, ids, n_sel)
+    assert L.launch_count(L.OP_TOPK, a) == n_expected
+    ws = L.workspace(L.workspace_size(L.OP_TOPK, a))
+    assert graph_kernel_count(lambda s: L.topk_select(st, 512, ids=ids, n_sel=n_sel, ws=ws, stream=s)) == n_expected
 
 
 def test_topk_rows_beyond_one_cluster_masked_and_nan():
@@ -219,6 +238,29 @@ def _attn_case(spec, n_sel=None, swa_len=None, ids=None, layer=0):
 ], ids=lambda s: s.name)
 def test_attn_parity(spec):
     _attn_case(spec)
+
+
+@pytest.mark.parametrize("fmt", ["bf16", "e4m3"])
+@pytest.mark.parametrize("k,swa_len", [(20, 37), (64, 128), (384, 128), (448, 128), (512, 128), (896, 128),
+                                       (960, 128), (1024, 128)])
+def test_attn_split_counts(fmt, k, swa_len):
+    """1 to 18 splits of 64 rows (window rows first, then ids), bf16 and E4M3
+    rows, against the oracle; the kernel count the library reports against
+    the captured graph."""
+    base = synth.DECODE_64K if fmt == "bf16" else synth.DECODE_500K_FP8
+    spec = synth.scaled(base, N=3000, B=2, k=k)
+    _attn_case(spec, swa_len=swa_len)
+    inp = synth.decode_layer(spec, 0)
+    kv, swa = dev_kv(inp["kv"], batch_rows=spec.N), dev_kv(inp["swa"], batch_rows=spec.swa)
+    q = dev_q(inp["q_attn"], spec.q_dtype)
+    ids = torch.from_numpy(np.tile(np.arange(k, dtype=np.int32), (spec.B, 1))).cuda()
+    out = torch.empty(spec.B, 64, 512, device="cuda")
+    a = L.attn_args(q, kv, spec.N, ids, None, swa, swa_len, spec.scale, out, None)
+    n = L.launch_count(L.OP_ATTN, a)
+    assert n == 2
+    ws = L.workspace(L.workspace_size(L.OP_ATTN, a))  # (allocated outside the captured call)
+    assert graph_kernel_count(lambda s: L.sparse_attn_decode(q, kv, spec.N, ids, None, swa, swa_len, spec.scale,
+                                                              out=out, want_lse=False, ws=ws, stream=s)) == n
 
 
 def test_attn_partial_selection_and_short_window():
