@@ -235,9 +235,19 @@ def _attn_case(spec, n_sel=None, swa_len=None, ids=None, layer=0):
     synth.scaled(synth.DECODE_64K, N=3000),
     synth.scaled(synth.DECODE_500K_FP8, N=5000, B=2),
     synth.scaled(synth.DECODE_128K_B32, N=4000, B=3, plant=False),
-], ids=lambda s: s.name)
+    # batches whose 16-head grid needs more than one wave: 64 heads per CTA
+    synth.scaled(synth.DECODE_128K_B32, N=2000, B=8, plant=False),
+    synth.scaled(synth.DECODE_500K_FP8, N=3000, B=8, k=512),
+], ids=lambda s: f"{s.name}-B{s.B}")
 def test_attn_parity(spec):
     _attn_case(spec)
+
+
+def test_attn_wide_partial_selection_and_short_window():
+    """The 64-head layout (10 sequences x 9 chunks) with partial and empty
+    selections and a window shorter than a chunk."""
+    spec = synth.scaled(synth.DECODE_64K, N=2000, B=10, k=512)
+    _attn_case(spec, n_sel=[512, 100, 0, 512, 511, 1, 64, 300, 0, 450], swa_len=37)
 
 
 @pytest.mark.parametrize("fmt", ["bf16", "e4m3"])
