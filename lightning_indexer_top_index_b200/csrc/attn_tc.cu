@@ -3,16 +3,11 @@
 // rows plus the 128-row sliding window; K = V = the full row).
 //
 // Grid (row chunk, head group, sequence).  One CTA takes 64 entries of one
-// sequence's row list (the window rows first, then the selected ids) and a
-// group of the 64 query heads, and produces the split partial (m_h, l_h,
-// O_h) in base-2 units for those heads.  Two layouts:
-//   16 heads per CTA (256 threads, about 90 KB of shared memory, 256 TMEM
-//     columns, two CTAs per SM): a single decode sequence spreads over 40
-//     SMs;
-//   all 64 heads per CTA (512 threads, about 150 KB, 512 TMEM columns, one
-//     CTA per SM): each selected row is gathered once instead of once per
-//     head group, for batches whose 16-head grid would need more than one
-//     wave of the GPU.
+// sequence's row list (the window rows first, then the selected ids) and 16
+// of the 64 query heads, and produces the split partial (m_h, l_h, O_h) in
+// base-2 units for those heads.  Small CTAs (about 90 KB of shared memory,
+// 128 TMEM columns) let a single decode sequence spread over 40 SMs and two
+// CTAs share an SM.
 //   1. Q [16 heads][512] arrives by TMA.  A chunk made only of window rows
 //      (contiguous in memory) arrives as eight 64-row TMA boxes before the
 //      top-k kernel has finished; gathered bf16 rows are copied with
@@ -27,11 +22,11 @@
 //      128-byte swizzled line of 64 rows per head, hi heads then lo heads.
 //   4. MMA 2: [O_hi | O_lo]^T[d][.] = X^T . [P_hi | P_lo]^T (N = 32),
 //      reading the same X tile as an MN-major operand (K = V), four 128-wide
-//      d tiles into TMEM; the epilogue adds the two parts.  (64 heads: the lo
-//      part accumulates into the hi part's columns, N = 64, so that S and O
-//      fit TMEM's 512 columns.)
+//      d tiles into TMEM; the epilogue adds the two parts.
 //   5. Each warp stores two d tiles, lanes = consecutive d: coalesced stores.
-// The partials are combined by the split-K merge kernel.
+// The partials are combined by the split-K merge kernel.  Batches whose
+// grid would need more than one wave of the GPU go to the wide kernel
+// (attn_wide.cu) instead: all 64 heads and several chunks per CTA.
 #include "kernels.cuh"
 #include "tc.cuh"
 
@@ -39,45 +34,33 @@ namespace lidx {
 
 cudaError_t launch_attn_merge(const lidx_attn_args &a, const float *part_o, const float2 *part_ml, int n_split,
                               cudaStream_t st);
+cudaError_t launch_attn_wide(const lidx_attn_args &a, float *part_o, float2 *part_ml, int n_chunks, uint32_t *status,
+                             cudaStream_t st);
 
 namespace {
 
 constexpr int kD = 512;
 constexpr int kH = 64;                       // query heads of the supported layout
+constexpr int kHG = 16;                      // heads per CTA
+constexpr int kGroups = kH / kHG;
 constexpr int kRows = 64;                    // row-list entries per CTA
+constexpr int kThreads = 256;
 constexpr int kXBytes = kRows * kD * 2;      // 64 KB: 8 panels of [64 rows][128 B]
 constexpr int kXPanel = kRows * 128;         // 8 KB
-// These MMAs are tiny, and each costs its issuing thread a roughly fixed
-// time: so MMA 1 is issued by kS1 threads over K quarters into separate
-// partial sums, MMA 2 by four threads, one d tile each.
+constexpr int kQBytes = kHG * kD * 2;        // 16 KB: 8 panels of [16 heads][128 B]
+constexpr int kQPanel = kHG * 128;           // 2 KB
+constexpr int kPBytes = kHG * kRows * 2;     // 2 KB: one bf16 P^T [16 heads][64 rows]
+// TMEM: S^T as kS1 partial sums over K at columns [16i, 16i + 16) (M = 64:
+// row 16q + r in lane 32q + r), O^T tile t at [64 + 32t, 96 + 32t) as the
+// P_hi part (16 columns) then the P_lo part.  These MMAs are tiny, and each
+// costs its issuing thread a roughly fixed time: so MMA 1 is issued by kS1
+// threads over K quarters into separate partial sums, MMA 2 by four threads
+// (one d tile each) multiplying X^T by P_hi and P_lo at once (N = 32).
 constexpr int kS1 = 4;
+constexpr uint32_t kOCol = 64;
+constexpr uint32_t kTmemCols = 256;
 constexpr float kLog2e = 1.4426950408889634f;
 
-// A layout of HG heads per CTA.  TMEM: S^T as kS1 partial sums over K at
-// columns [HG i, HG i + HG) (M = 64: row 16q + r in lane 32q + r); O^T tile
-// t at kOCol + kOTile t: with 16 heads the P_hi part (16 columns) then the
-// P_lo part, with 64 heads both parts accumulated into 64 columns.  The
-// softmax puts warp w on row quarter w & 3 and head part w >> 2.
-template <int HG>
-struct Lay {
-  static constexpr int kHG = HG;
-  static constexpr int kGroups = kH / HG;
-  static constexpr int kThreads = HG == 16 ? 256 : 512;
-  static constexpr int kMinBlocks = HG == 16 ? 2 : 1;
-  static constexpr int kWarps = kThreads / 32;
-  static constexpr int kHParts = kWarps / 4;            // head parts of the softmax
-  static constexpr int kHPW = HG / kHParts;             // heads per softmax warp: 8 or 16
-  static constexpr int kQBytes = HG * kD * 2;           // 8 panels of [HG heads][128 B]
-  static constexpr int kQPanel = HG * 128;
-  static constexpr int kPBytes = HG * kRows * 2;        // one bf16 P^T [HG heads][64 rows]
-  static constexpr bool kSplitLo = HG == 16;            // hi and lo parts in their own columns
-  static constexpr uint32_t kOCol = kS1 * HG;
-  static constexpr uint32_t kOTile = kSplitLo ? 2 * HG : HG;
-  static constexpr uint32_t kTmemCols = HG == 16 ? 256 : 512;
-  static_assert(kOCol + 4 * kOTile <= kTmemCols, "TMEM columns");
-};
-
-template <int HG>
 struct __align__(8) AttnTcSmem {
   uint64_t q_full;
   uint64_t s_full;
@@ -86,15 +69,12 @@ struct __align__(8) AttnTcSmem {
   uint32_t abort;
   int64_t row_src[kRows];  // row index in its cache; -1 when empty
   int32_t row_kind[kRows]; // 0 none, 1 selected, 2 window
-  float red[Lay<HG>::kHParts][4][Lay<HG>::kHPW];  // per head part, per row quarter
+  float red[2][4][8];      // per head half, per row quarter
 };
 
-// smem: X (64 KB) | Q | P^T hi, lo | bookkeeping.  Q follows X so that MMA
-// 1's padding rows stay inside the allocation.
-template <int HG>
-constexpr size_t smem_bytes() {
-  return 1024 + kXBytes + Lay<HG>::kQBytes + 2 * Lay<HG>::kPBytes + sizeof(AttnTcSmem<HG>);
-}
+// smem: X (64 KB) | Q (16 KB) | P^T hi, lo (2 x 2 KB) | bookkeeping.  Q
+// follows X so that MMA 1's padding rows stay inside the allocation.
+constexpr size_t smem_bytes() { return 1024 + kXBytes + kQBytes + 2 * kPBytes + sizeof(AttnTcSmem); }
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
@@ -109,20 +89,16 @@ __device__ __forceinline__ uint32_t x_off(int r, int c) {
   return (c >> 3) * kXPanel + r * 128 + (((c & 7) ^ (r & 7)) << 4);
 }
 
-template <bool kFp8, int HG>
-__global__ void __launch_bounds__(Lay<HG>::kThreads, Lay<HG>::kMinBlocks)
+template <bool kFp8>
+__global__ void __launch_bounds__(kThreads, 2)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_win,
                    const lidx_attn_args a, float *part_o, float2 *part_ml, int n_split, uint32_t *status) {
-  using T = Lay<HG>;
-  constexpr int kHG = HG, kThreads = T::kThreads, kQBytes = T::kQBytes, kQPanel = T::kQPanel,
-                kPBytes = T::kPBytes, kHPW = T::kHPW;
-  constexpr uint32_t kOCol = T::kOCol, kTmemCols = T::kTmemCols;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sX = smem;
   uint8_t *sQ = sX + kXBytes;
   uint8_t *sP = sQ + kQBytes;  // P^T hi at +0, lo at +kPBytes
-  AttnTcSmem<HG> *sm = reinterpret_cast<AttnTcSmem<HG> *>(sP + 2 * kPBytes);
+  AttnTcSmem *sm = reinterpret_cast<AttnTcSmem *>(sP + 2 * kPBytes);
   volatile uint32_t *abort_flag = &sm->abort;
 
   const int split = blockIdx.x, hg = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
@@ -292,8 +268,7 @@ __global__ void __launch_bounds__(Lay<HG>::kThreads, Lay<HG>::kMinBlocks)
         const int k = warp * (32 / kS1) + kk;
         const uint32_t ao = (k >> 2) * kXPanel + (k & 3) * 32;
         const uint32_t bo = (k >> 2) * kQPanel + (k & 3) * 32;
-        tc::mma_bf16(tmem + kHG * warp, tc::desc_kmajor_sw128(xs + ao), tc::desc_kmajor_sw128(qs + bo), idesc,
-                     kk > 0);
+        tc::mma_bf16(tmem + 16 * warp, tc::desc_kmajor_sw128(xs + ao), tc::desc_kmajor_sw128(qs + bo), idesc, kk > 0);
       }
       tc::mma_commit(&sm->s_full);
     }
@@ -301,52 +276,47 @@ __global__ void __launch_bounds__(Lay<HG>::kThreads, Lay<HG>::kMinBlocks)
 
   // ---- 3. softmax over the 64 rows, per head: warp w takes row quarter
   // q = w&3 (rows 16q + lane, lanes 0-15; M = 64 puts them in TMEM lanes
-  // 32q..32q+15) and the kHPW heads of head part hp = w>>2
-  const int quarter = warp & 3, hp = warp >> 2;
+  // 32q..32q+15) and heads 8h.. with h = w>>2
+  const int quarter = warp & 3, half = warp >> 2;
   bool ready = false;
   if (lane == 0) ready = tc::mbar_wait(&sm->s_full, 0, abort_flag);
   ready = __shfl_sync(0xFFFFFFFFu, ready, 0);
-  auto ld_heads = [&](uint32_t ta, float *v) {
-    if (kHPW == 8)
-      tc::tmem_ld8(ta, v);
-    else
-      tc::tmem_ld16(ta, v);
-  };
-  float mx[kHPW];
+  float mx[8];
   {
     const int r = quarter * 16 + (lane & 15);
     const bool valid = lane < 16 && sm->row_kind[r] != 0;
-    float s[kHPW];
+    float s[8];
     if (ready) {
       tc::tc_fence_after();
-      const uint32_t ta = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + hp * kHPW;
-      ld_heads(ta, s);
+      const uint32_t ta = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + half * 8;
+      tc::tmem_ld8(ta, s);
 #pragma unroll
       for (int i = 1; i < kS1; i++) {
-        float t[kHPW];
-        ld_heads(ta + kHG * i, t);
+        float t8[8];
+        tc::tmem_ld8(ta + 16 * i, t8);
 #pragma unroll
-        for (int h = 0; h < kHPW; h++) s[h] += t[h];
+        for (int h = 0; h < 8; h++) s[h] += t8[h];
       }
     }
     const float c2 = a.scale * kLog2e;
 #pragma unroll
-    for (int h = 0; h < kHPW; h++) {
+    for (int h = 0; h < 8; h++) {
       s[h] = valid && ready ? s[h] * c2 : -INFINITY;
       mx[h] = s[h];
     }
 #pragma unroll
     for (int o = 8; o > 0; o >>= 1)  // lanes 16-31 hold -inf copies: reduce within 16
 #pragma unroll
-      for (int h = 0; h < kHPW; h++) mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xFFFFFFFFu, mx[h], o));
+      for (int h = 0; h < 8; h++) mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xFFFFFFFFu, mx[h], o));
     if (lane == 0)
 #pragma unroll
-      for (int h = 0; h < kHPW; h++) sm->red[hp][quarter][h] = mx[h];
-    named_sync(1 + hp, 128);
-    float pv[kHPW];
+      for (int h = 0; h < 8; h++) sm->red[half][quarter][h] = mx[h];
+    named_sync(1 + half, 128);
+    float pv[8];
 #pragma unroll
-    for (int h = 0; h < kHPW; h++) {
-      const float m = fmaxf(fmaxf(sm->red[hp][0][h], sm->red[hp][1][h]), fmaxf(sm->red[hp][2][h], sm->red[hp][3][h]));
+    for (int h = 0; h < 8; h++) {
+      const float m = fmaxf(fmaxf(sm->red[half][0][h], sm->red[half][1][h]),
+                            fmaxf(sm->red[half][2][h], sm->red[half][3][h]));
       mx[h] = m;
       pv[h] = (m == -INFINITY || s[h] == -INFINITY) ? 0.f : exp2f(s[h] - m);
     }
@@ -354,8 +324,8 @@ __global__ void __launch_bounds__(Lay<HG>::kThreads, Lay<HG>::kMinBlocks)
     // rows in 16-byte chunks of 8, chunk index swizzled with h & 7
     if (lane < 16) {
 #pragma unroll
-      for (int i = 0; i < kHPW; i++) {
-        const int h = hp * kHPW + i;
+      for (int i = 0; i < 8; i++) {
+        const int h = half * 8 + i;
         const __nv_bfloat16 ph = __float2bfloat16_rn(pv[i]);
         const __nv_bfloat16 pl = __float2bfloat16_rn(pv[i] - __bfloat162float(ph));
         const int off = h * 128 + ((((r >> 3) ^ (h & 7))) << 4) + (r & 7) * 2;
@@ -363,27 +333,27 @@ __global__ void __launch_bounds__(Lay<HG>::kThreads, Lay<HG>::kMinBlocks)
         *reinterpret_cast<__nv_bfloat16 *>(sP + kPBytes + off) = pl;
       }
     }
-    float sum[kHPW];
+    float sum[8];
 #pragma unroll
-    for (int h = 0; h < kHPW; h++) sum[h] = lane < 16 ? pv[h] : 0.f;
+    for (int h = 0; h < 8; h++) sum[h] = lane < 16 ? pv[h] : 0.f;
 #pragma unroll
     for (int o = 8; o > 0; o >>= 1)
 #pragma unroll
-      for (int h = 0; h < kHPW; h++) sum[h] += __shfl_xor_sync(0xFFFFFFFFu, sum[h], o);
-    named_sync(1 + hp, 128);  // the four warps have read the maxima
+      for (int h = 0; h < 8; h++) sum[h] += __shfl_xor_sync(0xFFFFFFFFu, sum[h], o);
+    named_sync(1 + half, 128);  // the four warps have read the maxima
     if (lane == 0)
 #pragma unroll
-      for (int h = 0; h < kHPW; h++) sm->red[hp][quarter][h] = sum[h];
-    named_sync(1 + hp, 128);
+      for (int h = 0; h < 8; h++) sm->red[half][quarter][h] = sum[h];
+    named_sync(1 + half, 128);
   }
   if (pure_window) pdl_wait();  // no global write before the previous kernel is done
-  if (quarter == 0 && lane < kHPW) {
-    const float l = (sm->red[hp][0][lane] + sm->red[hp][1][lane]) + (sm->red[hp][2][lane] + sm->red[hp][3][lane]);
+  if (quarter == 0 && lane < 8) {
+    const float l = (sm->red[half][0][lane] + sm->red[half][1][lane]) + (sm->red[half][2][lane] + sm->red[half][3][lane]);
     float m = mx[0];
 #pragma unroll
-    for (int i = 1; i < kHPW; i++)
+    for (int i = 1; i < 8; i++)
       if (i == lane) m = mx[i];
-    part_ml[(static_cast<size_t>(b) * n_split + split) * kH + hg * kHG + hp * kHPW + lane] = make_float2(m, l);
+    part_ml[(static_cast<size_t>(b) * n_split + split) * kH + hg * kHG + half * 8 + lane] = make_float2(m, l);
   }
   tc::fence_proxy_async_smem();
   tc::tc_fence_before();
@@ -392,32 +362,19 @@ __global__ void __launch_bounds__(Lay<HG>::kThreads, Lay<HG>::kMinBlocks)
   // ---- 4. O^T = X^T . (P_hi + P_lo)^T: lane 0 of warp dt < 4 issues d tile dt
   if (warp < 4 && lane == 0 && !*abort_flag) {
     tc::tc_fence_after();
+    const uint32_t idesc = tc::idesc_bf16(128, 2 * kHG, true, false);
     const uint32_t ps = tc::smem_u32(sP);
     const int dt = warp;
-    const uint32_t d = tmem + kOCol + T::kOTile * dt;
-    if (T::kSplitLo) {
-      const uint32_t idesc = tc::idesc_bf16(128, 2 * kHG, true, false);
 #pragma unroll
-      for (int kk = 0; kk < kRows / 16; kk++) {
-        const uint64_t adesc = tc::desc_mnmajor_sw128(xs + 2 * dt * kXPanel + kk * 2048, kXPanel, 1024);
-        const uint64_t bdesc = tc::desc_kmajor_sw128(ps + kk * 32);  // 2 kHG lines: hi heads, then lo heads
-        tc::mma_bf16(d, adesc, bdesc, idesc, kk > 0);
-      }
-    } else {
-      const uint32_t idesc = tc::idesc_bf16(128, kHG, true, false);
-#pragma unroll
-      for (int part = 0; part < 2; part++)  // P_hi, then P_lo into the same columns
-#pragma unroll
-        for (int kk = 0; kk < kRows / 16; kk++) {
-          const uint64_t adesc = tc::desc_mnmajor_sw128(xs + 2 * dt * kXPanel + kk * 2048, kXPanel, 1024);
-          const uint64_t bdesc = tc::desc_kmajor_sw128(ps + part * kPBytes + kk * 32);
-          tc::mma_bf16(d, adesc, bdesc, idesc, part > 0 || kk > 0);
-        }
+    for (int kk = 0; kk < kRows / 16; kk++) {
+      const uint64_t adesc = tc::desc_mnmajor_sw128(xs + 2 * dt * kXPanel + kk * 2048, kXPanel, 1024);
+      const uint64_t bdesc = tc::desc_kmajor_sw128(ps + kk * 32);  // 32 lines: hi heads, then lo heads
+      tc::mma_bf16(tmem + kOCol + 32 * dt, adesc, bdesc, idesc, kk > 0);
     }
     tc::mma_commit(&sm->o_full);
   }
 
-  // ---- 5. partial O out: warp w stores d tiles hp, hp + kHParts, ... of its
+  // ---- 5. partial O out: warp w stores d tiles (w>>2) and (w>>2)+2 of its
   // TMEM lane quarter; lanes = consecutive d
   bool oready = false;
   if (lane == 0) oready = !*abort_flag && tc::mbar_wait(&sm->o_full, 0, abort_flag);
@@ -426,22 +383,13 @@ __global__ void __launch_bounds__(Lay<HG>::kThreads, Lay<HG>::kMinBlocks)
     tc::tc_fence_after();
     float *po = part_o + ((static_cast<size_t>(b) * n_split + split) * kH + hg * kHG) * kD;
 #pragma unroll
-    for (int dt = hp; dt < 4; dt += T::kHParts) {
+    for (int j = 0; j < 2; j++) {
+      const int dt = (warp >> 2) + 2 * j;
       const int d = dt * 128 + quarter * 32 + lane;
-      const uint32_t ta = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + kOCol + T::kOTile * dt;
       float v[32];
-      if (T::kSplitLo) {
-        tc::tmem_ld32(ta, v);
+      tc::tmem_ld32(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + kOCol + 32 * dt, v);
 #pragma unroll
-        for (int h = 0; h < kHG; h++) po[h * kD + d] = v[h] + v[kHG + h];
-      } else {
-#pragma unroll
-        for (int h0 = 0; h0 < kHG; h0 += 32) {
-          tc::tmem_ld32(ta + h0, v);
-#pragma unroll
-          for (int h = 0; h < 32; h++) po[(h0 + h) * kD + d] = v[h];
-        }
-      }
+      for (int h = 0; h < kHG; h++) po[h * kD + d] = v[h] + v[kHG + h];
     }
   }
   tc::tc_fence_before();
@@ -479,47 +427,43 @@ int sm_count() {
   return n;
 }
 
-template <bool kFp8, int HG>
-cudaError_t launch_lay(const lidx_attn_args &a, const CUtensorMap &tm_win, float *part_o, float2 *part_ml, int n_split,
-                       uint32_t *status, cudaStream_t st) {
-  CUtensorMap tm_q;
-  if (!make_tmap_2d(&tm_q, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kD, static_cast<uint64_t>(a.B) * kH, kD * 2, 64, HG,
-                    CU_TENSOR_MAP_SWIZZLE_128B))
-    return cudaErrorInvalidValue;
-  const size_t smem = smem_bytes<HG>();
-  cudaFuncSetAttribute(attn_tc_kernel<kFp8, HG>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-  return launch_kernel(attn_tc_kernel<kFp8, HG>, dim3(n_split, Lay<HG>::kGroups, a.B), dim3(Lay<HG>::kThreads), smem,
-                       st, (a.flags & LIDX_LAUNCH_PDL) != 0, tm_q, tm_win, a, part_o, part_ml, n_split, status);
-}
-
 }  // namespace
 
-// All 64 heads in one CTA once the 16-head grid (four CTAs per row chunk,
-// two CTAs per SM) would need more than one wave of the GPU.
+// The wide kernel once this kernel's grid (four head-group CTAs per row
+// chunk, two CTAs per SM) would need more than one wave of the GPU.
 bool attn_tc_wide(const lidx_attn_args &a) {
-  return static_cast<int64_t>(a.B) * attn_tc_splits(a) * Lay<16>::kGroups > 2ll * sm_count();
+  return static_cast<int64_t>(a.B) * attn_tc_splits(a) * kGroups > 2ll * sm_count();
 }
 
 cudaError_t launch_attn_tc(const lidx_attn_args &a, float *part_o, float2 *part_ml, int n_split, uint32_t *status,
                            cudaStream_t st) {
+  if (attn_tc_wide(a)) return launch_attn_wide(a, part_o, part_ml, n_split, status, st);
+  CUtensorMap tm_q;
+  if (!make_tmap_2d(&tm_q, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kD, static_cast<uint64_t>(a.B) * kH, kD * 2, 64, kHG,
+                    CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
   const int dt = a.n_ids > 0 ? a.kv.dtype : a.swa.dtype;
-  // window rows of one chunk as one 64-row box per 64-dim panel (a valid
-  // placeholder map otherwise: the kernel then never uses it)
-  CUtensorMap tm_win;
+  // window rows of one chunk as one 64-row box per 64-dim panel
+  CUtensorMap tm_win = tm_q;
   if (dt == LIDX_BF16 && a.swa_len >= kRows) {
     const uint64_t rows = static_cast<uint64_t>(a.B - 1) * (a.B > 1 ? a.swa.batch_rows : 0) + a.swa_len;
     if (!make_tmap_2d(&tm_win, a.swa.data, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kD, rows, a.swa.ld * 2, 64, kRows,
                       CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
-  } else if (!make_tmap_2d(&tm_win, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kD, static_cast<uint64_t>(a.B) * kH, kD * 2,
-                           64, 16, CU_TENSOR_MAP_SWIZZLE_128B)) {
-    return cudaErrorInvalidValue;
   }
-  const bool wide = attn_tc_wide(a);
-  cudaError_t e = dt == LIDX_E4M3 ? (wide ? launch_lay<true, 64>(a, tm_win, part_o, part_ml, n_split, status, st)
-                                          : launch_lay<true, 16>(a, tm_win, part_o, part_ml, n_split, status, st))
-                                  : (wide ? launch_lay<false, 64>(a, tm_win, part_o, part_ml, n_split, status, st)
-                                          : launch_lay<false, 16>(a, tm_win, part_o, part_ml, n_split, status, st));
+  const size_t smem = smem_bytes();
+  dim3 grid(n_split, kGroups, a.B);
+  const bool pdl = (a.flags & LIDX_LAUNCH_PDL) != 0;
+  cudaError_t e;
+  if (dt == LIDX_E4M3) {
+    cudaFuncSetAttribute(attn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    e = launch_kernel(attn_tc_kernel<true>, grid, dim3(kThreads), smem, st, pdl, tm_q, tm_win, a, part_o, part_ml, n_split,
+                      status);
+  } else {
+    cudaFuncSetAttribute(attn_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    e = launch_kernel(attn_tc_kernel<false>, grid, dim3(kThreads), smem, st, pdl, tm_q, tm_win, a, part_o, part_ml, n_split,
+                      status);
+  }
   if (e != cudaSuccess) return e;
   return launch_attn_merge(a, part_o, part_ml, n_split, st);
 }

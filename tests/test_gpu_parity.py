@@ -243,6 +243,25 @@ def test_attn_parity(spec):
     _attn_case(spec)
 
 
+@pytest.mark.parametrize("fmt,B,n_sel,swa_len", [
+    ("bf16", 32, None, 128),
+    ("e4m3", 32, None, 128),
+    ("bf16", 40, "mixed", 37),
+    ("bf16", 37, "mixed", 128),
+])
+def test_attn_wide_several_chunks_per_cta(fmt, B, n_sel, swa_len):
+    """Batches past 148 / chunks sequences: each CTA folds several 64-row
+    chunks with the online softmax (the accumulated O rescaled when a chunk
+    raises a head's maximum), including CTAs whose chunks hold no row."""
+    base = synth.DECODE_128K_B32 if fmt == "bf16" else synth.DECODE_500K_FP8
+    kw = dict(plant=False) if fmt == "bf16" else {}
+    spec = synth.scaled(base, N=1500, B=B, k=512, **kw)
+    ns = None
+    if n_sel == "mixed":
+        ns = [[512, 0, 77, 511, 1, 300, 64, 200][b % 8] for b in range(B)]
+    _attn_case(spec, n_sel=ns, swa_len=swa_len)
+
+
 def test_attn_wide_partial_selection_and_short_window():
     """The 64-head layout (10 sequences x 9 chunks) with partial and empty
     selections and a window shorter than a chunk."""
