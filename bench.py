@@ -113,7 +113,7 @@ def peaks() -> dict:
 CALL_SOURCES = {
     "score": ("score_tc.cu", "score_cc.cu"),
     "topk": ("topk.cu",),
-    "attn": ("attn.cu", "attn_tc.cu"),
+    "attn": ("attn.cu", "attn_tc.cu", "attn_wide.cu"),
     "layer": ("decode_fused.cu",),
     "golden": ("golden_tc.cu", "eval.cu"),
 }
