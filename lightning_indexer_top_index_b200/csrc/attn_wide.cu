@@ -86,6 +86,23 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// 16 consecutive fp32 columns of this thread's TMEM lane, without waiting;
+// tmem_ld16_pin (after tcgen05.wait::ld) keeps their uses after the wait.
+__device__ __forceinline__ void tmem_ld16_issue(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld16_pin(uint32_t (&r)[16]) {
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                 "+r"(r[15]));
+}
+
 template <bool kFp8>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_wide_kernel(const __grid_constant__ CUtensorMap tm_q, const lidx_attn_args a, float *part_o,
@@ -196,20 +213,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   for (int c = c0; c < c1; c++) {
     const int buf = (c - c0) & 1;
     const uint32_t par = static_cast<uint32_t>((c - c0) & 1);
-    // MMA 2 of the previous chunk has finished: its X buffer, P and O are free
-    if (c > c0) {
-      bool ok = true;
-      if (lane == 0) ok = tc::mbar_wait(&sm->o_full, par ^ 1u, abort_flag);
-      __syncwarp();
-      (void)ok;
-    }
-    tc::tc_fence_after();
-    if (c + 1 < c1) {
-      load_chunk(c + 1, buf ^ 1);
-      asm volatile("cp.async.wait_group 1;" ::: "memory");
-    } else {
-      asm volatile("cp.async.wait_group 0;" ::: "memory");
-    }
+    // this chunk's rows (gathered one iteration earlier) are in
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
     // (every thread read the previous chunk's flag before that chunk's
     // rescale barrier, or it was already clear)
     if (tid == 0) sm->rescale = 0u;
@@ -234,6 +239,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
 
+    // MMA 1 touches nothing MMA 2 of the previous chunk uses; once that has
+    // finished, its X buffer, P and O are free: gather the next chunk
+    if (c > c0 && lane == 0) tc::mbar_wait(&sm->o_full, par ^ 1u, abort_flag);
+    __syncwarp();
+    tc::tc_fence_after();
+    if (c + 1 < c1) load_chunk(c + 1, buf ^ 1);
+
     // ---- online softmax: thread (quarter q, lane l < 16) owns head 16q + l
     // and rows 16 rp .. 16 rp + 15 (TMEM lane 32q + l, M = 64)
     bool ready = false;
@@ -243,14 +255,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ready) {
       tc::tc_fence_after();
       const uint32_t ta = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + 16 * rp;
-      tc::tmem_ld16(ta, s);
+      uint32_t t[kS1][16];
 #pragma unroll
-      for (int i = 1; i < kS1; i++) {
-        float t[16];
-        tc::tmem_ld16(ta + 64 * i, t);
+      for (int i = 0; i < kS1; i++) tmem_ld16_issue(ta + 64 * i, t[i]);
+      tc::tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 16; j++) s[j] += t[j];
-      }
+      for (int i = 0; i < kS1; i++) tmem_ld16_pin(t[i]);
+#pragma unroll
+      for (int j = 0; j < 16; j++)
+        s[j] = (__uint_as_float(t[0][j]) + __uint_as_float(t[1][j])) + (__uint_as_float(t[2][j]) + __uint_as_float(t[3][j]));
     }
     float mloc = -INFINITY;
 #pragma unroll
