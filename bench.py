@@ -306,16 +306,17 @@ def timed_loop(fn, steps: int, repeats: int, dist, device, between=None, begin=N
 
 
 def pipelined_e2e(steps, h2d, d2h):
-    """End-to-end steps over the rotating replicas with the copies on a side
-    stream: step i copies its inputs into replica i % R (h2d(step)), replays
-    it, and copies its result back (d2h(step, r)); the copy of step i+1's
-    inputs overlaps step i.  Events keep a replica's inputs and outputs from
-    being overwritten while in use.  Returns (step(i), begin(), end()): begin
-    orders the side stream after the region's start, end makes the current
-    stream wait for the last copies."""
+    """End-to-end steps over the rotating replicas with the copies on two side
+    streams, one per direction (PCIe carries both at once): step i copies its
+    inputs into replica i % R (h2d(step)), replays it, and copies its result
+    back (d2h(step, r)); the copy of step i+1's inputs and the copy of step
+    i's result both overlap the steps around them.  Events keep a replica's
+    inputs and outputs from being overwritten while in use.  Returns
+    (step(i), begin(), end()): begin orders the side streams after the
+    region's start, end makes the current stream wait for the last copies."""
     import torch
     R = len(steps)
-    side = torch.cuda.Stream()
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
     h2d_done = [torch.cuda.Event() for _ in range(R)]
     used = [torch.cuda.Event() for _ in range(R)]     # the replica's step has read its inputs
     d2h_done = [torch.cuda.Event() for _ in range(R)]
@@ -323,10 +324,10 @@ def pipelined_e2e(steps, h2d, d2h):
 
     def copy_in(i):
         r = i % R
-        with torch.cuda.stream(side):
-            side.wait_event(used[r])
+        with torch.cuda.stream(up):
+            up.wait_event(used[r])
             h2d(steps[r])
-            h2d_done[r].record(side)
+            h2d_done[r].record(up)
 
     def step(i):
         main = torch.cuda.current_stream()
@@ -339,17 +340,19 @@ def pipelined_e2e(steps, h2d, d2h):
         used[r].record(main)
         copy_in(i + 1)
         state["next"] = i + 2
-        with torch.cuda.stream(side):
-            side.wait_event(used[r])
+        with torch.cuda.stream(down):
+            down.wait_event(used[r])
             d2h(steps[r], r)
-            d2h_done[r].record(side)
+            d2h_done[r].record(down)
 
     def begin():
-        side.wait_stream(torch.cuda.current_stream())
+        up.wait_stream(torch.cuda.current_stream())
+        down.wait_stream(torch.cuda.current_stream())
         state["next"] = 0
 
     def end():
-        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.current_stream().wait_stream(up)
+        torch.cuda.current_stream().wait_stream(down)
 
     return step, begin, end
 
