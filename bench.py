@@ -707,19 +707,40 @@ def measure_eval(args, world, dist, device, local_rank, rank, want_cpu) -> dict:
         torch.cuda.synchronize()
         for n in EVAL_STAGES:
             stage_ms[n] += ev[n][0].elapsed_time(ev[n][1]) / reps
+    # end to end: pinned host queries in, the overlap counts back, every
+    # window; two windows over the same caches, each with its own inputs, so
+    # the next window's queries go in while this one computes
     pins = [t.pin_memory() for t in (q_idx_h, w_h, qa_h, gq_h, gu_h)]
-    outs_src = (win.counts_nat_gold, win.counts_nat_f, win.counts_g_f, win.counts_natf_gold, win.counts_natf_nat)
-    outs = [torch.empty(c.shape, dtype=c.dtype).pin_memory() for c in outs_src]
-    dsts = (win.q_idx, win.w, win.qa, gq, gu)
+    win2_in = [t.clone() for t in (q_idx, w, qa, gq, gu)]
+    win2 = EvalWindow(keys, kv_all, *win2_in, spec.gate_layers, spec.N, spec.k,
+                      (spec.top_p_num, spec.top_p_den), spec.min_votes, spec.scale)
 
-    def e2e_step(i):
-        for d, hsrc in zip(dsts, pins):
+    class _Window:  # the replica interface pipelined_e2e drives
+        def __init__(self, wnd, inputs):
+            self.wnd, self.inputs = wnd, inputs
+            self.outs_src = (wnd.counts_nat_gold, wnd.counts_nat_f, wnd.counts_g_f, wnd.counts_natf_gold,
+                             wnd.counts_natf_nat)
+
+        def replay(self):
+            self.wnd.enqueue()
+
+    wins = [_Window(win, (q_idx, w, qa, gq, gu)), _Window(win2, win2_in)]
+    outs = [[torch.empty(c.shape, dtype=c.dtype).pin_memory() for c in x.outs_src] for x in wins]
+
+    def h2d(x):
+        for d, hsrc in zip(x.inputs, pins):
             d.copy_(hsrc, non_blocking=True)
-        win.enqueue()
-        for o, c in zip(outs, outs_src):
+
+    def d2h(x, r):
+        for o, c in zip(outs[r], x.outs_src):
             o.copy_(c, non_blocking=True)
 
-    e2e_ms, _ = timed_loop(e2e_step, steps, args.repeats, dist, device)
+    e2e_step, e2e_begin, e2e_end = pipelined_e2e(wins, h2d, d2h)
+    e2e_begin()
+    for i in range(2):
+        e2e_step(i)
+    e2e_end()
+    e2e_ms, _ = timed_loop(e2e_step, steps, args.repeats, dist, device, begin=e2e_begin, end=e2e_end)
     pk = peaks()
     gflops = win.golden_flops()
     achieved = gflops / (stage_ms["golden"] * 1e-3) / 1e12
@@ -738,7 +759,7 @@ def measure_eval(args, world, dist, device, local_rank, rank, want_cpu) -> dict:
                        "frac_of_sustained": score_tflops / peak, "ms_per_window": stage_ms["score"]},
         "e2e": {"value": job_rate(1, world, e2e_ms), "unit": "windows/s",
                 "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in pins),
-                "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in outs)},
+                "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in outs[0])},
         "gpu_launches": steps * args.repeats * win.kernel_launches(),
         "gpu_launches_per_step": win.kernel_launches(),
         "clocks": clk,
@@ -751,7 +772,7 @@ def measure_eval(args, world, dist, device, local_rank, rank, want_cpu) -> dict:
                                "kind": "oracle",
                                "sample": f"{n} (query, layer) golden rows with their top-p and top-k on {cores} "
                                          f"host threads ({n}/{spec.L * spec.T} of a window)"}
-    del win
+    del win, win2, wins
     torch.cuda.empty_cache()
     return res
 
