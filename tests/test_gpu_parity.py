@@ -481,6 +481,9 @@ def test_vote_union_lsa_overlap_bit_exact(N):
     (synth.scaled(synth.DECODE_64K, N=300, k=300, B=2), 0),
     (synth.scaled(synth.DECODE_500K_FP8, N=3907, k=3907, B=2), 128),
     (synth.scaled(synth.TINY_1K_F32, N=32, k=32), 128),
+    # many sequences: the wide kernel (several chunks per CTA)
+    (synth.scaled(synth.DECODE_64K, N=512, k=512, B=40), 128),
+    (synth.scaled(synth.DECODE_500K_FP8, N=700, k=700, B=36), 77),
 ], ids=lambda x: f"{x.name}-N{x.N}-B{x.B}" if hasattr(x, "name") else f"swa{x}")
 def test_attn_dense_rows_hca(spec, swa_len):
     """The HCA layers of the architecture post (section (A): 128:1
