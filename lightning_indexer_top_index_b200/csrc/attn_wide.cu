@@ -12,9 +12,11 @@
 //   * S[head][row] = Q . X^T (M = 64 heads, N = 64 rows, K = 512) into TMEM,
 //     issued by four threads over K quarters into partial sums; with the
 //     heads on M, each softmax thread owns one head and 16 of the rows.
-//   * The running maximum M_h and sum L_h live in shared memory; when a chunk
-//     raises M_h, the O accumulated so far is rescaled by 2^(M_old - M_new)
-//     in TMEM (read, scale, write back) before the chunk's MMA adds to it.
+//   * The running reference maximum M_h and sum L_h live in shared memory;
+//     when a chunk raises the maximum by more than 8 (base 2), M_h moves and
+//     the O accumulated so far is rescaled by 2^(M_old - M_new) in TMEM
+//     (read, scale, write back) before the chunk's MMA adds to it; smaller
+//     rises keep M_h, so probabilities stay below 2^8 and the rescale is rare.
 //   * O^T[d][head] += X^T . P^T (M = 128 d, N = 64 heads, K = 64 rows), P
 //     carried as bf16 hi + lo parts accumulated into the same columns.
 //   * The next chunk's rows are gathered into a second buffer while the
@@ -43,6 +45,7 @@ constexpr int kS1 = 4;                   // K-split partial sums of S
 constexpr uint32_t kOCol = kS1 * 64;     // O^T tile t at columns kOCol + 64 t
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLazy = 8.f;             // base-2 headroom of the reference maximum
 
 struct __align__(8) WideSmem {
   uint64_t q_full;
@@ -221,18 +224,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::fence_proxy_async_smem();
     __syncthreads();
 
-    // ---- S[head][row] = Q . X^T: lane 0 of warp i < kS1 issues K steps [8i, 8i + 8)
+    // ---- S[head][row] = Q . X^T: lane 0 of warp 4 + i (i < kS1) issues K
+    // steps [8i, 8i + 8).  Other threads than MMA 2's, so that the commit of
+    // S does not also wait for the previous chunk's O.
     const uint32_t xs = tc::smem_u32(sX + buf * kXBytes);
-    if (warp < kS1 && lane == 0 && !*abort_flag) {
+    if (warp >= 4 && warp < 4 + kS1 && lane == 0 && !*abort_flag) {
       if (c > c0 || tc::mbar_wait(&sm->q_full, 0, abort_flag)) {
         tc::tc_fence_after();
         const uint32_t idesc = tc::idesc_bf16(64, 64);
         const uint32_t qs = tc::smem_u32(sQ);
 #pragma unroll
+        const int part = warp - 4;
         for (int kk = 0; kk < 32 / kS1; kk++) {
-          const int k = warp * (32 / kS1) + kk;
+          const int k = part * (32 / kS1) + kk;
           const uint32_t off = (k >> 2) * kPanel + (k & 3) * 32;
-          tc::mma_bf16(tmem + 64 * warp, tc::desc_kmajor_sw128(qs + off), tc::desc_kmajor_sw128(xs + off), idesc,
+          tc::mma_bf16(tmem + 64 * part, tc::desc_kmajor_sw128(qs + off), tc::desc_kmajor_sw128(xs + off), idesc,
                        kk > 0);
         }
         tc::mma_commit(&sm->s_full);
@@ -274,9 +280,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (lane < 16) sm->red_m[rp][head] = mloc;
     named_sync(1 + quarter, 128);
+    // The reference maximum moves only when the chunk raises it by more than
+    // kLazy (so p stays below 2^kLazy and O is rescaled rarely); (m, l, O)
+    // stay consistent with it, which is all the merge needs.
     const float m_old = sm->run_m[head];
-    const float m_new = fmaxf(m_old, fmaxf(fmaxf(sm->red_m[0][head], sm->red_m[1][head]),
-                                           fmaxf(sm->red_m[2][head], sm->red_m[3][head])));
+    const float m_hi = fmaxf(m_old, fmaxf(fmaxf(sm->red_m[0][head], sm->red_m[1][head]),
+                                          fmaxf(sm->red_m[2][head], sm->red_m[3][head])));
+    const float m_new = (m_old != -INFINITY && m_hi - m_old <= kLazy) ? m_old : m_hi;
     float lsum = 0.f;
     uint32_t hi[8], lo[8];
 #pragma unroll
