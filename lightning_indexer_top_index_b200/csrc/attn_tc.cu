@@ -143,7 +143,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   // ---- 1. operands: `pass` 0 loads the window rows, pass 1 the selected rows
   // and zero-fills the empty ones
   auto load_rows = [&](int pass) {
-    if (!kFp8) {
+    if constexpr (!kFp8) {
       if (pass == 0 && tma_window) return;
       for (int r = warp; r < kRows; r += kThreads / 32) {
         const int kind = sm->row_kind[r];
@@ -158,41 +158,41 @@ __global__ void __launch_bounds__(kThreads, 2)
           *reinterpret_cast<uint4 *>(sX + x_off(r, lane + 32)) = make_uint4(0, 0, 0, 0);
         }
       }
-      return;
-    }
-    // RoPE dims [448, 512) as they are
-    for (int idx = tid; idx < kRows * 8; idx += kThreads) {
-      const int r = idx >> 3, c = 56 + (idx & 7);
-      const int kind = sm->row_kind[r];
-      if (pass == 0 ? kind != 2 : kind == 2) continue;
-      if (kind != 0) {
-        const lidx_kv &kv = kind == 1 ? a.kv : a.swa;
-        cp_async16(xs + x_off(r, c), static_cast<const uint16_t *>(kv.rope) + sm->row_src[r] * kv.ld_rope + (c - 56) * 8);
-      } else {
-        *reinterpret_cast<uint4 *>(sX + x_off(r, c)) = make_uint4(0, 0, 0, 0);
+    } else {
+      // RoPE dims [448, 512) as they are
+      for (int idx = tid; idx < kRows * 8; idx += kThreads) {
+        const int r = idx >> 3, c = 56 + (idx & 7);
+        const int kind = sm->row_kind[r];
+        if (pass == 0 ? kind != 2 : kind == 2) continue;
+        if (kind != 0) {
+          const lidx_kv &kv = kind == 1 ? a.kv : a.swa;
+          cp_async16(xs + x_off(r, c), static_cast<const uint16_t *>(kv.rope) + sm->row_src[r] * kv.ld_rope + (c - 56) * 8);
+        } else {
+          *reinterpret_cast<uint4 *>(sX + x_off(r, c)) = make_uint4(0, 0, 0, 0);
+        }
       }
-    }
-    // non-RoPE dims: 16 E4M3 codes per step, times their power-of-two block
-    // scale (exact while the product is a bf16 value)
-    for (int idx = tid; idx < kRows * 28; idx += kThreads) {
-      const int r = idx / 28, c16 = idx % 28;
-      const int kind = sm->row_kind[r];
-      if (pass == 0 ? kind != 2 : kind == 2) continue;
-      uint4 lo = make_uint4(0, 0, 0, 0), hi = lo;
-      if (kind != 0) {
-        const lidx_kv &kv = kind == 1 ? a.kv : a.swa;
-        const int64_t row = sm->row_src[r];
-        const uint4 x = __ldg(reinterpret_cast<const uint4 *>(static_cast<const uint8_t *>(kv.data) + row * kv.ld + c16 * 16));
-        const float sc = e8m0_to_f32(__ldg(kv.scale + row * kv.ld_scale + (c16 >> 2)));
-        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-        uint32_t o[8];
+      // non-RoPE dims: 16 E4M3 codes per step, times their power-of-two block
+      // scale (exact while the product is a bf16 value)
+      for (int idx = tid; idx < kRows * 28; idx += kThreads) {
+        const int r = idx / 28, c16 = idx % 28;
+        const int kind = sm->row_kind[r];
+        if (pass == 0 ? kind != 2 : kind == 2) continue;
+        uint4 lo = make_uint4(0, 0, 0, 0), hi = lo;
+        if (kind != 0) {
+          const lidx_kv &kv = kind == 1 ? a.kv : a.swa;
+          const int64_t row = sm->row_src[r];
+          const uint4 x = __ldg(reinterpret_cast<const uint4 *>(static_cast<const uint8_t *>(kv.data) + row * kv.ld + c16 * 16));
+          const float sc = e8m0_to_f32(__ldg(kv.scale + row * kv.ld_scale + (c16 >> 2)));
+          const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+          uint32_t o[8];
 #pragma unroll
-        for (int i = 0; i < 8; i++) o[i] = e4m3x2_to_bf16x2(w[i >> 1] >> (16 * (i & 1)), sc);
-        lo = make_uint4(o[0], o[1], o[2], o[3]);
-        hi = make_uint4(o[4], o[5], o[6], o[7]);
+          for (int i = 0; i < 8; i++) o[i] = e4m3x2_to_bf16x2(w[i >> 1] >> (16 * (i & 1)), sc);
+          lo = make_uint4(o[0], o[1], o[2], o[3]);
+          hi = make_uint4(o[4], o[5], o[6], o[7]);
+        }
+        *reinterpret_cast<uint4 *>(sX + x_off(r, 2 * c16)) = lo;
+        *reinterpret_cast<uint4 *>(sX + x_off(r, 2 * c16 + 1)) = hi;
       }
-      *reinterpret_cast<uint4 *>(sX + x_off(r, 2 * c16)) = lo;
-      *reinterpret_cast<uint4 *>(sX + x_off(r, 2 * c16 + 1)) = hi;
     }
   };
   load_rows(0);

@@ -233,8 +233,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::tc_fence_after();
         const uint32_t idesc = tc::idesc_bf16(64, 64);
         const uint32_t qs = tc::smem_u32(sQ);
-#pragma unroll
         const int part = warp - 4;
+#pragma unroll
         for (int kk = 0; kk < 32 / kS1; kk++) {
           const int k = part * (32 / kS1) + kk;
           const uint32_t off = (k >> 2) * kPanel + (k & 3) * 32;
